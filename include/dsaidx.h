@@ -1,0 +1,179 @@
+/*
+ * dsaidx.h — C ABI of the B200 (sm_100a) DSA lightning-indexer library.
+ *
+ * What the library computes (sources are the pages this project restates):
+ *
+ *   DSA indexer score.  H_I indexer query heads q_{t,j} (dimension d) share one
+ *   indexer key k_s per token; each head carries a weight w_{t,j}:
+ *       I_{t,s} = sum_j  w_{t,j} * ReLU(q_{t,j} . k_s)
+ *   Every query scans its whole causal prefix and keeps a token-level top-k
+ *   ("PaperTrace 2.2.2 MISA, LISA and ResMiSA", opening definition of the DSA
+ *   score and section 2.2 "kernel boundary"; "The new bottleneck of sparse
+ *   attention", section "level three: DeepSeek DSA").
+ *
+ *   MISA (head routing).  Pool keys into M = ceil(L/B) blocks, score each head
+ *   by E_{t,j} = (1/M) sum_b |w_{t,j} ReLU(q_{t,j} . k~_b)|, keep the top-h
+ *   heads, score every legal token with those heads only, take the top-k.
+ *   MISA-dagger keeps k' candidates from that pass and reranks them with all
+ *   H_I heads ("MISA: Mixture of Indexer Sparse Attention", method steps 1-6).
+ *
+ *   HISA (block -> token hierarchy).  Mean-pool keys into blocks of b tokens,
+ *   score the representatives with the same indexer query, keep the top-r
+ *   blocks and rerank only their tokens with the full formula
+ *   ("PaperTrace 2.2.2", section 2.1 "HISA"; "The new bottleneck of sparse
+ *   attention", section "route one: HISA").
+ *
+ * Conventions shared by every call
+ *   - All tensor pointers are DEVICE pointers, row-major, densely packed:
+ *       q      [batch, n_q, heads, dim]   dtype q_dtype
+ *       q_scale[batch, n_q]  fp32         required iff q_dtype == DSA_E4M3
+ *       k      [batch, n_k, dim]          dtype k_dtype
+ *       k_scale[batch, n_k]  fp32         required iff k_dtype == DSA_E4M3
+ *       w      [batch, n_q, heads] fp32
+ *       out_idx   [batch, n_q, topk] int32
+ *       out_score [batch, n_q, topk] fp32
+ *     bf16 is passed as raw 16-bit words, e4m3 as raw bytes (OCP FP8 E4M3).
+ *     The dequantised operand is scale * code; the scale of a key multiplies
+ *     its whole row, the scale of a query multiplies all heads of that query.
+ *   - Causality.  Query i of sequence b sits at position pos = q_pos0[b] + i
+ *     (q_pos0 == NULL: pos0 = n_k - n_q).  Its legal keys are
+ *     0 <= s <= pos and s < k_len[b] (k_len == NULL: n_k).
+ *   - Output contract.  Each query row receives min(topk, |legal|) entries
+ *     ordered by (score descending, index ascending) — the lower index wins a
+ *     tie — followed by padding (index -1, score -inf).  -0.0 is written as
+ *     +0.0.  The reported score is the one the final selection used: the full
+ *     I for dsa_index, misa_dagger_index and hisa_index (route_h == 0); the
+ *     routed-head score for misa_index and the stacked hisa_index.
+ *   - Memory.  The caller owns every buffer (inputs, outputs, workspace) and
+ *     the stream.  The library allocates no device memory, keeps no global
+ *     state between calls and never synchronises the stream unless
+ *     DSA_FLAG_CHECK is set.  Calls are asynchronous on `stream` (a
+ *     cudaStream_t passed as void*; NULL = the legacy default stream).  Two
+ *     calls in flight at once need two distinct workspaces.
+ *   - Errors.  Every call returns DSA_OK (0) or a negative status; nothing is
+ *     thrown across the ABI.  Argument errors are detected on the host before
+ *     any launch.  A bounded device wait that expires (DSA_ERR_TIMEOUT) or a
+ *     non-finite scale (DSA_ERR_NONFINITE, only checked under DSA_FLAG_CHECK)
+ *     is recorded in a status word inside the workspace; with DSA_FLAG_CHECK the
+ *     call synchronises the stream and returns it, otherwise
+ *     dsa_read_status() returns it after the caller synchronises.
+ *   - Supported shapes: dim == 128; heads a power of two in [8, 128];
+ *     topk in [1, 8192]; n_k <= 2^24.  Anything else returns
+ *     DSA_ERR_UNSUPPORTED.
+ */
+#ifndef DSAIDX_H
+#define DSAIDX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  DSA_OK = 0,
+  DSA_ERR_INVALID = -1,      /* null pointer, negative size, inconsistent shape */
+  DSA_ERR_UNSUPPORTED = -2,  /* dtype / dim / heads / topk outside the supported set */
+  DSA_ERR_WORKSPACE = -3,    /* workspace NULL or smaller than dsa_workspace_size() */
+  DSA_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
+  DSA_ERR_NONFINITE = -5,    /* a scale is NaN, inf, zero or negative (DSA_FLAG_CHECK) */
+  DSA_ERR_TIMEOUT = -6       /* a bounded device-side wait expired */
+};
+
+typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
+
+/* Algorithm ids for dsa_workspace_size(). */
+enum { DSA_ALGO_DSA = 0, DSA_ALGO_MISA = 1, DSA_ALGO_MISA_DAGGER = 2, DSA_ALGO_HISA = 3 };
+
+/* problem.flags */
+#define DSA_FLAG_CHECK 1u /* validate scales/lengths on device, synchronise, return device status */
+
+typedef struct {
+  int32_t batch;          /* sequences */
+  int32_t n_q;            /* query rows per sequence */
+  int32_t n_k;            /* key rows per sequence */
+  int32_t heads;          /* H_I */
+  int32_t dim;            /* indexer dimension d */
+  int32_t topk;           /* k */
+  int32_t q_dtype;        /* dsa_dtype */
+  int32_t k_dtype;        /* dsa_dtype; must equal q_dtype except (q BF16, k E4M3) */
+  const int32_t* q_pos0;  /* device [batch] or NULL */
+  const int32_t* k_len;   /* device [batch] or NULL */
+  uint32_t flags;
+} dsa_problem;
+
+/* Routing / hierarchy parameters (ignored fields may be zero).
+ *   misa_block  B  : tokens per pooled key of the MISA router (e.g. 1024)
+ *   misa_h      h  : routed heads kept per query (e.g. 8), 1 <= h <= heads
+ *   k_prime     k' : MISA-dagger candidate pool (e.g. 8192), k' >= topk
+ *   hisa_block  b  : tokens per HISA block (e.g. 64)
+ *   hisa_r      r  : HISA blocks kept per query (e.g. 128)
+ * Block sizes must be powers of two in [16, 4096]. */
+typedef struct {
+  int32_t misa_block;
+  int32_t misa_h;
+  int32_t k_prime;
+  int32_t hisa_block;
+  int32_t hisa_r;
+} dsa_route_params;
+
+/* Bytes of device workspace that `algo` needs for problem `p` (route params
+ * may be NULL for DSA_ALGO_DSA).  Writes *bytes; returns a status. */
+int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
+                       size_t* bytes);
+
+/* DSA lightning-indexer top-k: score -> causal mask -> token top-k. */
+int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+              const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
+              void* workspace, size_t workspace_bytes, void* stream);
+
+/* MISA: block-pooled router picks rp->misa_h heads per query, those heads score
+ * every legal token, token top-k.  out_heads [batch,n_q,h] int32 (ascending head
+ * order) and out_E [batch,n_q,heads] fp32 (the router importance E) are optional
+ * (NULL skips them).  Supports q_dtype == k_dtype in {F32, BF16}. */
+int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
+               const void* k, const float* w, int32_t* out_idx, float* out_score,
+               int32_t* out_heads, float* out_E, void* workspace, size_t workspace_bytes,
+               void* stream);
+
+/* MISA-dagger: the MISA pass keeps rp->k_prime candidates, which are reranked
+ * by the full H_I-head score; final token top-k.  out_heads as for misa_index;
+ * out_pool [batch,n_q,k_prime] int32 (optional) receives the first-pass pool
+ * (unordered, padded with -1). */
+int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
+                      const void* k, const float* w, int32_t* out_idx, float* out_score,
+                      int32_t* out_heads, int32_t* out_pool, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/* HISA: score block representatives (blocks of rp->hisa_block tokens), keep
+ * rp->hisa_r blocks, rerank their legal tokens, token top-k.  With
+ * rp->misa_h > 0 the MISA router (rp->misa_block) first picks misa_h heads and
+ * both HISA stages use only those heads (the stacked variant).  out_blocks
+ * [batch,n_q,r] int32 (optional) receives the kept block ids (unordered,
+ * padded with -1); out_heads [batch,n_q,h] (optional, stacked only). */
+int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
+               const void* k, const float* w, int32_t* out_idx, float* out_score,
+               int32_t* out_blocks, int32_t* out_heads, void* workspace,
+               size_t workspace_bytes, void* stream);
+
+/* Operand preparation for the FP8 path: per-row scale a = amax/448 (amax == 0
+ * gives a = 1), code = round-to-nearest-even, saturating e4m3 of x/a, both
+ * divisions in IEEE fp32 ("PaperTrace 2.2.2", section 2.3 "from formula to
+ * FP8 cache": k^ = round(k/a), FP8 data plus a scale).
+ *   x [rows, cols] (x_dtype F32 or BF16), out [rows, cols] uint8, out_scale [rows]. */
+int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols,
+                      uint8_t* out, float* out_scale, void* stream);
+
+/* Device status word recorded in `workspace` by the last call that used it
+ * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_NONFINITE).  Synchronises `stream`. */
+int dsa_read_status(const void* workspace, void* stream);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* dsa_status_string(int32_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSAIDX_H */

@@ -1,0 +1,603 @@
+/*
+ * dsa_oracle.c — plain, slow CPU definition of the DSA lightning indexer and
+ * its MISA / MISA-dagger / HISA reductions.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path calls this code: only
+ * the tests, the package's smoke check and the benchmark's CPU-baseline leg
+ * load it.  It shares no code, header, table or constant with the CUDA library.
+ *
+ * Every quantity is the definition written out: operands are decoded to their
+ * exact values, every dot product and head sum is accumulated in fp64 in
+ * ascending index order, every selection is a full sort by the total order
+ * (score descending, index ascending), and the final scores are rounded once
+ * from fp64 to fp32 (nearest-even; -0.0 written as +0.0).  OpenMP only spreads
+ * independent query rows over cores.
+ *
+ * Sources (page titles and sections):
+ *  [DSA]  "PaperTrace 2.2.2 MISA, LISA and ResMiSA": the DSA score that opens
+ *         the page (H_I heads share the history key k_s; query head q_{t,j}
+ *         with weight w_{t,j}); section 2.2 "kernel boundary" (score, causal
+ *         mask, top-k fused); section 2.3 "end-to-end acceptance" (explicit
+ *         formula, causal mask, stable-sort top-k on small tensors).
+ *  [MISA] "MISA: Mixture of Indexer Sparse Attention" summary, method steps
+ *         1-6: pool the prefix into M = ceil(L/B) blocks, A_{t,j,b} =
+ *         w_{t,j} ReLU(q_{t,j} . k~_b), E_{t,j} = (1/M) sum_b |A_{t,j,b}|,
+ *         top-h heads, I^_{t,s} over the routed heads, top-k; MISA-dagger runs
+ *         steps 4-5 twice, the second time with all H_I heads on k' candidates.
+ *  [HISA] "PaperTrace 2.2.2", section 2.1 "HISA: filter blocks, then rerank
+ *         tokens with the original formula"; "The new bottleneck of sparse
+ *         attention", route one: HISA (mean-pooled block keys scored with the
+ *         same indexer query, top blocks kept, DSA indexer run on their tokens).
+ *  [FP8]  "PaperTrace 2.2.2", section 2.3 "from formula to FP8 cache":
+ *         k^ = round(k/a), FP8 data plus scale, higher-precision accumulation.
+ *         The e4m3 code follows the OCP 8-bit floating point specification
+ *         (E4M3: bias 7, no infinities, S.1111.111 is NaN, max 448).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *  - The key is shared by all heads; the head subscript on k in the MISA
+ *    summary's step 4 is read as a typo.
+ *  - Query i of sequence b sits at position pos = q_pos0[b] + i; its legal
+ *    keys are 0 <= s <= pos and s < k_len[b] (self-inclusive causal mask).
+ *  - Rows with fewer than k legal keys return all of them, then (-1, -inf).
+ *  - Ties: lower token index, lower head index, lower block index wins.
+ *  - Blocks cover the legal prefix only; the block holding pos is the mean of
+ *    its legal tokens.  A representative is the exact mean rounded once to the
+ *    key storage type (bf16 or fp32).
+ *  - MISA ranks heads by the un-normalised sum S_{t,j} = M_t E_{t,j}; the
+ *    order is the same and E is reported as S / M_t.
+ *  - HISA scores a block with the DSA formula on its representative
+ *    (weights keep their sign, no absolute value).
+ *  - Stacked MISA + HISA: the routed heads are used in both HISA stages.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2 };
+enum { ORC_OK = 0, ORC_ERR = -1 };
+
+typedef struct {
+  int32_t batch, n_q, n_k, heads, dim;
+  int32_t q_dtype, k_dtype;
+  const int32_t* q_pos0; /* [batch] or NULL: n_k - n_q */
+  const int32_t* k_len;  /* [batch] or NULL: n_k */
+  const void* q;         /* [batch,n_q,heads,dim] */
+  const float* q_scale;  /* [batch,n_q] (e4m3 only) */
+  const void* k;         /* [batch,n_k,dim] */
+  const float* k_scale;  /* [batch,n_k] (e4m3 only) */
+  const float* w;        /* [batch,n_q,heads] */
+} orc_inputs;
+
+/* ---------------------------------------------------------------- codecs -- */
+
+/* OCP E4M3 decode: sign bit, 4 exponent bits (bias 7), 3 mantissa bits.
+ * Exponent field 0 is subnormal (m * 2^-9); S.1111.111 is NaN. */
+double orc_e4m3_decode(uint8_t c) {
+  int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+  double v;
+  if (e == 15 && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);
+  else
+    v = ldexp((double)(8 + m), e - 10);
+  return sign ? -v : v;
+}
+
+/* Round-to-nearest-even, saturating OCP E4M3 encode of an fp32 value.
+ * The representable magnitudes are m * 2^-9 (m = 0..7, subnormal) and
+ * (8 + m) * 2^(e-10) for e = 1..15 (excluding e = 15, m = 7).  Values at or
+ * beyond the largest finite magnitude 448 saturate to 448. */
+uint8_t orc_e4m3_encode(float x) {
+  double v = (double)x;
+  uint8_t sign = signbit(x) ? 0x80 : 0;
+  double a = fabs(v);
+  if (isnan(x)) return 0x7F;
+  if (a >= 448.0) return sign | 0x7E;
+  /* exponent e of the binade [2^(e-7), 2^(e-6)) holding a; subnormals use e = 1 spacing */
+  int ex;
+  frexp(a, &ex); /* a = f * 2^ex, f in [0.5, 1) => binade exponent ex-1 */
+  int E = ex - 1; /* a in [2^E, 2^(E+1)) */
+  if (a == 0.0) return sign;
+  if (E < -6) E = -6; /* subnormal range shares the spacing of the first binade */
+  double ulp = ldexp(1.0, E - 3);
+  double n = a / ulp; /* exact: scaling by a power of two */
+  double fl = floor(n);
+  double r = n - fl;
+  double m_int = fl;
+  if (r > 0.5 || (r == 0.5 && fmod(fl, 2.0) != 0.0)) m_int = fl + 1.0;
+  double q = m_int * ulp; /* rounded magnitude */
+  if (q >= 448.0) return sign | 0x7E;
+  if (q == 0.0) return sign;
+  /* re-derive the code from the rounded magnitude */
+  frexp(q, &ex);
+  E = ex - 1;
+  if (E < -6) { /* subnormal */
+    int mm = (int)(q / ldexp(1.0, -9));
+    return sign | (uint8_t)mm;
+  }
+  int mm = (int)(q / ldexp(1.0, E - 3)) - 8;
+  return sign | (uint8_t)(((E + 7) << 3) | mm);
+}
+
+/* Operand preparation: per-row scale a = amax / 448 in fp32 (amax == 0 gives
+ * a = 1), code = e4m3(x / a) with the division in fp32.  [FP8] */
+int orc_quantize_rows(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* out,
+                      float* out_scale) {
+  if (x_dtype != ORC_F32 && x_dtype != ORC_BF16) return ORC_ERR;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    float amax = 0.0f;
+    for (int32_t c = 0; c < cols; ++c) {
+      float v;
+      if (x_dtype == ORC_F32) {
+        v = ((const float*)x)[r * cols + c];
+      } else {
+        uint32_t b = (uint32_t)((const uint16_t*)x)[r * cols + c] << 16;
+        memcpy(&v, &b, 4);
+      }
+      float av = fabsf(v);
+      if (av > amax) amax = av;
+    }
+    volatile float a = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+    out_scale[r] = a;
+    for (int32_t c = 0; c < cols; ++c) {
+      float v;
+      if (x_dtype == ORC_F32) {
+        v = ((const float*)x)[r * cols + c];
+      } else {
+        uint32_t b = (uint32_t)((const uint16_t*)x)[r * cols + c] << 16;
+        memcpy(&v, &b, 4);
+      }
+      volatile float t = v / a;
+      out[r * cols + c] = orc_e4m3_encode(t);
+    }
+  }
+  return ORC_OK;
+}
+
+/* Nearest-even rounding of an exact fp64 value to bf16 (returned as double). */
+static double round_to_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  double a = fabs(x);
+  int ex;
+  frexp(a, &ex);
+  int E = ex - 1;
+  if (E < -126) E = -126;              /* subnormal spacing 2^-133 */
+  double ulp = ldexp(1.0, E - 7);      /* 8 significant bits */
+  double n = a / ulp, fl = floor(n), r = n - fl, m = fl;
+  if (r > 0.5 || (r == 0.5 && fmod(fl, 2.0) != 0.0)) m = fl + 1.0;
+  double q = m * ulp;
+  return x < 0 ? -q : q;
+}
+
+/* ------------------------------------------------------------- operands -- */
+
+static double bf16_value(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+static double q_val(const orc_inputs* in, int64_t row, int32_t j, int32_t c) {
+  int64_t off = (row * in->heads + j) * (int64_t)in->dim + c;
+  switch (in->q_dtype) {
+    case ORC_F32: return (double)((const float*)in->q)[off];
+    case ORC_BF16: return bf16_value(((const uint16_t*)in->q)[off]);
+    default: return (double)in->q_scale[row] * orc_e4m3_decode(((const uint8_t*)in->q)[off]);
+  }
+}
+
+static double k_val(const orc_inputs* in, int32_t b, int64_t s, int32_t c) {
+  int64_t kr = (int64_t)b * in->n_k + s;
+  int64_t off = kr * in->dim + c;
+  switch (in->k_dtype) {
+    case ORC_F32: return (double)((const float*)in->k)[off];
+    case ORC_BF16: return bf16_value(((const uint16_t*)in->k)[off]);
+    default: return (double)in->k_scale[kr] * orc_e4m3_decode(((const uint8_t*)in->k)[off]);
+  }
+}
+
+static int32_t row_pos(const orc_inputs* in, int64_t row) {
+  int32_t b = (int32_t)(row / in->n_q), i = (int32_t)(row % in->n_q);
+  int32_t p0 = in->q_pos0 ? in->q_pos0[b] : in->n_k - in->n_q;
+  return p0 + i;
+}
+
+/* Number of legal keys of a row: s <= pos and s < k_len. */
+static int64_t row_legal(const orc_inputs* in, int64_t row) {
+  int32_t b = (int32_t)(row / in->n_q);
+  int64_t kl = in->k_len ? in->k_len[b] : in->n_k;
+  int64_t n = (int64_t)row_pos(in, row) + 1;
+  if (n > kl) n = kl;
+  return n < 0 ? 0 : n;
+}
+
+/* q_{t,j} . x for an explicit d-vector x (fp64). */
+static double dot_q_vec(const orc_inputs* in, int64_t row, int32_t j, const double* x) {
+  double acc = 0.0;
+  for (int32_t c = 0; c < in->dim; ++c) acc += q_val(in, row, j, c) * x[c];
+  return acc;
+}
+
+/* [DSA] I_{t,s} restricted to the listed heads (ascending): sum_j w_{t,j} max(q_{t,j}.k_s, 0). */
+static double score_heads(const orc_inputs* in, int64_t row, int64_t s, const int32_t* heads,
+                          int32_t nh) {
+  int32_t b = (int32_t)(row / in->n_q);
+  double total = 0.0;
+  for (int32_t a = 0; a < nh; ++a) {
+    int32_t j = heads[a];
+    double z = 0.0;
+    for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * k_val(in, b, s, c);
+    total += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+  }
+  return total;
+}
+
+/* --------------------------------------------------------------- ranking -- */
+
+typedef struct {
+  double v;
+  int64_t i;
+} ranked;
+
+/* Total order: value descending, index ascending ("stable sort", lower index wins). */
+static int by_value_then_index(const void* a, const void* b) {
+  const ranked* x = (const ranked*)a;
+  const ranked* y = (const ranked*)b;
+  if (x->v > y->v) return -1;
+  if (x->v < y->v) return 1;
+  return (x->i > y->i) - (x->i < y->i);
+}
+
+static float to_output_score(double v) {
+  float f = (float)v;
+  return f == 0.0f ? 0.0f : f; /* -0.0 -> +0.0 */
+}
+
+/* Write the first min(k, n) ranked entries then (-1, -inf) padding. */
+static void emit_topk(const ranked* r, int64_t n, int32_t topk, int32_t* idx, float* sc,
+                      double* sc64) {
+  for (int32_t a = 0; a < topk; ++a) {
+    if (a < n) {
+      idx[a] = (int32_t)r[a].i;
+      sc[a] = to_output_score(r[a].v);
+      if (sc64) sc64[a] = r[a].v;
+    } else {
+      idx[a] = -1;
+      sc[a] = -INFINITY;
+      if (sc64) sc64[a] = -INFINITY;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------ DSA -- */
+
+/* [DSA] Exact top-k of I_{t,s} over the legal prefix, for the listed rows.
+ * out_dots[r] = H * |legal| (the indexer's low-dimensional dot products). */
+int orc_dsa_rows(const orc_inputs* in, int32_t topk, const int64_t* rows, int64_t n_rows,
+                 int32_t* out_idx, float* out_score, double* out_score64, int64_t* out_dots) {
+  int32_t* all = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+  for (int32_t j = 0; j < in->heads; ++j) all[j] = j;
+  int err = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t row = rows[r];
+    int64_t n = row_legal(in, row);
+    ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    if (!cand) { err = 1; continue; }
+    for (int64_t s = 0; s < n; ++s) {
+      cand[s].v = score_heads(in, row, s, all, in->heads);
+      cand[s].i = s;
+    }
+    qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
+    emit_topk(cand, n, topk, out_idx + r * topk, out_score + r * topk,
+              out_score64 ? out_score64 + r * topk : NULL);
+    if (out_dots) out_dots[r] = (int64_t)in->heads * n;
+    free(cand);
+  }
+  free(all);
+  return err ? ORC_ERR : ORC_OK;
+}
+
+/* fp64 scores at explicit (row, s) pairs; heads == NULL means all heads,
+ * otherwise heads is [n, nh] (one head list per pair). */
+int orc_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                    const int32_t* heads, int32_t nh, double* out) {
+  int32_t* all = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+  for (int32_t j = 0; j < in->heads; ++j) all[j] = j;
+#pragma omp parallel for schedule(static)
+  for (int64_t a = 0; a < n; ++a) {
+    if (heads)
+      out[a] = score_heads(in, rows[a], s[a], heads + a * nh, nh);
+    else
+      out[a] = score_heads(in, rows[a], s[a], all, in->heads);
+  }
+  free(all);
+  return ORC_OK;
+}
+
+/* Typical score magnitude at (row, s): sum_j |w_{t,j}| ||q_{t,j}|| ||k_s|| / sqrt(d).
+ * Used by the tests as the denominator of the relative score tolerance. */
+int orc_score_scale_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                          double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t a = 0; a < n; ++a) {
+    int64_t row = rows[a];
+    int32_t b = (int32_t)(row / in->n_q);
+    double kn = 0.0;
+    for (int32_t c = 0; c < in->dim; ++c) {
+      double v = k_val(in, b, s[a], c);
+      kn += v * v;
+    }
+    double acc = 0.0;
+    for (int32_t j = 0; j < in->heads; ++j) {
+      double qn = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) {
+        double v = q_val(in, row, j, c);
+        qn += v * v;
+      }
+      acc += fabs((double)in->w[row * in->heads + j]) * sqrt(qn);
+    }
+    out[a] = acc * sqrt(kn) / sqrt((double)in->dim);
+  }
+  return ORC_OK;
+}
+
+/* -------------------------------------------------------------- pooling -- */
+
+/* Mean of key rows [lo, hi) of sequence b, rounded once to the key storage
+ * type (bf16 or fp32).  [MISA] step 1 / [HISA] block representatives. */
+static void pooled_key(const orc_inputs* in, int32_t b, int64_t lo, int64_t hi, double* out) {
+  for (int32_t c = 0; c < in->dim; ++c) {
+    double sum = 0.0;
+    for (int64_t s = lo; s < hi; ++s) sum += k_val(in, b, s, c);
+    double mean = sum / (double)(hi - lo);
+    out[c] = (in->k_dtype == ORC_BF16) ? round_to_bf16(mean) : (double)(float)mean;
+  }
+}
+
+/* Representatives of the ceil(n/blk) blocks of the legal prefix [0, n). */
+static double* block_representatives(const orc_inputs* in, int32_t b, int64_t n, int32_t blk,
+                                     int64_t* n_blocks) {
+  int64_t m = (n + blk - 1) / blk;
+  double* reps = (double*)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1) * in->dim);
+  for (int64_t a = 0; a < m; ++a) {
+    int64_t lo = a * blk, hi = lo + blk < n ? lo + blk : n;
+    pooled_key(in, b, lo, hi, reps + a * in->dim);
+  }
+  *n_blocks = m;
+  return reps;
+}
+
+/* Exported for tests: representatives of sequence b's prefix [0, n). */
+int orc_pool(const orc_inputs* in, int32_t b, int64_t n, int32_t blk, double* out) {
+  int64_t m;
+  double* reps = block_representatives(in, b, n, blk, &m);
+  memcpy(out, reps, sizeof(double) * (size_t)m * in->dim);
+  free(reps);
+  return ORC_OK;
+}
+
+/* [MISA] steps 1-3 for one row: S_{t,j} = sum_b |w_{t,j}| max(q_{t,j}.k~_b, 0)
+ * over the M_t blocks of the legal prefix; the top-h heads by (S desc, j asc)
+ * are returned in ascending head order. */
+static void misa_route(const orc_inputs* in, int64_t row, int32_t blk, int32_t h, double* S,
+                       int32_t* heads_out, int64_t* m_out) {
+  int32_t b = (int32_t)(row / in->n_q);
+  int64_t n = row_legal(in, row), m;
+  double* reps = block_representatives(in, b, n, blk, &m);
+  ranked* order = (ranked*)malloc(sizeof(ranked) * in->heads);
+  for (int32_t j = 0; j < in->heads; ++j) {
+    double s = 0.0;
+    double aw = fabs((double)in->w[row * in->heads + j]);
+    for (int64_t a = 0; a < m; ++a) {
+      double z = dot_q_vec(in, row, j, reps + a * in->dim);
+      s += aw * (z > 0.0 ? z : 0.0);
+    }
+    S[j] = s;
+    order[j].v = s;
+    order[j].i = j;
+  }
+  qsort(order, (size_t)in->heads, sizeof(ranked), by_value_then_index);
+  /* ascending head order of the selected set */
+  char* chosen = (char*)calloc((size_t)in->heads, 1);
+  for (int32_t a = 0; a < h; ++a) chosen[order[a].i] = 1;
+  int32_t c = 0;
+  for (int32_t j = 0; j < in->heads; ++j)
+    if (chosen[j]) heads_out[c++] = j;
+  free(chosen);
+  free(order);
+  free(reps);
+  *m_out = m;
+}
+
+static int cmp_i32(const void* a, const void* b) {
+  int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+
+/* [MISA] MISA (k_prime == 0) and MISA-dagger (k_prime > 0) for the listed rows.
+ *  forced_heads [n_rows, h]  : use these heads instead of the router's (conditional parity)
+ *  forced_pool  [n_rows, k'] : use this first-pass pool (entries < 0 ignored)
+ * Outputs (optional ones may be NULL):
+ *  out_idx/out_score/out_score64 [n_rows, topk]; out_heads [n_rows, h] ascending;
+ *  out_E [n_rows, H] = S / M_t; out_pool [n_rows, k'] (pool in rank order, -1 padded);
+ *  out_dots [n_rows] = H*M_t + h*|legal| (+ H*min(k', |legal|) for MISA-dagger). */
+int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, int32_t k_prime,
+                  const int64_t* rows, int64_t n_rows, const int32_t* forced_heads,
+                  const int32_t* forced_pool, int32_t* out_idx, float* out_score,
+                  double* out_score64, int32_t* out_heads, double* out_E, int32_t* out_pool,
+                  int64_t* out_dots) {
+  if (in->k_dtype == ORC_E4M3 || h < 1 || h > in->heads || blk < 1) return ORC_ERR;
+  int32_t* all = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+  for (int32_t j = 0; j < in->heads; ++j) all[j] = j;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t row = rows[r];
+    int64_t n = row_legal(in, row), m = 0;
+    double* S = (double*)malloc(sizeof(double) * in->heads);
+    int32_t* heads = (int32_t*)malloc(sizeof(int32_t) * h);
+    misa_route(in, row, blk, h, S, heads, &m);
+    if (forced_heads) {
+      memcpy(heads, forced_heads + r * h, sizeof(int32_t) * h);
+      qsort(heads, (size_t)h, sizeof(int32_t), cmp_i32);
+    }
+    if (out_heads) memcpy(out_heads + r * h, heads, sizeof(int32_t) * h);
+    if (out_E)
+      for (int32_t j = 0; j < in->heads; ++j) out_E[r * in->heads + j] = m > 0 ? S[j] / (double)m : 0.0;
+    /* step 4: routed-head score over every legal token */
+    ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    for (int64_t s = 0; s < n; ++s) {
+      cand[s].v = score_heads(in, row, s, heads, h);
+      cand[s].i = s;
+    }
+    qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
+    int64_t dots = (int64_t)in->heads * m + (int64_t)h * n;
+    if (k_prime <= 0) {
+      emit_topk(cand, n, topk, out_idx + r * topk, out_score + r * topk,
+                out_score64 ? out_score64 + r * topk : NULL);
+    } else {
+      /* MISA-dagger: keep k' by the routed score, rerank with all heads */
+      int64_t np = n < k_prime ? n : k_prime;
+      ranked* pool = (ranked*)malloc(sizeof(ranked) * (np > 0 ? np : 1));
+      int64_t cnt = 0;
+      if (forced_pool) {
+        for (int32_t a = 0; a < k_prime; ++a) {
+          int32_t s = forced_pool[r * k_prime + a];
+          if (s >= 0 && cnt < np) pool[cnt++].i = s;
+        }
+      } else {
+        for (int64_t a = 0; a < np; ++a) pool[cnt++].i = cand[a].i;
+      }
+      if (out_pool)
+        for (int32_t a = 0; a < k_prime; ++a)
+          out_pool[r * k_prime + a] = a < cnt ? (int32_t)pool[a].i : -1;
+      for (int64_t a = 0; a < cnt; ++a) pool[a].v = score_heads(in, row, pool[a].i, all, in->heads);
+      qsort(pool, (size_t)cnt, sizeof(ranked), by_value_then_index);
+      emit_topk(pool, cnt, topk, out_idx + r * topk, out_score + r * topk,
+                out_score64 ? out_score64 + r * topk : NULL);
+      dots += (int64_t)in->heads * cnt;
+      free(pool);
+    }
+    if (out_dots) out_dots[r] = dots;
+    free(cand);
+    free(heads);
+    free(S);
+  }
+  free(all);
+  return ORC_OK;
+}
+
+/* [HISA] (route_h == 0) and stacked MISA + HISA (route_h > 0) for the listed rows.
+ *  1. (stacked) MISA router with block route_blk picks route_h heads;
+ *  2. blocks of blk tokens over the legal prefix, representatives as in MISA;
+ *     J_{t,b} = sum_{j in heads} w_{t,j} max(q_{t,j}.k~_b, 0);
+ *  3. keep the top-r blocks by (J desc, b asc)  (or forced_blocks [n_rows, r]);
+ *  4. score the legal tokens of the kept blocks with the same heads; top-k.
+ *  out_blocks [n_rows, r] kept blocks in rank order (-1 padded); out_J [n_rows, r]
+ *  their scores; out_dots = (H*M_t) + |heads|*M^b_t + |heads|*|candidates|. */
+int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_keep,
+                  int32_t route_h, int32_t route_blk, const int64_t* rows, int64_t n_rows,
+                  const int32_t* forced_heads, const int32_t* forced_blocks, int32_t* out_idx,
+                  float* out_score, double* out_score64, int32_t* out_blocks, double* out_J,
+                  int32_t* out_heads, int64_t* out_dots) {
+  if (in->k_dtype == ORC_E4M3 || blk < 1 || r_keep < 1) return ORC_ERR;
+  if (route_h < 0 || route_h > in->heads) return ORC_ERR;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t row = rows[r];
+    int32_t b = (int32_t)(row / in->n_q);
+    int64_t n = row_legal(in, row);
+    int32_t nh = route_h > 0 ? route_h : in->heads;
+    int32_t* heads = (int32_t*)malloc(sizeof(int32_t) * nh);
+    int64_t dots = 0;
+    if (route_h > 0) {
+      double* S = (double*)malloc(sizeof(double) * in->heads);
+      int64_t m = 0;
+      misa_route(in, row, route_blk, route_h, S, heads, &m);
+      dots += (int64_t)in->heads * m;
+      free(S);
+      if (forced_heads) {
+        memcpy(heads, forced_heads + r * nh, sizeof(int32_t) * nh);
+        qsort(heads, (size_t)nh, sizeof(int32_t), cmp_i32);
+      }
+      if (out_heads) memcpy(out_heads + r * nh, heads, sizeof(int32_t) * nh);
+    } else {
+      for (int32_t j = 0; j < nh; ++j) heads[j] = j;
+    }
+    /* coarse stage: block scores */
+    int64_t mb = 0;
+    double* reps = block_representatives(in, b, n, blk, &mb);
+    ranked* bl = (ranked*)malloc(sizeof(ranked) * (mb > 0 ? mb : 1));
+    for (int64_t a = 0; a < mb; ++a) {
+      double J = 0.0;
+      for (int32_t x = 0; x < nh; ++x) {
+        int32_t j = heads[x];
+        double z = dot_q_vec(in, row, j, reps + a * in->dim);
+        J += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+      }
+      bl[a].v = J;
+      bl[a].i = a;
+    }
+    dots += (int64_t)nh * mb;
+    qsort(bl, (size_t)mb, sizeof(ranked), by_value_then_index);
+    int64_t kept = mb < r_keep ? mb : r_keep;
+    char* keep = (char*)calloc((size_t)(mb > 0 ? mb : 1), 1);
+    if (forced_blocks) {
+      kept = 0;
+      for (int32_t a = 0; a < r_keep; ++a) {
+        int32_t x = forced_blocks[r * r_keep + a];
+        if (x >= 0 && x < mb && !keep[x]) { keep[x] = 1; ++kept; }
+      }
+    } else {
+      for (int64_t a = 0; a < kept; ++a) keep[bl[a].i] = 1;
+    }
+    if (out_blocks || out_J) {
+      for (int32_t a = 0; a < r_keep; ++a) {
+        int in_range = !forced_blocks && a < kept;
+        if (out_blocks) out_blocks[r * r_keep + a] = in_range ? (int32_t)bl[a].i : -1;
+        if (out_J) out_J[r * r_keep + a] = in_range ? bl[a].v : -INFINITY;
+      }
+    }
+    /* fine stage: the DSA formula on the kept blocks' legal tokens */
+    ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    int64_t nc = 0;
+    for (int64_t s = 0; s < n; ++s) {
+      if (!keep[s / blk]) continue;
+      cand[nc].v = score_heads(in, row, s, heads, nh);
+      cand[nc].i = s;
+      ++nc;
+    }
+    dots += (int64_t)nh * nc;
+    qsort(cand, (size_t)nc, sizeof(ranked), by_value_then_index);
+    emit_topk(cand, nc, topk, out_idx + r * topk, out_score + r * topk,
+              out_score64 ? out_score64 + r * topk : NULL);
+    if (out_dots) out_dots[r] = dots;
+    free(cand);
+    free(keep);
+    free(bl);
+    free(reps);
+    free(heads);
+  }
+  return ORC_OK;
+}
+
+/* Full fp64 score row (all legal s) of one query row for the listed heads
+ * (NULL = all); returns |legal|.  Used by tests for margins and tie checks. */
+int64_t orc_score_row(const orc_inputs* in, int64_t row, const int32_t* heads, int32_t nh,
+                      double* out) {
+  int64_t n = row_legal(in, row);
+  int32_t* all = NULL;
+  if (!heads) {
+    all = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+    for (int32_t j = 0; j < in->heads; ++j) all[j] = j;
+    heads = all;
+    nh = in->heads;
+  }
+#pragma omp parallel for schedule(static)
+  for (int64_t s = 0; s < n; ++s) out[s] = score_heads(in, row, s, heads, nh);
+  free(all);
+  return n;
+}
