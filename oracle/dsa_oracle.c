@@ -221,15 +221,56 @@ static double dot_q_vec(const orc_inputs* in, int64_t row, int32_t j, const doub
   return acc;
 }
 
-/* [DSA] I_{t,s} restricted to the listed heads (ascending): sum_j w_{t,j} max(q_{t,j}.k_s, 0). */
+/* [DSA] I_{t,s} restricted to the listed heads (ascending): sum_j w_{t,j} max(q_{t,j}.k_s, 0).
+ * The query row and the key are decoded to fp64 once; each head's dot product
+ * runs over c ascending and the head sum over the listed order. */
 static double score_heads(const orc_inputs* in, int64_t row, int64_t s, const int32_t* heads,
                           int32_t nh) {
   int32_t b = (int32_t)(row / in->n_q);
+  double* kd = (double*)malloc(sizeof(double) * in->dim);
+  for (int32_t c = 0; c < in->dim; ++c) kd[c] = k_val(in, b, s, c);
   double total = 0.0;
   for (int32_t a = 0; a < nh; ++a) {
     int32_t j = heads[a];
     double z = 0.0;
-    for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * k_val(in, b, s, c);
+    for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * kd[c];
+    total += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+  }
+  free(kd);
+  return total;
+}
+
+/* Decoded operands of one query row, reused across all its keys. */
+typedef struct {
+  double* q; /* [heads, dim] */
+  double* kd; /* [dim] scratch */
+} row_cache;
+
+static row_cache row_cache_new(const orc_inputs* in, int64_t row) {
+  row_cache rc;
+  rc.q = (double*)malloc(sizeof(double) * (size_t)in->heads * in->dim);
+  rc.kd = (double*)malloc(sizeof(double) * in->dim);
+  for (int32_t j = 0; j < in->heads; ++j)
+    for (int32_t c = 0; c < in->dim; ++c) rc.q[(size_t)j * in->dim + c] = q_val(in, row, j, c);
+  return rc;
+}
+
+static void row_cache_free(row_cache* rc) {
+  free(rc->q);
+  free(rc->kd);
+}
+
+/* Same value as score_heads, reading the decoded query row from the cache. */
+static double score_cached(const orc_inputs* in, row_cache* rc, int64_t row, int64_t s,
+                           const int32_t* heads, int32_t nh) {
+  int32_t b = (int32_t)(row / in->n_q);
+  for (int32_t c = 0; c < in->dim; ++c) rc->kd[c] = k_val(in, b, s, c);
+  double total = 0.0;
+  for (int32_t a = 0; a < nh; ++a) {
+    int32_t j = heads[a];
+    const double* qj = rc->q + (size_t)j * in->dim;
+    double z = 0.0;
+    for (int32_t c = 0; c < in->dim; ++c) z += qj[c] * rc->kd[c];
     total += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
   }
   return total;
@@ -287,10 +328,12 @@ int orc_dsa_rows(const orc_inputs* in, int32_t topk, const int64_t* rows, int64_
     int64_t n = row_legal(in, row);
     ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
     if (!cand) { err = 1; continue; }
+    row_cache rc = row_cache_new(in, row);
     for (int64_t s = 0; s < n; ++s) {
-      cand[s].v = score_heads(in, row, s, all, in->heads);
+      cand[s].v = score_cached(in, &rc, row, s, all, in->heads);
       cand[s].i = s;
     }
+    row_cache_free(&rc);
     qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
     emit_topk(cand, n, topk, out_idx + r * topk, out_score + r * topk,
               out_score64 ? out_score64 + r * topk : NULL);
@@ -449,8 +492,9 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
       for (int32_t j = 0; j < in->heads; ++j) out_E[r * in->heads + j] = m > 0 ? S[j] / (double)m : 0.0;
     /* step 4: routed-head score over every legal token */
     ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    row_cache rc = row_cache_new(in, row);
     for (int64_t s = 0; s < n; ++s) {
-      cand[s].v = score_heads(in, row, s, heads, h);
+      cand[s].v = score_cached(in, &rc, row, s, heads, h);
       cand[s].i = s;
     }
     qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
@@ -474,7 +518,8 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
       if (out_pool)
         for (int32_t a = 0; a < k_prime; ++a)
           out_pool[r * k_prime + a] = a < cnt ? (int32_t)pool[a].i : -1;
-      for (int64_t a = 0; a < cnt; ++a) pool[a].v = score_heads(in, row, pool[a].i, all, in->heads);
+      for (int64_t a = 0; a < cnt; ++a)
+        pool[a].v = score_cached(in, &rc, row, pool[a].i, all, in->heads);
       qsort(pool, (size_t)cnt, sizeof(ranked), by_value_then_index);
       emit_topk(pool, cnt, topk, out_idx + r * topk, out_score + r * topk,
                 out_score64 ? out_score64 + r * topk : NULL);
@@ -482,6 +527,7 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
       free(pool);
     }
     if (out_dots) out_dots[r] = dots;
+    row_cache_free(&rc);
     free(cand);
     free(heads);
     free(S);
@@ -564,9 +610,10 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
     /* fine stage: the DSA formula on the kept blocks' legal tokens */
     ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
     int64_t nc = 0;
+    row_cache rc = row_cache_new(in, row);
     for (int64_t s = 0; s < n; ++s) {
       if (!keep[s / blk]) continue;
-      cand[nc].v = score_heads(in, row, s, heads, nh);
+      cand[nc].v = score_cached(in, &rc, row, s, heads, nh);
       cand[nc].i = s;
       ++nc;
     }
@@ -575,6 +622,7 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
     emit_topk(cand, nc, topk, out_idx + r * topk, out_score + r * topk,
               out_score64 ? out_score64 + r * topk : NULL);
     if (out_dots) out_dots[r] = dots;
+    row_cache_free(&rc);
     free(cand);
     free(keep);
     free(bl);

@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libdsaidx.so (C ABI declared in include/dsaidx.h).
+
+Argument marshalling only: PyTorch provides device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no CPU fallback — importing this module without the built library
+raises.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdsaidx.so")
+
+DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE = 0, -1, -2, -3
+DSA_ERR_CUDA, DSA_ERR_NONFINITE, DSA_ERR_TIMEOUT = -4, -5, -6
+DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
+DSA_ALGO_DSA, DSA_ALGO_MISA, DSA_ALGO_MISA_DAGGER, DSA_ALGO_HISA = 0, 1, 2, 3
+DSA_FLAG_CHECK = 1
+
+
+class DsaProblem(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("n_q", C.c_int32), ("n_k", C.c_int32),
+                ("heads", C.c_int32), ("dim", C.c_int32), ("topk", C.c_int32),
+                ("q_dtype", C.c_int32), ("k_dtype", C.c_int32), ("q_pos0", C.c_void_p),
+                ("k_len", C.c_void_p), ("flags", C.c_uint32)]
+
+
+class DsaRouteParams(C.Structure):
+    _fields_ = [("misa_block", C.c_int32), ("misa_h", C.c_int32), ("k_prime", C.c_int32),
+                ("hisa_block", C.c_int32), ("hisa_r", C.c_int32)]
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m sparse_attention_token_dsa_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    vp, i32, i64, sz = C.c_void_p, C.c_int32, C.c_int64, C.c_size_t
+    P = C.POINTER(DsaProblem)
+    R = C.POINTER(DsaRouteParams)
+    lib.dsa_status_string.restype = C.c_char_p
+    lib.dsa_status_string.argtypes = [i32]
+    lib.dsa_read_status.argtypes = [vp, vp]
+    lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
+    lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.misa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.misa_dagger_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.hisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
+    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "misa_index",
+              "misa_dagger_index", "hisa_index", "dsa_quantize_e4m3"):
+        getattr(lib, f).restype = C.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_string(s: int) -> str:
+    return lib.dsa_status_string(s).decode()
+
+
+def _check(rc: int, what: str):
+    if rc != DSA_OK:
+        raise DsaError(rc, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DSA_F32
+    if t.dtype == torch.bfloat16:
+        return DSA_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return DSA_E4M3
+    raise TypeError(f"unsupported operand dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def problem(q: torch.Tensor, k: torch.Tensor, topk: int, q_pos0=None, k_len=None,
+            flags: int = 0) -> DsaProblem:
+    """q [batch, n_q, heads, dim], k [batch, n_k, dim]."""
+    B, nq, H, d = q.shape
+    nk = k.shape[1]
+    return DsaProblem(B, nq, nk, H, d, topk, _dtype_code(q), _dtype_code(k), _ptr(q_pos0),
+                      _ptr(k_len), flags)
+
+
+def route_params(misa_block=0, misa_h=0, k_prime=0, hisa_block=0, hisa_r=0) -> DsaRouteParams:
+    return DsaRouteParams(misa_block, misa_h, k_prime, hisa_block, hisa_r)
+
+
+def dsa_workspace_size(p: DsaProblem, algo: int = DSA_ALGO_DSA, rp: DsaRouteParams | None = None) -> int:
+    n = C.c_size_t(0)
+    _check(lib.dsa_workspace_size(C.byref(p), algo, None if rp is None else C.byref(rp),
+                                  C.byref(n)), "dsa_workspace_size")
+    return n.value
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None and workspace.numel() >= nbytes:
+        return workspace
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _outputs(B, nq, topk, device, out):
+    if out is not None:
+        return out
+    return (torch.empty((B, nq, topk), dtype=torch.int32, device=device),
+            torch.empty((B, nq, topk), dtype=torch.float32, device=device))
+
+
+def dsa_index(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_len=None, flags=0,
+              out=None, workspace=None, stream=None):
+    """DSA indexer top-k.  Returns (idx int32 [B,n_q,k], score fp32 [B,n_q,k])."""
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    ws = _workspace(dsa_workspace_size(p), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.dsa_index(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale), _ptr(w),
+                         _ptr(idx), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream)), "dsa_index")
+    return idx, sc
+
+
+def misa_index(q, k, w, topk, block, h, q_pos0=None, k_len=None, flags=0, out=None,
+               out_heads=None, out_E=None, workspace=None, stream=None):
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    rp = route_params(misa_block=block, misa_h=h)
+    ws = _workspace(dsa_workspace_size(p, DSA_ALGO_MISA, rp), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.misa_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(sc),
+                          _ptr(out_heads), _ptr(out_E), _ptr(ws), ws.numel(), _stream(stream)),
+           "misa_index")
+    return idx, sc
+
+
+def misa_dagger_index(q, k, w, topk, block, h, k_prime, q_pos0=None, k_len=None, flags=0,
+                      out=None, out_heads=None, out_pool=None, workspace=None, stream=None):
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    rp = route_params(misa_block=block, misa_h=h, k_prime=k_prime)
+    ws = _workspace(dsa_workspace_size(p, DSA_ALGO_MISA_DAGGER, rp), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.misa_dagger_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx),
+                                 _ptr(sc), _ptr(out_heads), _ptr(out_pool), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "misa_dagger_index")
+    return idx, sc
+
+
+def hisa_index(q, k, w, topk, block, r, route_h=0, route_block=1024, q_pos0=None, k_len=None,
+               flags=0, out=None, out_blocks=None, out_heads=None, workspace=None, stream=None):
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    rp = route_params(misa_block=route_block if route_h else 0, misa_h=route_h, hisa_block=block,
+                      hisa_r=r)
+    ws = _workspace(dsa_workspace_size(p, DSA_ALGO_HISA, rp), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.hisa_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(sc),
+                          _ptr(out_blocks), _ptr(out_heads), _ptr(ws), ws.numel(), _stream(stream)),
+           "hisa_index")
+    return idx, sc
+
+
+def dsa_quantize_e4m3(x: torch.Tensor, stream=None):
+    """Per-row e4m3 codes (uint8, same shape) and fp32 scales (shape[:-1])."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols
+    out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(lib.dsa_quantize_e4m3(_ptr(x), _dtype_code(x), rows, cols, _ptr(out), _ptr(sc),
+                                 _stream(stream)), "dsa_quantize_e4m3")
+    return out, sc
+
+
+def dsa_read_status(workspace: torch.Tensor, stream=None) -> int:
+    return lib.dsa_read_status(_ptr(workspace), _stream(stream))

@@ -1,0 +1,427 @@
+// dsaidx.cu — C ABI of the B200 DSA lightning-indexer library (see
+// include/dsaidx.h for the contract).  Host code here only validates
+// arguments, plans the launch, carves the caller's workspace, encodes TMA
+// descriptors and launches the kernels; every step of the computation runs on
+// the GPU.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/dsaidx.h"
+#include "common.cuh"
+#include "finalize.cuh"
+#include "prep.cuh"
+#include "scan.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr int kTargetCtas = 296;  // 148 SMs x 2: sizing target for split-K decode
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1)) == 0; }
+
+// ------------------------------------------------------------- scan plan --
+struct ScanPlan {
+  MmaKind kind;
+  bool split;
+  int parts, esz, atoms, kstages;
+  int QG, G, qcols, stage_cols, n_qt, C, chunk, n_items, keep, cap;
+  int rows;
+  size_t smem;
+  int ctas_per_sm;
+};
+
+size_t scan_smem_bytes(MmaKind kind, int G, int qcols) {
+  const int esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
+  const int atoms = esz;  // d = 128
+  const int kstages = kind == MmaKind::E4M3 ? 4 : 2;
+  size_t q = align_up((size_t)G * atoms * qcols * 128, 1024);
+  size_t k = (size_t)kstages * atoms * 128 * 128;
+  return 1024 + q + k + sizeof(ScanSmemTail);
+}
+
+// H: heads scanned; n_q / n_k / batch: geometry; keep: entries kept per row.
+ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H, int keep) {
+  ScanPlan pl{};
+  pl.kind = kind;
+  pl.split = split;
+  pl.parts = split ? 2 : 1;
+  pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
+  pl.atoms = pl.esz;
+  pl.kstages = kind == MmaKind::E4M3 ? 4 : 2;
+  const int ncols_max = kind == MmaKind::TF32 ? 128 : 256;
+  const int hp = H * pl.parts;
+  int qg_full = ncols_max / hp;
+  int qg_min = hp >= 16 ? 1 : 16 / hp;
+  int QG = qg_full;
+  while (QG > qg_min && QG / 2 >= n_q) QG /= 2;  // few query rows (decode): shrink
+  if (QG > 1 && (QG & 1)) QG = 1;
+  pl.QG = QG;
+  pl.G = (kind == MmaKind::TF32 || QG == 1 || n_q <= QG) ? 1 : 2;
+  pl.qcols = QG * hp;
+  pl.stage_cols = pl.qcols > 128 ? 256 : 128;
+  pl.n_qt = (n_q + QG * pl.G - 1) / (QG * pl.G);
+  pl.rows = batch * n_q;
+  pl.smem = scan_smem_bytes(kind, pl.G, pl.qcols);
+  const size_t per_sm = 228 * 1024;
+  int by_smem = (int)(per_sm / (pl.smem + 1024));
+  int by_tmem = 512 / (2 * pl.stage_cols);
+  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
+  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
+  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
+  // split-K over keys when there are too few query tiles to fill the GPU
+  const long long tiles = (long long)batch * pl.n_qt;
+  int C = 1, chunk = 0;
+  if (tiles < kTargetCtas && n_k > 4 * 128) {
+    C = (int)(kTargetCtas / tiles);  // one round: batch * tiles * C <= target
+    if (C < 1) C = 1;
+    if (C > kFinMaxSeg) C = kFinMaxSeg;
+    chunk = (n_k + C - 1) / C;
+    chunk = (chunk + 127) / 128 * 128;
+    if (chunk < 512) chunk = 512;
+    C = (n_k + chunk - 1) / chunk;
+    if (C <= 1) {
+      C = 1;
+      chunk = 0;
+    }
+  }
+  pl.C = C;
+  pl.chunk = chunk;
+  pl.n_items = (int)(tiles * C);
+  pl.keep = keep;
+  pl.cap = keep + (keep > 4096 ? keep : 4096) + 256;
+  return pl;
+}
+
+// ---------------------------------------------------------- TMA encoding --
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows, 128 elements] operand: box = 128 bytes x box_rows,
+// 128-byte swizzle (the layout the MMA descriptors expect).
+bool make_map(CUtensorMap* m, const void* base, int esz, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  CUtensorMapDataType dt = esz == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                           : esz == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                      : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {(cuuint64_t)(128), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)128 * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <MmaKind K, bool S>
+cudaError_t launch_scan_t(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
+                          const ScanArgs& a, cudaStream_t st) {
+  auto kern = scan_kernel<K, S>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)pl.smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int grid = sms * pl.ctas_per_sm;
+  if (grid > pl.n_items) grid = pl.n_items;
+  if (grid < 1) grid = 1;
+  kern<<<grid, kScanThreads, pl.smem, st>>>(qm, km, a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
+                        const ScanArgs& a, cudaStream_t st) {
+  switch (pl.kind) {
+    case MmaKind::TF32: return launch_scan_t<MmaKind::TF32, false>(pl, qm, km, a, st);
+    case MmaKind::BF16: return launch_scan_t<MmaKind::BF16, false>(pl, qm, km, a, st);
+    default:
+      return pl.split ? launch_scan_t<MmaKind::E4M3, true>(pl, qm, km, a, st)
+                      : launch_scan_t<MmaKind::E4M3, false>(pl, qm, km, a, st);
+  }
+}
+
+cudaError_t launch_finalize(int rows, int C, int topk, int cap, int sorted, const uint64_t* logs,
+                            const int32_t* cnt, const int32_t* buf, int32_t* out_idx,
+                            float* out_score, cudaStream_t st) {
+  FinalArgs f{};
+  f.rows = rows;
+  f.C = C;
+  f.topk = topk;
+  f.cap = cap;
+  int sc = 1;
+  while (sc < topk) sc <<= 1;
+  f.sort_cap = sc;
+  f.sorted = sorted;
+  f.logs = logs;
+  f.log_cnt = cnt;
+  f.log_buf = buf;
+  f.out_idx = out_idx;
+  f.out_score = out_score;
+  size_t smem = (size_t)sc * sizeof(uint64_t);
+  cudaError_t e =
+      cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  finalize_kernel<<<rows, kFinThreads, smem, st>>>(f);
+  return cudaGetLastError();
+}
+
+// Device-side input checks under DSA_FLAG_CHECK: scales finite and positive,
+// lengths inside [0, n_k].
+__global__ void check_inputs_kernel(const float* qs, int64_t nqs, const float* ks, int64_t nks,
+                                    const int32_t* pos0, const int32_t* klen, int batch, int n_k,
+                                    int32_t* status) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t j = i; j < nqs; j += stride)
+    if (!(isfinite(qs[j]) && qs[j] > 0.f)) set_status(status, DSA_ERR_NONFINITE, 100);
+  for (int64_t j = i; j < nks; j += stride)
+    if (!(isfinite(ks[j]) && ks[j] > 0.f)) set_status(status, DSA_ERR_NONFINITE, 101);
+  for (int64_t j = i; j < batch; j += stride) {
+    if (klen && (klen[j] < 0 || klen[j] > n_k)) set_status(status, DSA_ERR_INVALID, 102);
+    if (pos0 && pos0[j] < 0) set_status(status, DSA_ERR_INVALID, 103);
+  }
+}
+
+// ------------------------------------------------------------ validation --
+int validate_problem(const dsa_problem* p) {
+  if (!p) return DSA_ERR_INVALID;
+  if (p->batch < 1 || p->n_q < 1 || p->n_k < 1 || p->heads < 1 || p->dim < 1 || p->topk < 1)
+    return DSA_ERR_INVALID;
+  if (p->dim != 128) return DSA_ERR_UNSUPPORTED;
+  if (!pow2_in(p->heads, 8, 128)) return DSA_ERR_UNSUPPORTED;
+  if (p->topk > 8192) return DSA_ERR_UNSUPPORTED;
+  if (p->n_k > (1 << 24) || (long long)p->batch * p->n_k > (1ll << 31)) return DSA_ERR_UNSUPPORTED;
+  if ((long long)p->batch * p->n_q * p->heads * 2 > (1ll << 31)) return DSA_ERR_UNSUPPORTED;
+  const int qd = p->q_dtype, kd = p->k_dtype;
+  if (qd < DSA_F32 || qd > DSA_E4M3 || kd < DSA_F32 || kd > DSA_E4M3) return DSA_ERR_INVALID;
+  const bool same = qd == kd;
+  const bool split = (qd == DSA_BF16 || qd == DSA_F32) && kd == DSA_E4M3;
+  if (!same && !split) return DSA_ERR_UNSUPPORTED;
+  if (split && p->heads < 32) return DSA_ERR_UNSUPPORTED;
+  return DSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Kind / split decision of a validated problem.
+void kind_of(const dsa_problem* p, MmaKind* kind, bool* split) {
+  *split = (p->q_dtype != DSA_E4M3) && p->k_dtype == DSA_E4M3;
+  if (p->k_dtype == DSA_E4M3)
+    *kind = MmaKind::E4M3;
+  else if (p->k_dtype == DSA_BF16)
+    *kind = MmaKind::BF16;
+  else
+    *kind = MmaKind::TF32;
+}
+
+struct DsaLayout {
+  ScanPlan pl;
+  size_t off_logs, off_cnt, off_buf, off_parts, off_hscale, total;
+};
+
+DsaLayout dsa_layout(const dsa_problem* p) {
+  DsaLayout L{};
+  MmaKind kind;
+  bool split;
+  kind_of(p, &kind, &split);
+  L.pl = plan_scan(kind, split, p->batch, p->n_q, p->n_k, p->heads, p->topk);
+  size_t off = kWsHeaderBytes;
+  const size_t slots = (size_t)L.pl.rows * L.pl.C;
+  L.off_logs = off;
+  off += align_up(slots * 2 * L.pl.cap * sizeof(uint64_t));
+  L.off_cnt = off;
+  off += align_up(slots * sizeof(int32_t));
+  L.off_buf = off;
+  off += align_up(slots * sizeof(int32_t));
+  L.off_parts = off;
+  if (split) off += align_up((size_t)L.pl.rows * 2 * p->heads * p->dim);
+  L.off_hscale = off;
+  if (split) off += align_up((size_t)L.pl.rows * p->heads * sizeof(float));
+  L.total = off;
+  return L;
+}
+
+int finish(const dsa_problem* p, void* ws, cudaStream_t st) {
+  if (cudaPeekAtLastError() != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_CUDA;
+  }
+  if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(ws, st);
+  return DSA_OK;
+}
+
+}  // namespace
+
+// ===================================================================== ABI ==
+extern "C" {
+
+const char* dsa_status_string(int32_t s) {
+  switch (s) {
+    case DSA_OK: return "ok";
+    case DSA_ERR_INVALID: return "invalid argument (null pointer, bad size or inconsistent shape)";
+    case DSA_ERR_UNSUPPORTED: return "unsupported dtype, dim, heads or top-k";
+    case DSA_ERR_WORKSPACE: return "workspace missing or smaller than dsa_workspace_size()";
+    case DSA_ERR_CUDA: return "CUDA runtime error or launch failure";
+    case DSA_ERR_NONFINITE: return "non-finite, zero or negative scale";
+    case DSA_ERR_TIMEOUT: return "a bounded device wait expired";
+    default: return "unknown status";
+  }
+}
+
+int dsa_read_status(const void* workspace, void* stream) {
+  if (!workspace) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  int32_t s = 0;
+  if (cudaMemcpy(&s, workspace, sizeof(s), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return s;
+}
+
+int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
+                       size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID;
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  (void)rp;
+  if (algo == DSA_ALGO_DSA) {
+    *bytes = dsa_layout(p).total;
+    return DSA_OK;
+  }
+  return DSA_ERR_UNSUPPORTED;
+}
+
+int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+              const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  if (!q || !k || !w || !out_idx || !out_score) return DSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID;
+  if (p->q_dtype == DSA_E4M3 && !q_scale) return DSA_ERR_INVALID;
+  if (p->k_dtype == DSA_E4M3 && !k_scale) return DSA_ERR_INVALID;
+  const DsaLayout L = dsa_layout(p);
+  if (!workspace || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+  const ScanPlan& pl = L.pl;
+  if (p->flags & DSA_FLAG_CHECK) {
+    check_inputs_kernel<<<64, 256, 0, st>>>(
+        p->q_dtype == DSA_E4M3 ? q_scale : nullptr,
+        p->q_dtype == DSA_E4M3 ? (int64_t)p->batch * p->n_q : 0,
+        p->k_dtype == DSA_E4M3 ? k_scale : nullptr,
+        p->k_dtype == DSA_E4M3 ? (int64_t)p->batch * p->n_k : 0, p->q_pos0, p->k_len, p->batch,
+        p->n_k, status);
+  }
+  const void* qop = q;
+  const float* hscale = nullptr;
+  if (pl.split) {
+    uint8_t* parts = ws + L.off_parts;
+    float* hs = reinterpret_cast<float*>(ws + L.off_hscale);
+    const int64_t rh = (int64_t)pl.rows * p->heads;
+    split_query_kernel<<<(unsigned)((rh + 7) / 8), 256, 0, st>>>(q, p->q_dtype, pl.rows, p->heads,
+                                                               p->dim, parts, hs);
+    qop = parts;
+    hscale = hs;
+  }
+  CUtensorMap qm, km;
+  const int qesz = pl.split ? 1 : pl.esz;
+  if (!make_map(&qm, qop, qesz, (uint64_t)pl.rows * p->heads * pl.parts, (uint32_t)pl.qcols))
+    return DSA_ERR_CUDA;
+  if (!make_map(&km, k, pl.esz, (uint64_t)p->batch * p->n_k, 128)) return DSA_ERR_CUDA;
+  ScanArgs a{};
+  a.batch = p->batch;
+  a.n_q = p->n_q;
+  a.n_k = p->n_k;
+  a.H = p->heads;
+  a.d = p->dim;
+  a.keep = p->topk;
+  a.QG = pl.QG;
+  a.G = pl.G;
+  a.stage_cols = pl.stage_cols;
+  a.n_qt = pl.n_qt;
+  a.C = pl.C;
+  a.chunk = pl.chunk;
+  a.n_items = pl.n_items;
+  a.q_pos0 = p->q_pos0;
+  a.k_len = p->k_len;
+  a.w = w;
+  a.row_scale = p->q_dtype == DSA_E4M3 ? q_scale : nullptr;
+  a.head_scale = hscale;
+  a.k_scale = p->k_dtype == DSA_E4M3 ? k_scale : nullptr;
+  a.logs = reinterpret_cast<uint64_t*>(ws + L.off_logs);
+  a.log_cnt = reinterpret_cast<int32_t*>(ws + L.off_cnt);
+  a.log_buf = reinterpret_cast<int32_t*>(ws + L.off_buf);
+  a.cap = pl.cap;
+  a.status = status;
+  if (launch_scan(pl, qm, km, a, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (launch_finalize(pl.rows, pl.C, p->topk, pl.cap, 1, a.logs, a.log_cnt, a.log_buf, out_idx,
+                      out_score, st) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return finish(p, workspace, st);
+}
+
+int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* out,
+                      float* out_scale, void* stream) {
+  if (!x || !out || !out_scale || rows < 0 || cols < 1) return DSA_ERR_INVALID;
+  if (x_dtype != DSA_F32 && x_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  if (rows == 0) return DSA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  quantize_rows_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(x, x_dtype, rows, cols, out,
+                                                                   out_scale);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+               const float* w, int32_t* out_idx, float* out_score, int32_t* out_heads,
+               float* out_E, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
+  (void)out_heads; (void)out_E; (void)workspace; (void)workspace_bytes; (void)stream;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
+                      const void* k, const float* w, int32_t* out_idx, float* out_score,
+                      int32_t* out_heads, int32_t* out_pool, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
+  (void)out_heads; (void)out_pool; (void)workspace; (void)workspace_bytes; (void)stream;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+               const float* w, int32_t* out_idx, float* out_score, int32_t* out_blocks,
+               int32_t* out_heads, void* workspace, size_t workspace_bytes, void* stream) {
+  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
+  (void)out_blocks; (void)out_heads; (void)workspace; (void)workspace_bytes; (void)stream;
+  return DSA_ERR_UNSUPPORTED;
+}
+
+}  // extern "C"

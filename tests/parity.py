@@ -1,0 +1,90 @@
+"""Comparison rules between the CUDA path and the CPU oracle.
+
+Exact rule (integer-valued inputs, where fp32 accumulation is exact in any
+order): indices and scores must be bit-identical, padding included.
+
+Tolerance rule (real-valued inputs).  With nu(t, s) = sum_j |w_tj| ||q_tj||
+||k_s|| / sqrt(d), the typical magnitude of a score:
+  - every returned score satisfies |I_gpu - I_ref| <= tol * max(|I_ref|, nu);
+  - the returned sets may differ only on tokens whose reference score lies
+    within tol * nu of the reference k-th score (several sets are then correct);
+  - the number of valid entries is exactly min(k, |legal|), indices are unique,
+    legal, and ordered by (score desc, index asc);
+  - the IoU against the reference set is reported.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+
+
+def exact(gpu_idx, gpu_score, ref_idx, ref_score):
+    gi, gs = np.asarray(gpu_idx), np.asarray(gpu_score)
+    assert np.array_equal(gi, ref_idx), _first_diff(gi, ref_idx)
+    both_inf = np.isneginf(gs) & np.isneginf(ref_score)
+    assert np.array_equal(gs[~both_inf], ref_score[~both_inf])
+    assert not np.any(np.signbit(gs[gs == 0]))
+
+
+def _first_diff(a, b):
+    d = np.argwhere(a != b)
+    if len(d) == 0:
+        return "shapes differ"
+    r = tuple(d[0])
+    return f"first difference at {r}: gpu {a[r]} ref {b[r]}"
+
+
+def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_score64, tol,
+                     heads=None, legal=None):
+    """Check the tolerance rule row by row; returns the mean IoU.
+
+    heads: per-row head lists [n_rows, h] for routed scores (None: all heads).
+    legal: per-row legal key counts (None: from the problem)."""
+    p = inp.prob
+    ious = []
+    for a, row in enumerate(rows):
+        gi = np.asarray(gpu_idx[a])
+        gs = np.asarray(gpu_score[a])
+        ri = np.asarray(ref_idx[a])
+        nv = int(np.sum(ri >= 0))
+        gv = int(np.sum(gi >= 0))
+        assert gv == nv, f"row {row}: {gv} valid entries, reference {nv}"
+        assert np.all(gi[nv:] == -1) and np.all(np.isneginf(gs[nv:]))
+        if nv == 0:
+            ious.append(1.0)
+            continue
+        g_set = gi[:nv]
+        assert len(np.unique(g_set)) == nv, f"row {row}: duplicate indices"
+        n_legal = p.legal_count(int(row)) if legal is None else int(legal[a])
+        assert np.all((g_set >= 0) & (g_set < n_legal)), f"row {row}: illegal index"
+        hrow = None if heads is None else np.repeat(np.asarray(heads[a])[None], nv, 0)
+        rows_v = np.full(nv, row, np.int64)
+        ref_at_g = oracle.score_pairs(inp, rows_v, g_set, hrow)
+        nu_g = oracle.score_scale_pairs(inp, rows_v, g_set)
+        err = np.abs(gs[:nv].astype(np.float64) - ref_at_g)
+        bound = tol * np.maximum(np.abs(ref_at_g), nu_g)
+        bad = np.argwhere(err > bound)
+        assert len(bad) == 0, (f"row {row}: score error {err[bad[0][0]]:.3e} > "
+                               f"{bound[bad[0][0]]:.3e} at s={g_set[bad[0][0]]}")
+        # order by (score desc, index asc) on the GPU's own scores
+        s0, s1 = gs[: nv - 1], gs[1:nv]
+        i0, i1 = g_set[:-1], g_set[1:]
+        assert np.all((s0 > s1) | ((s0 == s1) & (i0 < i1))), f"row {row}: output not ordered"
+        # set difference only near the reference cutoff
+        cutoff = ref_score64[a, nv - 1]
+        extra = np.setdiff1d(g_set, ri[:nv])
+        missing = np.setdiff1d(ri[:nv], g_set)
+        for group in (extra, missing):
+            if len(group) == 0:
+                continue
+            rr = np.full(len(group), row, np.int64)
+            hh = None if heads is None else np.repeat(np.asarray(heads[a])[None], len(group), 0)
+            v = oracle.score_pairs(inp, rr, group, hh)
+            nu = oracle.score_scale_pairs(inp, rr, group)
+            far = np.abs(v - cutoff) > tol * nu
+            assert not np.any(far), (f"row {row}: token {group[far][0]} differs from the "
+                                     f"reference set but is not near the cut-off")
+        inter = len(np.intersect1d(g_set, ri[:nv]))
+        ious.append(inter / (2 * nv - inter))
+    return float(np.mean(ious)) if ious else 1.0

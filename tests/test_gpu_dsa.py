@@ -1,0 +1,210 @@
+"""GPU parity of dsa_index (and the FP8 quantiser) against the CPU oracle.
+
+Exact on integer-valued inputs; within the tolerance rule of tests/parity.py on
+real-valued inputs (1e-3 for bf16 operands, 2e-2 for fp8 against the
+unquantised values).  Sizes span several 128-key tiles and query tiles with
+ragged tails; full-size workloads are checked on sampled rows.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import parity
+from sparse_attention_token_dsa_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 1e-3
+TOL_FP8 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def B():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from sparse_attention_token_dsa_b200 import binding
+    oracle.build()
+    return binding
+
+
+def dev(x):
+    import torch
+    if x is None:
+        return None
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def run_dsa(B, p, q=None, k=None, q_scale=None, k_scale=None, flags=0):
+    q = dev(p.q) if q is None else q
+    k = dev(p.k) if k is None else k
+    idx, sc = B.dsa_index(q, k, dev(p.w), p.topk, q_scale=q_scale, k_scale=k_scale,
+                          q_pos0=dev(p.q_pos0), k_len=dev(p.k_len), flags=flags)
+    import torch
+    torch.cuda.synchronize()
+    return (idx.cpu().numpy().reshape(-1, p.topk), sc.cpu().numpy().reshape(-1, p.topk))
+
+
+# ------------------------------------------------------------------ exact ---
+
+@pytest.mark.parametrize("dtype", [gen.F32, gen.BF16])
+def test_integer_full_layer_bit_exact(B, dtype):
+    """L = 1024 causal, H = 64, d = 128, k = 128, integer q, k, w: bit-exact."""
+    p = gen.integer_problem(1, 1, 1024, 1024, 64, 128, 128, dtype=dtype)
+    gi, gs = run_dsa(B, p, flags=B.DSA_FLAG_CHECK)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
+@pytest.mark.parametrize("heads", [8, 16, 32, 128])
+def test_integer_heads_bit_exact(B, heads):
+    p = gen.integer_problem(2, 1, 300, 700, heads, 128, 64, q_pos0=[400], dtype=gen.BF16)
+    gi, gs = run_dsa(B, p)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
+def test_integer_ragged_batches_bit_exact(B):
+    """Several sequences, per-sequence query offsets and key lengths, rows with
+    fewer legal keys than k (padding), tails in both tiles."""
+    p = gen.integer_problem(3, 3, 150, 500, 64, 128, 200, q_pos0=[0, 100, 37],
+                            k_len=[300, 500, 200], dtype=gen.BF16)
+    gi, gs = run_dsa(B, p)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
+def test_integer_topk_above_keys_pads(B):
+    p = gen.integer_problem(4, 1, 40, 300, 64, 128, 512, dtype=gen.F32)
+    gi, gs = run_dsa(B, p)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+    assert np.all(gi[:, 300:] == -1)
+
+
+def test_integer_many_ties_long_rows_bit_exact(B):
+    """Small value range => massive score ties; several threshold raises per row."""
+    p = gen.integer_problem(5, 1, 64, 20000, 64, 128, 1024, qk_max=1, w_max=1, dtype=gen.BF16)
+    gi, gs = run_dsa(B, p)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
+def test_single_key_and_single_query(B):
+    p = gen.integer_problem(6, 2, 1, 1, 64, 128, 4, dtype=gen.F32)
+    gi, gs = run_dsa(B, p)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
+# -------------------------------------------------------------- real-valued --
+
+def test_bf16_real_small(B):
+    p = gen.normal_problem(20, 2, 1000, 1300, 64, 128, 256, q_pos0=[300, 0], k_len=[1300, 1000])
+    gi, gs = run_dsa(B, p)
+    inp = oracle.Inputs(p)
+    rows = np.arange(p.batch * p.n_q)[::7]
+    ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
+    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
+    assert iou > 0.99
+
+
+def test_bf16_needles_32k_sampled(B):
+    """Full-size 32K prefill layer (H = 64, k = 2048) with planted needles."""
+    p = gen.normal_problem(2, 1, 32768, 32768, 64, 128, 2048, n_needles=32)
+    gi, gs = run_dsa(B, p)
+    inp = oracle.Inputs(p)
+    rows = gen.stratified_rows(p, 24)
+    ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
+    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
+    assert iou > 0.99
+    for b, t, s in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
+        assert s in set(gi[b * p.n_q + t].tolist()), "needle not selected"
+
+
+# ---------------------------------------------------------------------- FP8 --
+
+def test_quantizer_matches_oracle_bit_exact(B):
+    import torch
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((777, 128)).astype(np.float32)
+    x[5] = 0.0
+    x[6] *= 1e-6
+    x[7] *= 1e4
+    x[8, :5] = [448.0, -448.0, 1e-12, -0.0, 3.0]
+    for dt, arr in ((gen.F32, x), (gen.BF16, gen.f32_to_bf16_bits(x))):
+        codes, sc = B.dsa_quantize_e4m3(dev(arr))
+        torch.cuda.synchronize()
+        rc, rsc = oracle.quantize_rows(arr, dt)
+        assert np.array_equal(sc.cpu().numpy(), rsc)
+        assert np.array_equal(codes.cpu().numpy(), rc)
+
+
+def _fp8_problem(p, B):
+    """GPU-quantised operands (checked bit-exact against the oracle's quantiser)."""
+    qd, kd = dev(p.q), dev(p.k)
+    qc, qs = B.dsa_quantize_e4m3(qd.reshape(p.batch * p.n_q, p.heads * p.dim))
+    kc, ks = B.dsa_quantize_e4m3(kd)
+    rqc, rqs = oracle.quantize_rows(p.q.reshape(p.batch * p.n_q, -1), gen.BF16)
+    rkc, rks = oracle.quantize_rows(p.k, gen.BF16)
+    assert np.array_equal(qc.cpu().numpy(), rqc) and np.array_equal(kc.cpu().numpy(), rkc)
+    return qc.reshape(p.q.shape), qs, kc, ks, rqc.reshape(p.q.shape), rqs, rkc, rks
+
+
+def test_fp8_prefill(B):
+    p = gen.normal_problem(21, 1, 2048, 2048, 64, 128, 256)
+    qc, qs, kc, ks, rqc, rqs, rkc, rks = _fp8_problem(p, B)
+    gi, gs = run_dsa(B, p, q=qc, k=kc, q_scale=qs, k_scale=ks, flags=B.DSA_FLAG_CHECK)
+    rows = np.arange(p.n_q)[::5]
+    # quantisation-faithful: oracle on the same e4m3 codes
+    inq = oracle.Inputs(p, q=rqc, k=rkc, q_dtype=gen.E4M3, k_dtype=gen.E4M3, q_scale=rqs,
+                        k_scale=rks)
+    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
+    parity.within_tolerance(inq, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
+    # against the unquantised bf16 values
+    inp = oracle.Inputs(p)
+    ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
+    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_FP8)
+    assert iou > 0.7
+
+
+@pytest.mark.parametrize("batch,n_k", [(4, 20000), (3, 5000)])
+def test_fp8_decode_split_query(B, batch, n_k):
+    """Decode: bf16 q (split into two e4m3 parts inside the library), e4m3 keys."""
+    p, _ = gen.decode_problem(30 + batch, batch, n_k, 64, 128, 2048,
+                              k_len=[n_k - 37 * b for b in range(batch)])
+    kc, ks = B.dsa_quantize_e4m3(dev(p.k))
+    gi, gs = run_dsa(B, p, k=kc, k_scale=ks)
+    rkc, rks = oracle.quantize_rows(p.k, gen.BF16)
+    assert np.array_equal(kc.cpu().numpy(), rkc)
+    inq = oracle.Inputs(p, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
+    rows = np.arange(batch)
+    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
+    iou = parity.within_tolerance(inq, rows, gi, gs, ri, rs64, TOL_FP8)
+    assert iou > 0.9
+
+
+def test_fp8_decode_full_size(B):
+    """32 sequences x 131072 cached keys, H = 64, k = 2048 (every row checked)."""
+    p, _ = gen.decode_problem(3, 32, 131072, 64, 128, 2048)
+    kc, ks = B.dsa_quantize_e4m3(dev(p.k))
+    gi, gs = run_dsa(B, p, k=kc, k_scale=ks)
+    rkc, rks = oracle.quantize_rows(p.k, gen.BF16)
+    inq = oracle.Inputs(p, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
+    rows = np.arange(32)
+    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
+    iou = parity.within_tolerance(inq, rows, gi, gs, ri, rs64, TOL_FP8)
+    assert iou > 0.9
+
+
+def test_check_flag_reports_bad_scale(B):
+    import torch
+    p = gen.normal_problem(22, 1, 64, 256, 64, 128, 16)
+    qc, qs, kc, ks, *_ = _fp8_problem(p, B)
+    ks[3] = float("nan")
+    with pytest.raises(B.DsaError) as e:
+        B.dsa_index(qc, kc, dev(p.w), p.topk, q_scale=qs, k_scale=ks, flags=B.DSA_FLAG_CHECK)
+    assert e.value.status == B.DSA_ERR_NONFINITE
+    torch.cuda.synchronize()
