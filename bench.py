@@ -1,0 +1,419 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 DSA lightning indexer (one JSON line on rank 0).
+
+Default workload: DSA indexer prefill, batch 1, L = 32768 causal, H_I = 64,
+d = 128, top-k = 2048, bf16 q / k ~ N(0,1), w ~ N(0, 1/64), 32 planted needles.
+A step is one whole indexer layer (score -> causal mask -> exact token top-k,
+ordered output) through the library's C ABI.  Inputs are larger than L2
+(q alone is 512 MiB), so no explicit flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+N > 1 (torchrun): every rank runs its own independent layer (weak scaling, no
+collective on the data path); the reported time is the max over ranks.
+--impl reference times the CPU oracle (the only reference this method has) on
+a bounded sample of rows of the same workload, extrapolated to a full layer.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_attention_token_dsa_b200 import inputs as gen  # noqa: E402
+
+METRIC = "indexer ms/layer @128K prefill; decode µs/query; % of tensor-pipe / HBM peak"
+
+WORKLOADS = {
+    "dsa_prefill_32k": dict(
+        desc="DSA indexer prefill, batch 1, L=32768 causal, H_I=64, d=128, top-k=2048, "
+             "bf16 q,k ~N(0,1), w ~N(0,1/64), 32 planted needles",
+        kind="prefill", batch=1, L=32768, H=64, topk=2048, fp8=False, seed=2, needles=32),
+    "dsa_prefill_32k_fp8": dict(
+        desc="DSA indexer prefill, batch 1, L=32768 causal, H_I=64, d=128, top-k=2048, "
+             "e4m3 q,k with per-token fp32 scales (quantised outside the timed region)",
+        kind="prefill", batch=1, L=32768, H=64, topk=2048, fp8=True, seed=2, needles=32),
+    "dsa_prefill_8k": dict(
+        desc="DSA indexer prefill, batch 1, L=8192 causal, H_I=64, d=128, top-k=2048, bf16 "
+             "(small case of the 32K workload, sized for ncu captures)",
+        kind="prefill", batch=1, L=8192, H=64, topk=2048, fp8=False, seed=2, needles=8),
+    "dsa_decode_128k": dict(
+        desc="DSA indexer decode, 32 sequences x 131072 cached keys, one query each, H_I=64, "
+             "d=128, e4m3 K with per-token fp32 scale, bf16 q, fp32 w, top-k=2048",
+        kind="decode", batch=32, L=131072, H=64, topk=2048, fp8=True, seed=3, needles=0),
+}
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one scan-kernel launch, from the
+# ncu captures summarised under profiles/, valid only while the kernel sources
+# hash to `src`; otherwise the traffic is reported as null.
+TRAFFIC = {}
+
+KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_attention_token_dsa_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            d = json.load(fh)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d["bf16_tflops_sustained"], src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
+
+
+def make_problem(w):
+    if w["kind"] == "prefill":
+        return gen.normal_problem(w["seed"], w["batch"], w["L"], w["L"], w["H"], 128, w["topk"],
+                                  n_needles=w["needles"])
+    p, _ = gen.decode_problem(w["seed"], w["batch"], w["L"], w["H"], 128, w["topk"])
+    return p
+
+
+def algorithmic_work(p):
+    """Causal (query, key) pairs, tensor FLOPs (2 * pairs * H * d) and operand bytes."""
+    pairs = sum(p.legal_count(r) for r in range(p.batch * p.n_q)) if p.n_q <= 4096 else None
+    if pairs is None:  # closed form for the default causal layouts
+        pairs = 0
+        for b in range(p.batch):
+            n0 = p.pos0(b)
+            n = p.n_q
+            pairs += n * (n0 + 1) + n * (n - 1) // 2
+    flops = 2.0 * pairs * p.heads * p.dim
+    return pairs, flops
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}",
+                 "--query-gpu=index,clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+def cpu_baseline(p, w, seconds=15.0):
+    """Oracle on a bounded, stratified sample of rows, extrapolated to the whole layer."""
+    import oracle
+    oracle.build()
+    inp = _oracle_inputs(p, w)
+    total_pairs, _ = algorithmic_work(p)
+    rows_all = gen.stratified_rows(p, 64)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    done, pairs_done, t_used = 0, 0, 0.0
+    for i in range(0, len(rows_all), cores):       # one row per core per call
+        chunk = rows_all[i:i + cores]
+        t0 = time.perf_counter()
+        oracle.dsa(inp, p.topk, chunk)
+        t_used += time.perf_counter() - t0
+        done += len(chunk)
+        pairs_done += sum(p.legal_count(int(r)) for r in chunk)
+        if t_used > seconds:
+            break
+    per_pair = t_used / max(pairs_done, 1)
+    layer_s = per_pair * total_pairs
+    return dict(layer_ms=layer_s * 1e3, rows=done, pairs=pairs_done, wall_s=t_used, omp=cores)
+
+
+def _oracle_inputs(p, w):
+    import oracle
+    if w["fp8"] and w["kind"] == "decode":
+        kc, ks = oracle.quantize_rows(p.k, gen.BF16)
+        return oracle.Inputs(p, k=kc, k_dtype=gen.E4M3, k_scale=ks)
+    if w["fp8"]:
+        qc, qs = oracle.quantize_rows(p.q.reshape(p.batch * p.n_q, -1), gen.BF16)
+        kc, ks = oracle.quantize_rows(p.k, gen.BF16)
+        return oracle.Inputs(p, q=qc.reshape(p.q.shape), k=kc, q_dtype=gen.E4M3,
+                             k_dtype=gen.E4M3, q_scale=qs, k_scale=ks)
+    return oracle.Inputs(p)
+
+
+def unit_of(w):
+    return ("µs/query", 1e3 / (w["batch"])) if w["kind"] == "decode" else ("ms/layer", 1.0)
+
+
+def run_reference(args, w, p):
+    """Reference arm: the CPU oracle as it stands, K timed sample steps."""
+    import oracle
+    oracle.build()
+    inp = _oracle_inputs(p, w)
+    total_pairs, _ = algorithmic_work(p)
+    rows = gen.stratified_rows(p, 16)
+    unit, scale = unit_of(w)
+
+    def step():
+        t0 = time.perf_counter()
+        oracle.dsa(inp, p.topk, rows)
+        dt = time.perf_counter() - t0
+        pairs = sum(p.legal_count(int(r)) for r in rows)
+        return dt * total_pairs / pairs * 1e3   # ms per layer, extrapolated
+
+    for _ in range(args.warmup):
+        step()
+    vals = [step() for _ in range(args.steps)]
+    ms = statistics.mean(vals)
+    value = ms * scale
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w["desc"]},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                             "sample": f"{len(rows)} stratified query rows per step, "
+                                       "extrapolated by causal pair count"},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="dsa_prefill_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = WORKLOADS[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w, make_problem(w))
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from sparse_attention_token_dsa_b200 import binding as B
+
+    p = make_problem(w)
+    dev = torch.device("cuda", local)
+
+    def to_dev(x):
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(np.ascontiguousarray(x)).to(dev)
+
+    qh = torch.from_numpy(p.q.view(np.int16)).view(torch.bfloat16)
+    kh = torch.from_numpy(p.k.view(np.int16)).view(torch.bfloat16)
+    wh = torch.from_numpy(p.w)
+    q, k, wt = qh.to(dev), kh.to(dev), wh.to(dev)
+    q_scale = k_scale = None
+    if w["fp8"]:
+        k, k_scale = B.dsa_quantize_e4m3(k)
+        if w["kind"] == "prefill":
+            q2, q_scale = B.dsa_quantize_e4m3(q.reshape(p.batch * p.n_q, -1))
+            q = q2.reshape(p.q.shape)
+            q_scale = q_scale.reshape(p.batch, p.n_q)
+    torch.cuda.synchronize()
+    prob = B.problem(q, k, p.topk)
+    ws = torch.empty(B.dsa_workspace_size(prob), dtype=torch.uint8, device=dev)
+    idx = torch.empty((p.batch, p.n_q, p.topk), dtype=torch.int32, device=dev)
+    sc = torch.empty((p.batch, p.n_q, p.topk), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        B.dsa_index_scan(prob, q, k, wt, ws, q_scale=q_scale, k_scale=k_scale, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        B.dsa_index_select(prob, idx, sc, ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    st = B.dsa_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    torch.cuda.synchronize()
+
+    stage_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(stage_ev[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed = t0.elapsed_time(t1)
+    scan_ms = statistics.mean(a.elapsed_time(b) for a, b in stage_ev)
+    st = B.dsa_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    if world > 1:
+        t = torch.tensor([elapsed], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+
+    # end to end through the public call with host buffers (pinned), copies inside
+    qp, kp, wp = qh.pin_memory(), kh.pin_memory(), wh.pin_memory()
+    idx_h = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
+    sc_h = torch.empty(sc.shape, dtype=torch.float32).pin_memory()
+    q_d = torch.empty_like(qh, device=dev)
+    k_d = torch.empty_like(kh, device=dev)
+    w_d = torch.empty_like(wh, device=dev)
+
+    def e2e_step():
+        q_d.copy_(qp, non_blocking=True)
+        k_d.copy_(kp, non_blocking=True)
+        w_d.copy_(wp, non_blocking=True)
+        qq, kk, qs_, ks_ = q_d, k_d, None, None
+        if w["fp8"]:
+            kk, ks_ = B.dsa_quantize_e4m3(k_d)
+            if w["kind"] == "prefill":
+                q2, qs_ = B.dsa_quantize_e4m3(q_d.reshape(p.batch * p.n_q, -1))
+                qq, qs_ = q2.reshape(p.q.shape), qs_.reshape(p.batch, p.n_q)
+        B.dsa_index(qq, kk, w_d, p.topk, q_scale=qs_, k_scale=ks_, out=(idx, sc), workspace=ws)
+        idx_h.copy_(idx, non_blocking=True)
+        sc_h.copy_(sc, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = qh.numel() * qh.element_size() + kh.numel() * kh.element_size() + wh.numel() * 4
+    d2h = idx.numel() * 4 + sc.numel() * 4
+
+    if rank == 0:
+        unit, scale = unit_of(w)
+        ms_per_step = elapsed / args.steps
+        value = ms_per_step / world * scale
+        pk = peaks()
+        pairs, flops = algorithmic_work(p)
+        long_region = elapsed > 1000.0
+        if w["kind"] == "prefill":
+            tf = flops / (scan_ms * 1e-3) / 1e12
+            fp8_peak = 2.0 * (pk["bf16_sustained"] if long_region else pk["bf16"])
+            peak = fp8_peak if w["fp8"] else (pk["bf16_sustained"] if long_region else pk["bf16"])
+            roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                    "frac": tf / peak,
+                    "peak_source": f"{pk['src']} bf16 {'sustained' if long_region else 'burst'}"
+                                   + (" x2 (fp8 nominal ratio)" if w["fp8"] else ""),
+                    "work": f"{flops / 1e12:.3f} TFLOP per launch (2*pairs*H*d)"}
+        else:
+            kbytes = p.batch * p.n_k * (128 + 4)
+            qbytes = p.batch * p.heads * 128 * 2 + p.batch * p.heads * 4
+            gbs = (kbytes + qbytes) / (scan_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                    "frac": gbs / pk["hbm"], "peak_source": f"{pk['src']} copy bandwidth",
+                    "work": f"{(kbytes + qbytes) / 1e6:.1f} MB per launch (e4m3 K + scales + q + w)"}
+        tr = TRAFFIC.get(args.workload)
+        roof["traffic"] = tr["bytes"] if tr and tr["src"] == kernel_hash() else None
+        roof["kernel"] = "scan_kernel"
+        roof["kernel_ms"] = scan_ms
+        line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+                "dtype": "e4m3/f32" if w["fp8"] else "bf16/f32", "data": "synthetic",
+                "config": {"workload": w["desc"], "l2": "inputs larger than L2 (no flush)",
+                           "parallelism": f"replicas x{world}", "select_ms": ms_per_step - scan_ms},
+                "roofline": roof,
+                "e2e": {"value": e2e_ms / world * scale, "unit": unit, "h2d_bytes_per_step": h2d,
+                        "d2h_bytes_per_step": d2h},
+                "gpu_launches": args.steps * (2 + (1 if (w["fp8"] and w["kind"] == "decode") else 0)),
+                "clocks": clk.summary()}
+        if world == 1 and not args.no_cpu_baseline:
+            cb = cpu_baseline(p, w)
+            line["cpu_baseline"] = {"value": cb["layer_ms"] * scale, "unit": unit,
+                                    "cores": cb["omp"], "kind": "oracle",
+                                    "sample": f"{cb['rows']} stratified rows "
+                                              f"({cb['pairs']} causal pairs, {cb['wall_s']:.1f} s), "
+                                              "extrapolated by pair count"}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

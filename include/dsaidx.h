@@ -128,6 +128,18 @@ int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const v
               const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
               void* workspace, size_t workspace_bytes, void* stream);
 
+/* The two stages of dsa_index, for callers that schedule (or time) them
+ * separately: dsa_index is exactly dsa_index_scan followed by
+ * dsa_index_select on the same workspace and stream.  The scan stage scores
+ * every legal (query, key) pair and leaves per-row candidate logs in the
+ * workspace; the select stage takes each row's exact top-k from them and
+ * writes the outputs. */
+int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+                   const float* k_scale, const float* w, void* workspace, size_t workspace_bytes,
+                   void* stream);
+int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
 /* MISA: block-pooled router picks rp->misa_h heads per query, those heads score
  * every legal token, token top-k.  out_heads [batch,n_q,h] int32 (ascending head
  * order) and out_E [batch,n_q,heads] fp32 (the router importance E) are optional

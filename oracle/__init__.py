@@ -52,7 +52,7 @@ def lib():
         _lib.orc_quantize_rows.argtypes = [vp, i32, i64, i32, vp, vp]
         _lib.orc_dsa_rows.argtypes = [vp, i32, vp, i64, vp, vp, vp, vp]
         _lib.orc_score_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
-        _lib.orc_score_scale_pairs.argtypes = [vp, vp, vp, i64, vp]
+        _lib.orc_abs_score_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
         _lib.orc_pool.argtypes = [vp, i32, i64, i32, vp]
         _lib.orc_misa_rows.argtypes = [vp, i32, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp,
                                        vp, vp, vp]
@@ -167,12 +167,17 @@ def score_pairs(inp: Inputs, rows, s, heads=None):
     return out
 
 
-def score_scale_pairs(inp: Inputs, rows, s):
-    """nu(t, s) = sum_j |w| ||q_j|| ||k_s|| / sqrt(d): the score-magnitude scale."""
+def abs_score_pairs(inp: Inputs, rows, s, heads=None):
+    """A(t, s) = sum_j |w| sum_c |q_jc k_c|: the error scale of each score."""
     rows = np.ascontiguousarray(rows, np.int64)
     s = np.ascontiguousarray(s, np.int64)
     out = np.empty(len(rows), np.float64)
-    lib().orc_score_scale_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(out))
+    if heads is not None:
+        heads = np.ascontiguousarray(heads, np.int32)
+        nh = heads.shape[1]
+    else:
+        nh = 0
+    lib().orc_abs_score_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(heads), nh, _p(out))
     return out
 
 

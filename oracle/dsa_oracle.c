@@ -361,29 +361,26 @@ int orc_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s,
   return ORC_OK;
 }
 
-/* Typical score magnitude at (row, s): sum_j |w_{t,j}| ||q_{t,j}|| ||k_s|| / sqrt(d).
- * Used by the tests as the denominator of the relative score tolerance. */
-int orc_score_scale_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
-                          double* out) {
+/* Error scale of a score at (row, s): A = sum_j |w_{t,j}| sum_c |q_{t,j,c} k_{s,c}|,
+ * the sum of the absolute values of the products the score adds up (the
+ * standard scale of rounding and quantisation error in a sum of products).
+ * heads == NULL means all heads, otherwise heads is [n, nh].  Used by the
+ * tests as the denominator of the relative score tolerance. */
+int orc_abs_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                        const int32_t* heads, int32_t nh, double* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t a = 0; a < n; ++a) {
     int64_t row = rows[a];
     int32_t b = (int32_t)(row / in->n_q);
-    double kn = 0.0;
-    for (int32_t c = 0; c < in->dim; ++c) {
-      double v = k_val(in, b, s[a], c);
-      kn += v * v;
-    }
+    int32_t cnt = heads ? nh : in->heads;
     double acc = 0.0;
-    for (int32_t j = 0; j < in->heads; ++j) {
-      double qn = 0.0;
-      for (int32_t c = 0; c < in->dim; ++c) {
-        double v = q_val(in, row, j, c);
-        qn += v * v;
-      }
-      acc += fabs((double)in->w[row * in->heads + j]) * sqrt(qn);
+    for (int32_t x = 0; x < cnt; ++x) {
+      int32_t j = heads ? heads[a * nh + x] : x;
+      double t = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) t += fabs(q_val(in, row, j, c) * k_val(in, b, s[a], c));
+      acc += fabs((double)in->w[row * in->heads + j]) * t;
     }
-    out[a] = acc * sqrt(kn) / sqrt((double)in->dim);
+    out[a] = acc;
   }
   return ORC_OK;
 }

@@ -53,11 +53,14 @@ def _load():
     lib.dsa_read_status.argtypes = [vp, vp]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_index_scan.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_index_select.argtypes = [P, vp, vp, vp, sz, vp]
     lib.misa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.misa_dagger_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
-    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "misa_index",
+    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "dsa_index_scan",
+              "dsa_index_select", "misa_index",
               "misa_dagger_index", "hisa_index", "dsa_quantize_e4m3"):
         getattr(lib, f).restype = C.c_int
     return lib
@@ -137,6 +140,18 @@ def dsa_index(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_len=None
     _check(lib.dsa_index(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale), _ptr(w),
                          _ptr(idx), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream)), "dsa_index")
     return idx, sc
+
+
+def dsa_index_scan(p: DsaProblem, q, k, w, workspace, q_scale=None, k_scale=None, stream=None):
+    """First stage of dsa_index (scores + candidate logs in `workspace`)."""
+    _check(lib.dsa_index_scan(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale), _ptr(w),
+                              _ptr(workspace), workspace.numel(), _stream(stream)), "dsa_index_scan")
+
+
+def dsa_index_select(p: DsaProblem, idx, score, workspace, stream=None):
+    """Second stage of dsa_index (exact top-k per row from the logs)."""
+    _check(lib.dsa_index_select(C.byref(p), _ptr(idx), _ptr(score), _ptr(workspace),
+                                workspace.numel(), _stream(stream)), "dsa_index_select")
 
 
 def misa_index(q, k, w, topk, block, h, q_pos0=None, k_len=None, flags=0, out=None,

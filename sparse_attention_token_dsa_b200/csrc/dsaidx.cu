@@ -32,19 +32,22 @@ struct ScanPlan {
   MmaKind kind;
   bool split;
   int parts, esz, atoms, kstages;
-  int QG, G, qcols, stage_cols, n_qt, C, chunk, n_items, keep, cap;
+  int QG, G, qcols, stage_cols, n_qt, C, chunk, n_items, keep, nsub, capw;
   int rows;
   size_t smem;
   int ctas_per_sm;
 };
 
-size_t scan_smem_bytes(MmaKind kind, int G, int qcols) {
+constexpr size_t kSmemBudget = 227 * 1024;
+
+size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols) {
   const int esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   const int atoms = esz;  // d = 128
-  const int kstages = kind == MmaKind::E4M3 ? 4 : 2;
+  const int kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
   size_t q = align_up((size_t)G * atoms * qcols * 128, 1024);
   size_t k = (size_t)kstages * atoms * 128 * 128;
-  return 1024 + q + k + sizeof(ScanSmemTail);
+  size_t h = (size_t)G * QG * kHistWords * sizeof(uint32_t);
+  return 1024 + q + k + h + sizeof(ScanSmemTail);
 }
 
 // H: heads scanned; n_q / n_k / batch: geometry; keep: entries kept per row.
@@ -55,34 +58,43 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.parts = split ? 2 : 1;
   pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   pl.atoms = pl.esz;
-  pl.kstages = kind == MmaKind::E4M3 ? 4 : 2;
+  pl.kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
   const int ncols_max = kind == MmaKind::TF32 ? 128 : 256;
   const int hp = H * pl.parts;
-  int qg_full = ncols_max / hp;
-  int qg_min = hp >= 16 ? 1 : 16 / hp;
-  int QG = qg_full;
+  int QG = ncols_max / hp;
+  const int qg_min = hp >= 16 ? 1 : 16 / hp;
   while (QG > qg_min && QG / 2 >= n_q) QG /= 2;  // few query rows (decode): shrink
-  if (QG > 1 && (QG & 1)) QG = 1;
+  int G = (kind == MmaKind::TF32 || QG == 1 || n_q <= QG) ? 1 : 2;
+#ifdef DSA_ONE_GROUP
+  G = 1;
+#endif
+  // fit the shared-memory budget and the per-item row limit
+  while (G * QG > kMaxRows || scan_smem_bytes(kind, G, QG, QG * hp) > kSmemBudget) {
+    if (G == 2) G = 1;
+    else if (QG > qg_min) QG /= 2;
+    else break;
+  }
   pl.QG = QG;
-  pl.G = (kind == MmaKind::TF32 || QG == 1 || n_q <= QG) ? 1 : 2;
+  pl.G = G;
   pl.qcols = QG * hp;
   pl.stage_cols = pl.qcols > 128 ? 256 : 128;
-  pl.n_qt = (n_q + QG * pl.G - 1) / (QG * pl.G);
+  pl.n_qt = (n_q + QG * G - 1) / (QG * G);
   pl.rows = batch * n_q;
-  pl.smem = scan_smem_bytes(kind, pl.G, pl.qcols);
+  pl.smem = scan_smem_bytes(kind, G, QG, pl.qcols);
   const size_t per_sm = 228 * 1024;
   int by_smem = (int)(per_sm / (pl.smem + 1024));
   int by_tmem = 512 / (2 * pl.stage_cols);
   pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
   if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
   if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
+  pl.nsub = QG == 1 ? 8 : 4;
   // split-K over keys when there are too few query tiles to fill the GPU
   const long long tiles = (long long)batch * pl.n_qt;
   int C = 1, chunk = 0;
   if (tiles < kTargetCtas && n_k > 4 * 128) {
     C = (int)(kTargetCtas / tiles);  // one round: batch * tiles * C <= target
     if (C < 1) C = 1;
-    if (C > kFinMaxSeg) C = kFinMaxSeg;
+    if (C * pl.nsub > kFinMaxSeg) C = kFinMaxSeg / pl.nsub;
     chunk = (n_k + C - 1) / C;
     chunk = (chunk + 127) / 128 * 128;
     if (chunk < 512) chunk = 512;
@@ -96,7 +108,7 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.chunk = chunk;
   pl.n_items = (int)(tiles * C);
   pl.keep = keep;
-  pl.cap = keep + (keep > 4096 ? keep : 4096) + 256;
+  pl.capw = 2 * keep + kCompactSlack + 128;
   return pl;
 }
 
@@ -137,10 +149,10 @@ bool make_map(CUtensorMap* m, const void* base, int esz, uint64_t rows, uint32_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <MmaKind K, bool S>
+template <MmaKind K, bool S, int HT>
 cudaError_t launch_scan_t(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
                           const ScanArgs& a, cudaStream_t st) {
-  auto kern = scan_kernel<K, S>;
+  auto kern = scan_kernel<K, S, HT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pl.smem);
   if (e != cudaSuccess) return e;
@@ -154,39 +166,78 @@ cudaError_t launch_scan_t(const ScanPlan& pl, const CUtensorMap& qm, const CUten
   return cudaGetLastError();
 }
 
-cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
-                        const ScanArgs& a, cudaStream_t st) {
-  switch (pl.kind) {
-    case MmaKind::TF32: return launch_scan_t<MmaKind::TF32, false>(pl, qm, km, a, st);
-    case MmaKind::BF16: return launch_scan_t<MmaKind::BF16, false>(pl, qm, km, a, st);
-    default:
-      return pl.split ? launch_scan_t<MmaKind::E4M3, true>(pl, qm, km, a, st)
-                      : launch_scan_t<MmaKind::E4M3, false>(pl, qm, km, a, st);
+template <MmaKind K, bool S>
+cudaError_t launch_scan_h(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
+                          const ScanArgs& a, cudaStream_t st) {
+  switch (a.H) {
+    case 8: return launch_scan_t<K, S, 8>(pl, qm, km, a, st);
+    case 16: return launch_scan_t<K, S, 16>(pl, qm, km, a, st);
+    case 32: return launch_scan_t<K, S, 32>(pl, qm, km, a, st);
+    case 64: return launch_scan_t<K, S, 64>(pl, qm, km, a, st);
+    default: return launch_scan_t<K, S, 128>(pl, qm, km, a, st);
   }
 }
 
-cudaError_t launch_finalize(int rows, int C, int topk, int cap, int sorted, const uint64_t* logs,
-                            const int32_t* cnt, const int32_t* buf, int32_t* out_idx,
+cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
+                        const ScanArgs& a, cudaStream_t st) {
+  switch (pl.kind) {
+    case MmaKind::TF32: return launch_scan_h<MmaKind::TF32, false>(pl, qm, km, a, st);
+    case MmaKind::BF16: return launch_scan_h<MmaKind::BF16, false>(pl, qm, km, a, st);
+    default:
+      if (pl.split) {
+        switch (a.H) {  // split-query path: heads >= 32
+          case 32: return launch_scan_t<MmaKind::E4M3, true, 32>(pl, qm, km, a, st);
+          case 64: return launch_scan_t<MmaKind::E4M3, true, 64>(pl, qm, km, a, st);
+          default: return launch_scan_t<MmaKind::E4M3, true, 128>(pl, qm, km, a, st);
+        }
+      }
+      return launch_scan_h<MmaKind::E4M3, false>(pl, qm, km, a, st);
+  }
+}
+
+cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint64_t* logs,
+                            const int32_t* cnt, const unsigned long long* thr, int32_t* out_idx,
                             float* out_score, cudaStream_t st) {
   FinalArgs f{};
-  f.rows = rows;
-  f.C = C;
+  f.rows = pl.rows;
+  f.C = pl.C;
+  f.nsub = pl.nsub;
   f.topk = topk;
-  f.cap = cap;
+  f.capw = pl.capw;
   int sc = 1;
   while (sc < topk) sc <<= 1;
   f.sort_cap = sc;
   f.sorted = sorted;
   f.logs = logs;
   f.log_cnt = cnt;
-  f.log_buf = buf;
+  f.log_thr = thr;
   f.out_idx = out_idx;
   f.out_score = out_score;
-  size_t smem = (size_t)sc * sizeof(uint64_t);
-  cudaError_t e =
-      cudaFuncSetAttribute(finalize_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
-  finalize_kernel<<<rows, kFinThreads, smem, st>>>(f);
+  cudaError_t e;
+  if (pl.C == 1) {
+    // one key chunk per row: about k candidates; four rows per CTA
+    const int stage_cap = sc + sc / 2;
+    const size_t per_group = ((size_t)sc + stage_cap) * sizeof(uint64_t);
+    int groups = (int)((160 * 1024) / per_group);
+    if (groups > kFinMaxGroups) groups = kFinMaxGroups;
+    if (groups < 1) groups = 1;
+    const size_t smem = per_group * groups;
+    e = cudaFuncSetAttribute(finalize_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    finalize_kernel<256><<<(pl.rows + groups - 1) / groups, 256 * groups, smem, st>>>(f, groups,
+                                                                                     stage_cap);
+  } else {
+    // split-K rows: about C * k candidates; one row per 1024-thread CTA
+    const size_t budget = 200 * 1024;
+    int stage_cap = (int)(budget / sizeof(uint64_t)) - sc;
+    if (stage_cap < sc) stage_cap = sc;
+    const size_t smem = ((size_t)sc + stage_cap) * sizeof(uint64_t);
+    e = cudaFuncSetAttribute(finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    finalize_kernel<1024><<<pl.rows, 1024, smem, st>>>(f, 1, stage_cap);
+  }
   return cudaGetLastError();
 }
 
@@ -241,7 +292,7 @@ void kind_of(const dsa_problem* p, MmaKind* kind, bool* split) {
 
 struct DsaLayout {
   ScanPlan pl;
-  size_t off_logs, off_cnt, off_buf, off_parts, off_hscale, total;
+  size_t off_logs, off_cnt, off_thr, off_parts, off_hscale, total;
 };
 
 DsaLayout dsa_layout(const dsa_problem* p) {
@@ -253,11 +304,11 @@ DsaLayout dsa_layout(const dsa_problem* p) {
   size_t off = kWsHeaderBytes;
   const size_t slots = (size_t)L.pl.rows * L.pl.C;
   L.off_logs = off;
-  off += align_up(slots * 2 * L.pl.cap * sizeof(uint64_t));
+  off += align_up(slots * L.pl.nsub * L.pl.capw * sizeof(uint64_t));
   L.off_cnt = off;
-  off += align_up(slots * sizeof(int32_t));
-  L.off_buf = off;
-  off += align_up(slots * sizeof(int32_t));
+  off += align_up(slots * L.pl.nsub * sizeof(int32_t));
+  L.off_thr = off;
+  off += align_up(slots * sizeof(unsigned long long));
   L.off_parts = off;
   if (split) off += align_up((size_t)L.pl.rows * 2 * p->heads * p->dim);
   L.off_hscale = off;
@@ -316,12 +367,12 @@ int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_param
   return DSA_ERR_UNSUPPORTED;
 }
 
-int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
-              const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
-              void* workspace, size_t workspace_bytes, void* stream) {
+int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+                   const float* k_scale, const float* w, void* workspace, size_t workspace_bytes,
+                   void* stream) {
   int v = validate_problem(p);
   if (v != DSA_OK) return v;
-  if (!q || !k || !w || !out_idx || !out_score) return DSA_ERR_INVALID;
+  if (!q || !k || !w) return DSA_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID;
   if (p->q_dtype == DSA_E4M3 && !q_scale) return DSA_ERR_INVALID;
   if (p->k_dtype == DSA_E4M3 && !k_scale) return DSA_ERR_INVALID;
@@ -376,16 +427,41 @@ int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const v
   a.row_scale = p->q_dtype == DSA_E4M3 ? q_scale : nullptr;
   a.head_scale = hscale;
   a.k_scale = p->k_dtype == DSA_E4M3 ? k_scale : nullptr;
+  a.nsub = pl.nsub;
+  a.capw = pl.capw;
   a.logs = reinterpret_cast<uint64_t*>(ws + L.off_logs);
   a.log_cnt = reinterpret_cast<int32_t*>(ws + L.off_cnt);
-  a.log_buf = reinterpret_cast<int32_t*>(ws + L.off_buf);
-  a.cap = pl.cap;
+  a.log_thr = reinterpret_cast<unsigned long long*>(ws + L.off_thr);
   a.status = status;
   if (launch_scan(pl, qm, km, a, st) != cudaSuccess) return DSA_ERR_CUDA;
-  if (launch_finalize(pl.rows, pl.C, p->topk, pl.cap, 1, a.logs, a.log_cnt, a.log_buf, out_idx,
+  return DSA_OK;
+}
+
+int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, void* workspace,
+                     size_t workspace_bytes, void* stream) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  if (!out_idx || !out_score) return DSA_ERR_INVALID;
+  const DsaLayout L = dsa_layout(p);
+  if (!workspace || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  const ScanPlan& pl = L.pl;
+  if (launch_finalize(pl, p->topk, 1, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
+                      reinterpret_cast<const int32_t*>(ws + L.off_cnt),
+                      reinterpret_cast<const unsigned long long*>(ws + L.off_thr), out_idx,
                       out_score, st) != cudaSuccess)
     return DSA_ERR_CUDA;
   return finish(p, workspace, st);
+}
+
+int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+              const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  if (p && (!out_idx || !out_score)) return DSA_ERR_INVALID;
+  int rc = dsa_index_scan(p, q, q_scale, k, k_scale, w, workspace, workspace_bytes, stream);
+  if (rc != DSA_OK) return rc;
+  return dsa_index_select(p, out_idx, out_score, workspace, workspace_bytes, stream);
 }
 
 int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* out,

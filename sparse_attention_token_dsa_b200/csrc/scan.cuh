@@ -11,13 +11,29 @@
 //
 // Layout of one CTA (persistent, one work item at a time):
 //   warps 0-7  epilogue: TMEM -> registers, ReLU, * w, sum over heads, causal
-//              mask, composite key, threshold filter, append to the row's
-//              candidate log; exact threshold raises when a log fills
+//              mask, composite key, threshold filter, append to warp-owned
+//              candidate sub-logs, per-row threshold maintenance
 //   warp 8     TMA producer: Q tile of the item (resident), K tiles streamed
 //   warp 9     MMA issuer (one thread) + TMEM allocator
 // MMA: M = 128 keys (TMEM lane = key), N = query rows x heads (x 2 for the
 // split-query fp8 form), K = d; fp32 accumulate in TMEM, two accumulator
 // stages so the epilogue of one unit overlaps the MMA of the next.
+//
+// Streaming top-k.  A candidate (score, key) is kept while its composite key
+// (order-preserving score bits, then ~index) is >= the row's threshold thr.
+// thr is always a lower bound of the row's final keep-th best composite, so no
+// winner is ever dropped.  It is raised every step from per-row histograms of
+// the kept candidates: h1 counts them by the top byte of the 32-bit score key;
+// h2[0] / h2[1] count those whose top byte equals b1 / b1 + 1 by the second
+// byte, where b1 is the top-byte bin holding the keep-th best.  The pair gives
+// thr at 16-bit score-key resolution (bf16 precision) without rescanning the
+// logs (a first threshold, or a jump of b1 by more than one, rebuilds h2 from
+// the logs).  Counts can only be low (never high) in the bins the search
+// reaches, which can only make thr looser, never invalid.  Each epilogue warp
+// appends to its own sub-log per row (no atomics) and compacts it in place
+// (keep >= thr) when it nears capacity; if that is not enough (long runs of
+// tied scores) an exact radix-select raise sets thr to the keep-th best
+// composite itself.
 #pragma once
 #include "common.cuh"
 #include "select.cuh"
@@ -40,10 +56,11 @@ struct ScanArgs {
   const float* row_scale;   // [rows] or null: multiplies w (query dequant scale)
   const float* head_scale;  // [rows, H] or null: multiplies w (split-query part scale)
   const float* k_scale;     // [batch * n_k] or null: multiplies the score (key dequant scale)
-  uint64_t* logs;        // [rows * C][2][cap] composite keys
-  int32_t* log_cnt;      // [rows * C]
-  int32_t* log_buf;      // [rows * C]
-  int32_t cap;           // entries per log buffer (>= keep + 256)
+  int32_t nsub;          // sub-logs per row slot (4: one per lane quadrant; 8: one per warp)
+  int32_t capw;          // entries per sub-log (>= keep + 256)
+  uint64_t* logs;        // [rows * C][nsub][capw] composite keys
+  int32_t* log_cnt;      // [rows * C][nsub]
+  unsigned long long* log_thr;  // [rows * C] final threshold of the slot
   int32_t* status;       // workspace status word
 };
 
@@ -52,16 +69,26 @@ constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kScanThreads = 320;
-constexpr int kMaxRows = 64;          // rows per work item
+constexpr int kMaxRows = 16;          // rows per work item
 constexpr int kMaxItemCols = 512;     // rows x heads per item
 constexpr int kBarEpi = 1;            // named barrier among the epilogue warps
+constexpr int kHistWords = 768;       // h1[256] + h2[2][256] per row
+constexpr int kUpdateSteps = 4;       // steps (key tiles) between threshold updates
+// Sub-log slack: a step appends at most 64 entries per row to one sub-log, and a
+// flagged row waits at most two update periods (8 steps) for its exact raise.
+constexpr int kCompactSlack = 640;
+
+#ifndef DSA_BF16_KSTAGES
+#define DSA_BF16_KSTAGES 2   // K-tile pipeline depth for bf16 operands
+#endif
 
 template <MmaKind KIND>
 struct ScanCfg {
   static constexpr int ESZ = KIND == MmaKind::TF32 ? 4 : (KIND == MmaKind::BF16 ? 2 : 1);
   static constexpr int A = 128 * ESZ / 128;   // 128-byte atoms per key row (d = 128)
   static constexpr int EPA = 128 / ESZ;       // elements per atom
-  static constexpr int KSTAGES = KIND == MmaKind::E4M3 ? 4 : 2;
+  static constexpr int KSTAGES =
+      KIND == MmaKind::E4M3 ? 4 : (KIND == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
   static constexpr int KTILE_BYTES = A * 128 * 128;
 };
 
@@ -73,9 +100,12 @@ struct ScanSmemTail {
   uint32_t tmem_base;
   int32_t abort;
   int32_t epi_stop[2];
-  int32_t row_cnt[kMaxRows];
-  int32_t row_buf[kMaxRows];
-  int32_t row_pos[kMaxRows];   // causal position (-1: row absent)
+  int32_t raise_snap[2];
+  int32_t row_nleg[kMaxRows];  // legal keys of the row in this item, counted from kbeg
+  int32_t row_b1[kMaxRows];    // top-byte bin of the keep-th best (-1: fewer kept)
+  int32_t row_raise[kMaxRows]; // a sub-log could not be compacted enough
+  int32_t raise_any;           // some row needs an exact raise
+  int32_t subcnt[kMaxRows][8]; // sub-log fill, written only by the owning warp
   unsigned long long row_thr[kMaxRows];
   alignas(16) float wsm[kMaxItemCols];
   SelectScratch sel;
@@ -87,13 +117,11 @@ struct ItemGeom {
 
 __device__ __forceinline__ ItemGeom item_geom(const ScanArgs& a, int item) {
   ItemGeom g;
-  const int per_b = a.n_qt * a.C;
   const int qt_rev = item / (a.batch * a.C);
   const int rem = item % (a.batch * a.C);
   g.b = rem / a.C;
   g.c = rem % a.C;
   g.qt = a.n_qt - 1 - qt_rev;
-  (void)per_b;
   const int QT = a.QG * a.G;
   g.row0 = g.qt * QT;
   g.nrows = min(QT, a.n_q - g.row0);
@@ -124,19 +152,272 @@ __device__ __forceinline__ int sched_item(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
-template <MmaKind KIND, bool SPLIT>
+// Warp-wide search over 256 histogram bins (lane l owns bins 255-8l .. 248-8l):
+// the highest bin b with base + (count of bins >= b) >= need.  Returns the bin
+// (-1 when the total stays below need) and, in *above, base + count strictly
+// above it.
+__device__ __forceinline__ int hist_find(const uint32_t* h, int base, int need, int lane,
+                                         int* above) {
+  int c[8];
+  int tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = (int)h[255 - 8 * lane - i];
+    tot += c[i];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const int excl = incl - tot;
+  const bool mine = base + excl < need && need <= base + incl;
+  const unsigned bal = __ballot_sync(0xffffffffu, mine);
+  if (!bal) {
+    *above = 0;
+    return -1;
+  }
+  const int src = __ffs(bal) - 1;
+  int bin = 0, ab = 0;
+  if (lane == src) {
+    int cum = base + excl;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (cum + c[i] >= need) {
+        bin = 255 - 8 * lane - i;
+        ab = cum;
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  *above = __shfl_sync(0xffffffffu, ab, src);
+  return __shfl_sync(0xffffffffu, bin, src);
+}
+
+// In-place warp compaction of one sub-log: keep entries >= thr; returns the
+// count.  Eight independent loads per lane are in flight per round.
+__device__ __forceinline__ int compact_sublog(uint64_t* lg, int n, unsigned long long thr,
+                                              int lane) {
+  int wpos = 0;
+  for (int i0 = 0; i0 < n; i0 += 256) {
+    uint64_t vv[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * 32 + lane;
+      vv[j] = i < n ? lg[i] : 0ull;
+    }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * 32 + lane;
+      const bool kp = i < n && vv[j] >= thr;
+      const unsigned bal = __ballot_sync(0xffffffffu, kp);
+      if (kp) lg[wpos + __popc(bal & ((1u << lane) - 1))] = vv[j];
+      wpos += __popc(bal);
+    }
+    __syncwarp();
+  }
+  return wpos;
+}
+
+// Fine-histogram rebuild from one sub-log (entries whose top byte is b1 or b1+1).
+__device__ __forceinline__ void rebuild_fine(uint32_t* h, const uint64_t* lg, int n, int b1,
+                                             int lane) {
+  for (int i0 = 0; i0 < n; i0 += 256) {
+    uint32_t sk[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * 32 + lane;
+      sk[j] = i < n ? (uint32_t)(lg[i] >> 32) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int i = i0 + j * 32 + lane;
+      const int d1 = (int)(sk[j] >> 24) - b1;
+      if (i < n && (d1 == 0 || d1 == 1)) atomicAdd(&h[256 + d1 * 256 + ((sk[j] >> 16) & 255)], 1u);
+    }
+  }
+}
+
+// Per-unit context of the filter: the lane's key, its dequant scale, and where
+// this warp's sub-logs and the row histograms live.
+struct FilterCtx {
+  int key;
+  float ks;
+  int kbeg;
+  int lane;
+  unsigned lanemask_lt;
+  int sub;
+  uint64_t* logs;        // this warp's sub-log of item row 0
+  int64_t row_stride;    // entries between consecutive rows' sub-logs
+  uint32_t* hist;
+  ScanSmemTail* T;
+};
+
+// Legality, composite key, threshold filter and append for one query row.
+// The common path (no lane survives) costs one limit load, one threshold load,
+// the key arithmetic and a vote.
+__device__ __forceinline__ void filter_append(const FilterCtx& f, int r, float acc) {
+  ScanSmemTail* T = f.T;
+  const uint32_t sk = score_key(acc * f.ks);
+  const uint64_t comp = ((uint64_t)sk << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)f.key);
+  const bool surv = (unsigned)(f.key - f.kbeg) < (unsigned)T->row_nleg[r] && comp >= T->row_thr[r];
+  const unsigned bal = __ballot_sync(0xffffffffu, surv);
+  if (bal) {
+    int* cnt = &T->subcnt[r][f.sub];
+    const int base = *cnt;
+    if (surv) {
+      f.logs[r * f.row_stride + base + __popc(bal & f.lanemask_lt)] = comp;
+      uint32_t* h = f.hist + r * kHistWords;
+      const int b1 = (int)(sk >> 24);
+      atomicAdd(&h[b1], 1u);
+      const unsigned d1 = (unsigned)(b1 - T->row_b1[r]);
+      if (d1 <= 1u) atomicAdd(&h[256 + d1 * 256 + ((sk >> 16) & 255)], 1u);
+    }
+    __syncwarp();
+    if (f.lane == 0) *cnt = base + __popc(bal);
+    __syncwarp();
+  }
+}
+
+// Packed fp32 pair FMA (sm_100a): acc.{x,y} += w.{x,y} * {a, b}, each lane an
+// IEEE round-to-nearest fma, identical to two scalar fmaf.
+__device__ __forceinline__ void ffma2(unsigned long long& acc, unsigned long long w, float a,
+                                      float b) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(r));
+}
+__device__ __forceinline__ float pair_sum(unsigned long long v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
+
+// sum_j w_j ReLU(v_j) over NC 32-column chunks into four packed partial sums.
+template <int NC>
+__device__ __forceinline__ void relu_dot(const uint32_t (&v)[NC][32], const float* w,
+                                         unsigned long long (&acc)[4]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+#pragma unroll
+    for (int jj = 0; jj < 32; jj += 4) {
+      const ulonglong2 wv = *reinterpret_cast<const ulonglong2*>(w + c * 32 + jj);
+      const int o = (jj >> 2) & 1;
+      ffma2(acc[2 * o + 0], wv.x, fmaxf(__uint_as_float(v[c][jj + 0]), 0.f),
+            fmaxf(__uint_as_float(v[c][jj + 1]), 0.f));
+      ffma2(acc[2 * o + 1], wv.y, fmaxf(__uint_as_float(v[c][jj + 2]), 0.f),
+            fmaxf(__uint_as_float(v[c][jj + 3]), 0.f));
+    }
+  }
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_chunks(uint32_t taddr, uint32_t (&v)[NC][32]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) tmem_ld32(taddr + c * 32, v[c]);
+}
+template <int NC>
+__device__ __forceinline__ void tmem_wait_chunks(uint32_t (&v)[NC][32]) {
+#pragma unroll
+  for (int c = 0; c < NC; ++c) tmem_ld_wait(v[c]);
+}
+
+__device__ __forceinline__ float sum8(const unsigned long long (&a)[4]) {
+  return (pair_sum(a[0]) + pair_sum(a[1])) + (pair_sum(a[2]) + pair_sum(a[3]));
+}
+
+// One unit of this warp: nq query rows of HT heads starting at TMEM column
+// address `col` (row r = rbase + i, weights w + i * HT).  Work is split into
+// segments of at most 64 columns; the TMEM loads of segment i+1 are in flight
+// while segment i is reduced.
+template <int HT>
+__device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, const float* w,
+                                           int nq, int rbase) {
+  if constexpr (HT >= 32) {
+    constexpr int SEGC = 1;                       // 32-column chunks per segment
+    constexpr int SPQ = HT / (32 * SEGC);          // segments per query row
+    const int nseg = nq * SPQ;
+    uint32_t va[SEGC][32], vb[SEGC][32];
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+    tmem_ld_chunks<SEGC>(col, va);
+    tmem_wait_chunks<SEGC>(va);
+    for (int sg = 0; sg < nseg; sg += 2) {
+      const bool has_b = sg + 1 < nseg;
+      if (has_b) tmem_ld_chunks<SEGC>(col + (sg + 1) * 32 * SEGC, vb);
+      relu_dot<SEGC>(va, w + sg * 32 * SEGC, acc);
+      if ((sg + 1) % SPQ == 0) {
+        filter_append(f, rbase + sg / SPQ, sum8(acc));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = 0ull;
+      }
+      if (!has_b) break;
+      tmem_wait_chunks<SEGC>(vb);
+      if (sg + 2 < nseg) tmem_ld_chunks<SEGC>(col + (sg + 2) * 32 * SEGC, va);
+      relu_dot<SEGC>(vb, w + (sg + 1) * 32 * SEGC, acc);
+      if ((sg + 2) % SPQ == 0) {
+        filter_append(f, rbase + (sg + 1) / SPQ, sum8(acc));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = 0ull;
+      }
+      if (sg + 2 < nseg) tmem_wait_chunks<SEGC>(va);
+    }
+  } else {
+    // HT in {8, 16}: one 32-column chunk holds 32 / HT query rows
+    constexpr int QPC = 32 / HT;
+    const int nchunk = nq / QPC;
+    uint32_t va[1][32], vb[1][32];
+    auto chunk = [&](const uint32_t (&v)[1][32], int c) {
+#pragma unroll
+      for (int qq = 0; qq < QPC; ++qq) {
+        float b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int jj = 0; jj < HT; jj += 4) {
+          const float4 wv = *reinterpret_cast<const float4*>(w + c * 32 + qq * HT + jj);
+          b[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[0][qq * HT + jj + 0]), 0.f), b[0]);
+          b[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[0][qq * HT + jj + 1]), 0.f), b[1]);
+          b[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[0][qq * HT + jj + 2]), 0.f), b[2]);
+          b[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[0][qq * HT + jj + 3]), 0.f), b[3]);
+        }
+        filter_append(f, rbase + c * QPC + qq, (b[0] + b[1]) + (b[2] + b[3]));
+      }
+    };
+    tmem_ld_chunks<1>(col, va);
+    tmem_wait_chunks<1>(va);
+    for (int c = 0; c < nchunk; c += 2) {
+      const bool has_b = c + 1 < nchunk;
+      if (has_b) tmem_ld_chunks<1>(col + (c + 1) * 32, vb);
+      chunk(va, c);
+      if (!has_b) break;
+      tmem_wait_chunks<1>(vb);
+      if (c + 2 < nchunk) tmem_ld_chunks<1>(col + (c + 2) * 32, va);
+      chunk(vb, c + 1);
+      if (c + 2 < nchunk) tmem_wait_chunks<1>(va);
+    }
+  }
+}
+
+// 320 threads: ten warps over four sub-partitions of 16K registers each allow
+// at most 168 registers per thread.
+template <MmaKind KIND, bool SPLIT, int HT>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const ScanArgs a) {
   using Cfg = ScanCfg<KIND>;
   constexpr int PARTS = SPLIT ? 2 : 1;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base; plain pointer arithmetic on the __shared__ array
+  // keeps the shared address space visible to the compiler (LDS/ATOMS, not generic)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int qcols = a.QG * a.H * PARTS;                     // MMA N per group
+  const int QT = a.QG * a.G;
   uint8_t* Qs = smem;                                       // [G][A][qcols x 128B]
   const int q_bytes = a.G * Cfg::A * qcols * 128;
   uint8_t* Ks = smem + ((q_bytes + 1023) & ~1023);          // [KSTAGES][A][128 x 128B]
-  ScanSmemTail* T = reinterpret_cast<ScanSmemTail*>(Ks + Cfg::KSTAGES * Cfg::KTILE_BYTES);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + Cfg::KSTAGES * Cfg::KTILE_BYTES);  // [QT][768]
+  ScanSmemTail* T = reinterpret_cast<ScanSmemTail*>(hist + QT * kHistWords);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool modeB = (a.QG == 1);  // one query per group: halves take alternate stages
@@ -169,9 +450,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = T->tmem_base;
   volatile int* abort = &T->abort;
-
   const int grid = gridDim.x;
-  const int QT = a.QG * a.G;
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer --
@@ -227,7 +506,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         tc_fence_after();
         const int nunits = g.ntiles * a.G;
         for (int u = 0; u < nunits; ++u) {
-          const int gg = u % a.G;
+          const int gg = u & (a.G - 1);
           const int slot = kcount % Cfg::KSTAGES;
           if (gg == 0) {
             if (!mbar_wait(&T->k_full[slot], (kcount / Cfg::KSTAGES) & 1, abort, a.status, 4)) { ok = false; break; }
@@ -268,7 +547,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     const int etid = threadIdx.x;              // 0..255
     const int quad = warp & 3;                 // TMEM lane quadrant
     const int half = warp >> 2;                // column half / stage (mode B)
-    const int H = a.H;
+    const int sub = modeB ? warp : quad;       // this warp's sub-log index
+    constexpr int H = HT;
+    const int hshift = 31 - __clz(H);          // log2(H)
+    const int qhalf = modeB ? 1 : (a.QG >> 1); // query rows per warp per group
     uint32_t ucount = 0;
     int step_par = 0;
     bool stop = false;
@@ -278,15 +560,20 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       ItemGeom g = item_geom(a, item);
       const int pos0 = a.q_pos0 ? a.q_pos0[g.b] : a.n_k - a.n_q;
       const int klen = a.k_len ? a.k_len[g.b] : a.n_k;
-      // ---- item init: row states and head weights
+      const int64_t slot0 = ((int64_t)g.b * a.n_q + g.row0) * a.C + g.c;  // slot of row 0
+      // ---- item init: row states, histograms, head weights
       for (int r = etid; r < QT; r += kEpiThreads) {
-        T->row_cnt[r] = 0;
-        T->row_buf[r] = 0;
         T->row_thr[r] = 0ull;
-        T->row_pos[r] = (r < g.nrows) ? pos0 + g.row0 + r : -1;
+        T->row_b1[r] = -1;
+        T->row_raise[r] = 0;
+        T->row_nleg[r] =
+            (r < g.nrows) ? max(0, min(min(pos0 + g.row0 + r, klen - 1), g.kend - 1) - g.kbeg + 1) : 0;
+#pragma unroll
+        for (int w8 = 0; w8 < 8; ++w8) T->subcnt[r][w8] = 0;
       }
+      for (int i = etid; i < QT * kHistWords; i += kEpiThreads) hist[i] = 0u;
       for (int i = etid; i < QT * H; i += kEpiThreads) {
-        const int r = i / H, j = i % H;
+        const int r = i >> hshift, j = i & (H - 1);
         float wv = 0.f;
         if (r < g.nrows) {
           const int64_t grow = (int64_t)g.b * a.n_q + g.row0 + r;
@@ -296,9 +583,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
         T->wsm[i] = wv;
       }
+      if (etid == 0) T->raise_any = 0;
       named_bar_sync(kBarEpi, kEpiThreads);
       const int nunits = g.ntiles * a.G;
       int u = 0;
+      int steps = 0;
       while (u < nunits) {
         // one step = up to two units (stage 0 / stage 1)
         const int nstep = min(2, nunits - u);
@@ -312,110 +601,52 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
           tc_fence_after();
-          const int gg = uu % a.G;
-          const int t = uu / a.G;
+          const int gg = uu & (a.G - 1);
+          const int t = uu >> (a.G - 1);
           const int key = ((g.t_hi - t) << 7) + quad * 32 + lane;
           float ks = 1.f;
           if (a.k_scale && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
           const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + s * a.stage_cols;
           // queries handled by this warp inside group gg
-          const int qbeg = modeB ? 0 : half * (a.QG >> 1);
-          const int qnum = modeB ? 1 : (a.QG >> 1);
+          const int qbeg = modeB ? 0 : half * qhalf;
           const int rbase = gg * a.QG + qbeg;          // first item row of this warp
-          // legality, composite key, threshold filter, append (one query row)
-          auto finish = [&](int r, float score) {
-            score *= ks;
-            const int pos = T->row_pos[r];
-            const bool legal = pos >= 0 && key <= pos && key < klen && key >= g.kbeg && key < g.kend;
-            const uint64_t comp = make_comp(score, key);
-            const bool surv = legal && comp >= T->row_thr[r];
-            const unsigned bal = __ballot_sync(0xffffffffu, surv);
-            if (bal) {
-              int base = 0;
-              const int leader = __ffs(bal) - 1;
-              if (lane == leader) base = atomicAdd(&T->row_cnt[r], __popc(bal));
-              base = __shfl_sync(0xffffffffu, base, leader);
-              if (surv) {
-                const int slot = base + __popc(bal & ((1u << lane) - 1));
-                const int64_t rs = ((int64_t)g.b * a.n_q + g.row0 + r) * a.C + g.c;
-                a.logs[(rs * 2 + T->row_buf[r]) * a.cap + slot] = comp;
-              }
-            }
-          };
-          if (H >= 32) {
-            for (int qi = 0; qi < qnum; ++qi) {
+          FilterCtx fc;
+          fc.key = key;
+          fc.ks = ks;
+          fc.kbeg = g.kbeg;
+          fc.lane = lane;
+          fc.lanemask_lt = (1u << lane) - 1u;
+          fc.sub = sub;
+          fc.logs = a.logs + (slot0 * a.nsub + sub) * a.capw;
+          fc.row_stride = (int64_t)a.C * a.nsub * a.capw;
+          fc.hist = hist;
+          fc.T = T;
+          if constexpr (SPLIT) {
+            for (int qi = 0; qi < qhalf; ++qi) {
               const int r = rbase + qi;
-              const float* wr = &T->wsm[r * H];
-              const uint32_t cb = taddr + (qbeg + qi) * H * PARTS;
+              const float* wr = &T->wsm[r * HT];
+              const uint32_t cb = taddr + (qbeg + qi) * HT * PARTS;
               float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-              for (int c0 = 0; c0 < H; c0 += 32) {
-                uint32_t v0[32];
+#pragma unroll
+              for (int c0 = 0; c0 < HT; c0 += 32) {
+                uint32_t v0[32], v1[32];
                 tmem_ld32(cb + c0, v0);
-                if constexpr (SPLIT) {
-                  uint32_t v1[32];
-                  tmem_ld32(cb + H + c0, v1);
-                  tmem_ld_wait();
+                tmem_ld32(cb + HT + c0, v1);
+                tmem_ld_wait(v0);
+                tmem_ld_wait(v1);
 #pragma unroll
-                  for (int jj = 0; jj < 32; jj += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(wr + c0 + jj);
-                    acc0 = fmaf(wv.x, fmaxf(fmaf(__uint_as_float(v1[jj + 0]), 0.0625f, __uint_as_float(v0[jj + 0])), 0.f), acc0);
-                    acc1 = fmaf(wv.y, fmaxf(fmaf(__uint_as_float(v1[jj + 1]), 0.0625f, __uint_as_float(v0[jj + 1])), 0.f), acc1);
-                    acc2 = fmaf(wv.z, fmaxf(fmaf(__uint_as_float(v1[jj + 2]), 0.0625f, __uint_as_float(v0[jj + 2])), 0.f), acc2);
-                    acc3 = fmaf(wv.w, fmaxf(fmaf(__uint_as_float(v1[jj + 3]), 0.0625f, __uint_as_float(v0[jj + 3])), 0.f), acc3);
-                  }
-                } else {
-                  tmem_ld_wait();
-#pragma unroll
-                  for (int jj = 0; jj < 32; jj += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(wr + c0 + jj);
-                    acc0 = fmaf(wv.x, fmaxf(__uint_as_float(v0[jj + 0]), 0.f), acc0);
-                    acc1 = fmaf(wv.y, fmaxf(__uint_as_float(v0[jj + 1]), 0.f), acc1);
-                    acc2 = fmaf(wv.z, fmaxf(__uint_as_float(v0[jj + 2]), 0.f), acc2);
-                    acc3 = fmaf(wv.w, fmaxf(__uint_as_float(v0[jj + 3]), 0.f), acc3);
-                  }
+                for (int jj = 0; jj < 32; jj += 4) {
+                  const float4 wv = *reinterpret_cast<const float4*>(wr + c0 + jj);
+                  acc0 = fmaf(wv.x, fmaxf(fmaf(__uint_as_float(v1[jj + 0]), 0.0625f, __uint_as_float(v0[jj + 0])), 0.f), acc0);
+                  acc1 = fmaf(wv.y, fmaxf(fmaf(__uint_as_float(v1[jj + 1]), 0.0625f, __uint_as_float(v0[jj + 1])), 0.f), acc1);
+                  acc2 = fmaf(wv.z, fmaxf(fmaf(__uint_as_float(v1[jj + 2]), 0.0625f, __uint_as_float(v0[jj + 2])), 0.f), acc2);
+                  acc3 = fmaf(wv.w, fmaxf(fmaf(__uint_as_float(v1[jj + 3]), 0.0625f, __uint_as_float(v0[jj + 3])), 0.f), acc3);
                 }
               }
-              finish(r, (acc0 + acc1) + (acc2 + acc3));
+              filter_append(fc, r, (acc0 + acc1) + (acc2 + acc3));
             }
-          } else if constexpr (!SPLIT) {
-            // H in {8, 16}: a 32-column load covers 32 / H query rows
-            const int ncol = qnum * H;                  // multiple of 32
-            for (int c = 0; c < ncol; c += 32) {
-              uint32_t v0[32];
-              tmem_ld32(taddr + qbeg * H + c, v0);
-              tmem_ld_wait();
-              const float* wr = &T->wsm[rbase * H + c];
-              const int r0 = rbase + c / H;
-              if (H == 16) {
-#pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
-                  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-                  for (int jj = 0; jj < 16; jj += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(wr + qq * 16 + jj);
-                    acc0 = fmaf(wv.x, fmaxf(__uint_as_float(v0[qq * 16 + jj + 0]), 0.f), acc0);
-                    acc1 = fmaf(wv.y, fmaxf(__uint_as_float(v0[qq * 16 + jj + 1]), 0.f), acc1);
-                    acc2 = fmaf(wv.z, fmaxf(__uint_as_float(v0[qq * 16 + jj + 2]), 0.f), acc2);
-                    acc3 = fmaf(wv.w, fmaxf(__uint_as_float(v0[qq * 16 + jj + 3]), 0.f), acc3);
-                  }
-                  finish(r0 + qq, (acc0 + acc1) + (acc2 + acc3));
-                }
-              } else {
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll
-                  for (int jj = 0; jj < 8; jj += 4) {
-                    const float4 wv = *reinterpret_cast<const float4*>(wr + qq * 8 + jj);
-                    acc0 = fmaf(wv.x, fmaxf(__uint_as_float(v0[qq * 8 + jj + 0]), 0.f), acc0);
-                    acc1 = fmaf(wv.y, fmaxf(__uint_as_float(v0[qq * 8 + jj + 1]), 0.f), acc1);
-                    acc2 = fmaf(wv.z, fmaxf(__uint_as_float(v0[qq * 8 + jj + 2]), 0.f), acc2);
-                    acc3 = fmaf(wv.w, fmaxf(__uint_as_float(v0[qq * 8 + jj + 3]), 0.f), acc3);
-                  }
-                  finish(r0 + qq, (acc0 + acc1) + (acc2 + acc3));
-                }
-              }
-            }
+          } else {
+            unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
           }
           tc_fence_before();
           __syncwarp();
@@ -423,36 +654,113 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         }
         ucount += nstep;
         u += nstep;
-        // uniform stop decision: thread 0 snapshots the abort flag before the barrier
-        if (etid == 0) T->epi_stop[step_par] = *abort;
+        ++steps;
+        // ---- compaction of this warp's own sub-logs that near capacity (no barrier:
+        // only this warp writes them; thr may be raised concurrently, which only
+        // keeps fewer entries, all still >= a valid threshold)
+        for (int gg = 0; gg < a.G; ++gg) {
+          for (int qi = 0; qi < qhalf; ++qi) {
+            const int r = gg * a.QG + (modeB ? 0 : half * qhalf) + qi;
+            if (r >= g.nrows) continue;
+            const int n = T->subcnt[r][sub];
+            if (n <= a.capw - kCompactSlack) continue;
+            uint64_t* lg = a.logs + ((slot0 + (int64_t)r * a.C) * a.nsub + sub) * a.capw;
+            const int kept = compact_sublog(lg, n, T->row_thr[r], lane);
+            if (lane == 0) {
+              T->subcnt[r][sub] = kept;
+              if (kept > a.capw - kCompactSlack) T->raise_any = T->row_raise[r] = 1;
+            }
+            __syncwarp();
+          }
+        }
+        // ---- every kUpdateSteps steps (and at the item end): threshold update
+        const bool last = u >= nunits;
+        if (!last && (steps & (kUpdateSteps - 1)) != 0) continue;
+        // uniform decisions: thread 0 snapshots the abort and raise flags before the
+        // barrier (a raise flagged after the snapshot waits for the next update)
+        if (etid == 0) {
+          T->epi_stop[step_par] = *abort;
+          T->raise_snap[step_par] = T->raise_any;
+        }
         named_bar_sync(kBarEpi, kEpiThreads);
         stop = T->epi_stop[step_par] != 0;
+        const bool do_raise = T->raise_snap[step_par] != 0;
         step_par ^= 1;
         if (stop) break;
-        // ---- exact threshold raises for rows whose log is nearly full
+        // one warp per row, from the row's histograms
+        for (int r = warp; r < g.nrows; r += kEpiWarps) {
+          uint32_t* h = hist + r * kHistWords;
+          int above1;
+          const int nb1 = hist_find(h, 0, a.keep, lane, &above1);
+          if (nb1 < 0) continue;                           // fewer than keep kept so far
+          const int ob1 = T->row_b1[r];
+          if (nb1 != ob1) {
+            if (ob1 >= 0 && nb1 == ob1 + 1) {
+              // the upper fine histogram becomes the lower one
+              for (int i = lane; i < 256; i += 32) {
+                h[256 + i] = h[512 + i];
+                h[512 + i] = 0u;
+              }
+            } else {
+              // first threshold or a jump: rebuild both fine histograms from the sub-logs
+              for (int i = lane; i < 512; i += 32) h[256 + i] = 0u;
+              __syncwarp();
+              const int64_t rs = slot0 + (int64_t)r * a.C;
+              for (int sb = 0; sb < a.nsub; ++sb)
+                rebuild_fine(h, a.logs + (rs * a.nsub + sb) * a.capw, T->subcnt[r][sb], nb1, lane);
+            }
+            __syncwarp();
+            if (lane == 0) T->row_b1[r] = nb1;
+          }
+          __syncwarp();
+          int above2;
+          const int b2 = hist_find(h + 256, above1, a.keep, lane, &above2);
+          if (b2 >= 0 && lane == 0) {
+            const unsigned long long thr =
+                (unsigned long long)(((uint32_t)nb1 << 24) | ((uint32_t)b2 << 16)) << 32;
+            if (thr > T->row_thr[r]) T->row_thr[r] = thr;
+          }
+          __syncwarp();
+        }
+        named_bar_sync(kBarEpi, kEpiThreads);
+        if (!do_raise) continue;
+        // ---- exact raise (rare: long runs of tied scores)
         for (int r = 0; r < g.nrows; ++r) {
-          if (T->row_cnt[r] <= a.cap - 256) continue;
-          const int64_t rs = ((int64_t)g.b * a.n_q + g.row0 + r) * a.C + g.c;
-          const int cur = T->row_buf[r];
-          const uint64_t* src = a.logs + (rs * 2 + cur) * a.cap;
-          uint64_t* dst = a.logs + (rs * 2 + (cur ^ 1)) * a.cap;
-          const int n = T->row_cnt[r];
-          const uint64_t pfx = radix_select<kEpiThreads>(&src, &n, 1, a.keep, &T->sel, etid, kBarEpi);
-          uint64_t kmin;
-          const int kept = compact_ge<kEpiThreads>(&src, &n, 1, pfx, dst, &T->sel, etid, kBarEpi, &kmin);
-          if (etid == 0) {
-            T->row_cnt[r] = kept;
-            T->row_buf[r] = cur ^ 1;
-            T->row_thr[r] = kmin + 1;
+          if (!T->row_raise[r]) continue;
+          const int64_t rs = slot0 + (int64_t)r * a.C;
+          const uint64_t* segs[8];
+          int segn[8];
+          int total = 0;
+          for (int sb = 0; sb < a.nsub; ++sb) {
+            segs[sb] = a.logs + (rs * a.nsub + sb) * a.capw;
+            segn[sb] = T->subcnt[r][sb];
+            total += segn[sb];
+          }
+          if (total > a.keep) {
+            const uint64_t pfx = radix_select<kEpiThreads>(segs, segn, a.nsub, a.keep, &T->sel, etid, kBarEpi);
+            if (etid == 0 && pfx > T->row_thr[r]) T->row_thr[r] = pfx;
           }
           named_bar_sync(kBarEpi, kEpiThreads);
+          // the owners of row r's sub-logs compact them with the new threshold
+          const bool owner = modeB || ((r % a.QG) / qhalf == half);
+          if (owner && T->subcnt[r][sub] > 0) {
+            uint64_t* lg = a.logs + (rs * a.nsub + sub) * a.capw;
+            const int kept = compact_sublog(lg, T->subcnt[r][sub], T->row_thr[r], lane);
+            if (lane == 0) T->subcnt[r][sub] = kept;
+            __syncwarp();
+          }
+          named_bar_sync(kBarEpi, kEpiThreads);
+          if (etid == 0) T->row_raise[r] = 0;
+          named_bar_sync(kBarEpi, kEpiThreads);
         }
+        if (etid == 0) T->raise_any = 0;
+        named_bar_sync(kBarEpi, kEpiThreads);
       }
-      // ---- item end: publish log state of every row
+      // ---- item end: publish sub-log fills and thresholds
       for (int r = etid; r < g.nrows; r += kEpiThreads) {
-        const int64_t rs = ((int64_t)g.b * a.n_q + g.row0 + r) * a.C + g.c;
-        a.log_cnt[rs] = T->row_cnt[r];
-        a.log_buf[rs] = T->row_buf[r];
+        const int64_t rs = slot0 + (int64_t)r * a.C;
+        for (int sb = 0; sb < a.nsub; ++sb) a.log_cnt[rs * a.nsub + sb] = T->subcnt[r][sb];
+        a.log_thr[rs] = T->row_thr[r];
       }
       if (etid == 0) T->epi_stop[step_par] = *abort;
       named_bar_sync(kBarEpi, kEpiThreads);

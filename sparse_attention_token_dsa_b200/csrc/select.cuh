@@ -29,12 +29,21 @@ __device__ uint64_t radix_select(const uint64_t* const* seg, const int* seg_n, i
   for (int shift = 56; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += NTHR) sc->hist[i] = 0;
     named_bar_sync(bar_id, NTHR);
+    // histogram of the next digit; lanes sharing a bin add once (one atomic per
+    // distinct bin per warp: candidates cluster in very few bins)
     for (int g = 0; g < nseg; ++g) {
       const uint64_t* p = seg[g];
       const int n = seg_n[g];
-      for (int i = tid; i < n; i += NTHR) {
-        uint64_t v = p[i];
-        if ((v & mask) == prefix) atomicAdd(&sc->hist[(int)((v >> shift) & 255)], 1);
+      for (int i0 = 0; i0 < n; i0 += NTHR) {
+        const int i = i0 + tid;
+        const uint64_t v = i < n ? p[i] : 0ull;
+        const bool m = i < n && (v & mask) == prefix;
+        const unsigned act = __ballot_sync(0xffffffffu, m);
+        if (m) {
+          const int bin = (int)((v >> shift) & 255);
+          const unsigned peers = __match_any_sync(act, bin);
+          if ((tid & 31) == __ffs(peers) - 1) atomicAdd(&sc->hist[bin], __popc(peers));
+        }
       }
     }
     named_bar_sync(bar_id, NTHR);
@@ -81,7 +90,8 @@ __device__ uint64_t radix_select(const uint64_t* const* seg, const int* seg_n, i
 }
 
 // Copy the keys >= thr of the segments into out (unordered).  Returns the
-// count; *kmin receives the smallest copied key (all threads see both).
+// count; *kmin (when not null) receives the smallest copied key (all threads
+// see both).
 template <int NTHR>
 __device__ int compact_ge(const uint64_t* const* seg, const int* seg_n, int nseg, uint64_t thr,
                           uint64_t* out, SelectScratch* sc, int tid, int bar_id, uint64_t* kmin) {
@@ -93,18 +103,32 @@ __device__ int compact_ge(const uint64_t* const* seg, const int* seg_n, int nseg
   for (int g = 0; g < nseg; ++g) {
     const uint64_t* p = seg[g];
     const int n = seg_n[g];
-    for (int i = tid; i < n; i += NTHR) {
-      uint64_t v = p[i];
-      if (v >= thr) {
-        int slot = atomicAdd(&sc->newcnt, 1);
-        out[slot] = v;
-        atomicMin(&sc->kmin, (unsigned long long)v);
+    for (int i0 = 0; i0 < n; i0 += NTHR) {
+      const int i = i0 + tid;
+      const uint64_t v = i < n ? p[i] : 0ull;
+      const bool keep = i < n && v >= thr;
+      const unsigned bal = __ballot_sync(0xffffffffu, keep);
+      if (bal) {
+        const int lane = tid & 31;
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&sc->newcnt, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        if (keep) out[base + __popc(bal & ((1u << lane) - 1))] = v;
+        if (kmin) {  // warp minimum of the kept keys, one atomic per warp
+          unsigned long long m = keep ? v : ~0ull;
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const unsigned long long o = __shfl_xor_sync(0xffffffffu, m, off);
+            m = o < m ? o : m;
+          }
+          if (lane == 0) atomicMin(&sc->kmin, m);
+        }
       }
     }
   }
   named_bar_sync(bar_id, NTHR);
   const int n = sc->newcnt;
-  *kmin = sc->kmin;
+  if (kmin) *kmin = sc->kmin;
   named_bar_sync(bar_id, NTHR);
   return n;
 }

@@ -3,11 +3,12 @@
 Exact rule (integer-valued inputs, where fp32 accumulation is exact in any
 order): indices and scores must be bit-identical, padding included.
 
-Tolerance rule (real-valued inputs).  With nu(t, s) = sum_j |w_tj| ||q_tj||
-||k_s|| / sqrt(d), the typical magnitude of a score:
-  - every returned score satisfies |I_gpu - I_ref| <= tol * max(|I_ref|, nu);
+Tolerance rule (real-valued inputs).  With A(t, s) = sum_j |w_tj| sum_c
+|q_tjc k_sc|, the sum of the absolute values of the products a score adds up
+(the scale that bounds both fp32 rounding and operand quantisation error):
+  - every returned score satisfies |I_gpu - I_ref| <= tol * A;
   - the returned sets may differ only on tokens whose reference score lies
-    within tol * nu of the reference k-th score (several sets are then correct);
+    within tol * A of the reference k-th score (several sets are then correct);
   - the number of valid entries is exactly min(k, |legal|), indices are unique,
     legal, and ordered by (score desc, index asc);
   - the IoU against the reference set is reported.
@@ -61,9 +62,9 @@ def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_
         hrow = None if heads is None else np.repeat(np.asarray(heads[a])[None], nv, 0)
         rows_v = np.full(nv, row, np.int64)
         ref_at_g = oracle.score_pairs(inp, rows_v, g_set, hrow)
-        nu_g = oracle.score_scale_pairs(inp, rows_v, g_set)
+        scale_g = oracle.abs_score_pairs(inp, rows_v, g_set, hrow)
         err = np.abs(gs[:nv].astype(np.float64) - ref_at_g)
-        bound = tol * np.maximum(np.abs(ref_at_g), nu_g)
+        bound = tol * scale_g
         bad = np.argwhere(err > bound)
         assert len(bad) == 0, (f"row {row}: score error {err[bad[0][0]]:.3e} > "
                                f"{bound[bad[0][0]]:.3e} at s={g_set[bad[0][0]]}")
@@ -81,8 +82,8 @@ def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_
             rr = np.full(len(group), row, np.int64)
             hh = None if heads is None else np.repeat(np.asarray(heads[a])[None], len(group), 0)
             v = oracle.score_pairs(inp, rr, group, hh)
-            nu = oracle.score_scale_pairs(inp, rr, group)
-            far = np.abs(v - cutoff) > tol * nu
+            scale = oracle.abs_score_pairs(inp, rr, group, hh)
+            far = np.abs(v - cutoff) > tol * scale
             assert not np.any(far), (f"row {row}: token {group[far][0]} differs from the "
                                      f"reference set but is not near the cut-off")
         inter = len(np.intersect1d(g_set, ri[:nv]))

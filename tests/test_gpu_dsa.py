@@ -203,7 +203,7 @@ def test_check_flag_reports_bad_scale(B):
     import torch
     p = gen.normal_problem(22, 1, 64, 256, 64, 128, 16)
     qc, qs, kc, ks, *_ = _fp8_problem(p, B)
-    ks[3] = float("nan")
+    ks[0, 3] = float("nan")
     with pytest.raises(B.DsaError) as e:
         B.dsa_index(qc, kc, dev(p.w), p.topk, q_scale=qs, k_scale=ks, flags=B.DSA_FLAG_CHECK)
     assert e.value.status == B.DSA_ERR_NONFINITE
