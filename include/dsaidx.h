@@ -38,12 +38,17 @@
  *   - Causality.  Query i of sequence b sits at position pos = q_pos0[b] + i
  *     (q_pos0 == NULL: pos0 = n_k - n_q).  Its legal keys are
  *     0 <= s <= pos and s < k_len[b] (k_len == NULL: n_k).
- *   - Output contract.  Each query row receives min(topk, |legal|) entries
- *     ordered by (score descending, index ascending) — the lower index wins a
- *     tie — followed by padding (index -1, score -inf).  -0.0 is written as
- *     +0.0.  The reported score is the one the final selection used: the full
- *     I for dsa_index, misa_dagger_index and hisa_index (route_h == 0); the
- *     routed-head score for misa_index and the stacked hisa_index.
+ *   - Output contract.  Each query row receives its top-k set: the
+ *     min(topk, |legal|) legal keys that are best by (score descending, index
+ *     ascending) — the lower index wins a tie — followed by padding (index -1,
+ *     score -inf).  The entries come in an unspecified order unless
+ *     DSA_FLAG_SORTED is set, which orders them by (score descending, index
+ *     ascending).  Sparse attention consumes the set, so order is optional
+ *     ("PaperTrace 2.2.2", section 2.2: indices returned by the top-k are
+ *     unordered or score-ordered).  -0.0 is written as +0.0.  The reported
+ *     score is the one the final selection used: the full I for dsa_index,
+ *     misa_dagger_index and hisa_index (route_h == 0); the routed-head score
+ *     for misa_index and the stacked hisa_index.
  *   - Memory.  The caller owns every buffer (inputs, outputs, workspace) and
  *     the stream.  The library allocates no device memory, keeps no global
  *     state between calls and never synchronises the stream unless
@@ -87,7 +92,8 @@ typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
 enum { DSA_ALGO_DSA = 0, DSA_ALGO_MISA = 1, DSA_ALGO_MISA_DAGGER = 2, DSA_ALGO_HISA = 3 };
 
 /* problem.flags */
-#define DSA_FLAG_CHECK 1u /* validate scales/lengths on device, synchronise, return device status */
+#define DSA_FLAG_CHECK 1u  /* validate scales/lengths on device, synchronise, return device status */
+#define DSA_FLAG_SORTED 2u /* order each row's top-k by (score desc, index asc) */
 
 typedef struct {
   int32_t batch;          /* sequences */

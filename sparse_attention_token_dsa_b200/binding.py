@@ -20,6 +20,7 @@ DSA_ERR_CUDA, DSA_ERR_NONFINITE, DSA_ERR_TIMEOUT = -4, -5, -6
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
 DSA_ALGO_DSA, DSA_ALGO_MISA, DSA_ALGO_MISA_DAGGER, DSA_ALGO_HISA = 0, 1, 2, 3
 DSA_FLAG_CHECK = 1
+DSA_FLAG_SORTED = 2
 
 
 class DsaProblem(C.Structure):

@@ -195,6 +195,16 @@ cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtenso
   }
 }
 
+template <int NT, int E>
+cudaError_t launch_fin(const FinalArgs& f, int groups, int stage_cap, size_t smem, cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(finalize_kernel<NT, E>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  finalize_kernel<NT, E><<<(f.rows + groups - 1) / groups, NT * groups, smem, st>>>(f, groups,
+                                                                                  stage_cap);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint64_t* logs,
                             const int32_t* cnt, const unsigned long long* thr, int32_t* out_idx,
                             float* out_score, cudaStream_t st) {
@@ -204,7 +214,7 @@ cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint
   f.nsub = pl.nsub;
   f.topk = topk;
   f.capw = pl.capw;
-  int sc = 1;
+  int sc = pl.C == 1 ? 256 : 1024;  // at least one key per thread of a row group
   while (sc < topk) sc <<= 1;
   f.sort_cap = sc;
   f.sorted = sorted;
@@ -213,32 +223,36 @@ cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint
   f.log_thr = thr;
   f.out_idx = out_idx;
   f.out_score = out_score;
-  cudaError_t e;
   if (pl.C == 1) {
-    // one key chunk per row: about k candidates; four rows per CTA
+    // one key chunk per row: about k candidates; up to four rows per CTA
     const int stage_cap = sc + sc / 2;
-    const size_t per_group = ((size_t)sc + stage_cap) * sizeof(uint64_t);
+    const size_t per_group = ((size_t)sc + stage_cap + kFinBoundary) * sizeof(uint64_t);
+    const int e_per = sc / 256;
     int groups = (int)((160 * 1024) / per_group);
     if (groups > kFinMaxGroups) groups = kFinMaxGroups;
+    if (e_per > 8) groups = 1;
     if (groups < 1) groups = 1;
     const size_t smem = per_group * groups;
-    e = cudaFuncSetAttribute(finalize_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    finalize_kernel<256><<<(pl.rows + groups - 1) / groups, 256 * groups, smem, st>>>(f, groups,
-                                                                                     stage_cap);
-  } else {
-    // split-K rows: about C * k candidates; one row per 1024-thread CTA
-    const size_t budget = 200 * 1024;
-    int stage_cap = (int)(budget / sizeof(uint64_t)) - sc;
-    if (stage_cap < sc) stage_cap = sc;
-    const size_t smem = ((size_t)sc + stage_cap) * sizeof(uint64_t);
-    e = cudaFuncSetAttribute(finalize_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem);
-    if (e != cudaSuccess) return e;
-    finalize_kernel<1024><<<pl.rows, 1024, smem, st>>>(f, 1, stage_cap);
+    switch (e_per) {
+      case 1: return launch_fin<256, 1>(f, groups, stage_cap, smem, st);
+      case 2: return launch_fin<256, 2>(f, groups, stage_cap, smem, st);
+      case 4: return launch_fin<256, 4>(f, groups, stage_cap, smem, st);
+      case 8: return launch_fin<256, 8>(f, groups, stage_cap, smem, st);
+      case 16: return launch_fin<256, 16>(f, groups, stage_cap, smem, st);
+      default: return launch_fin<256, 32>(f, groups, stage_cap, smem, st);
+    }
   }
-  return cudaGetLastError();
+  // split-K rows: about C * k candidates; one row per 1024-thread CTA
+  const size_t budget = 200 * 1024;
+  int stage_cap = (int)(budget / sizeof(uint64_t)) - sc - kFinBoundary;
+  if (stage_cap < sc) stage_cap = sc;
+  const size_t smem = ((size_t)sc + stage_cap + kFinBoundary) * sizeof(uint64_t);
+  switch (sc / 1024) {
+    case 1: return launch_fin<1024, 1>(f, 1, stage_cap, smem, st);
+    case 2: return launch_fin<1024, 2>(f, 1, stage_cap, smem, st);
+    case 4: return launch_fin<1024, 4>(f, 1, stage_cap, smem, st);
+    default: return launch_fin<1024, 8>(f, 1, stage_cap, smem, st);
+  }
 }
 
 // Device-side input checks under DSA_FLAG_CHECK: scales finite and positive,
@@ -447,7 +461,8 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   const ScanPlan& pl = L.pl;
-  if (launch_finalize(pl, p->topk, 1, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
+  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  if (launch_finalize(pl, p->topk, sorted, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
                       reinterpret_cast<const int32_t*>(ws + L.off_cnt),
                       reinterpret_cast<const unsigned long long*>(ws + L.off_thr), out_idx,
                       out_score, st) != cudaSuccess)

@@ -15,7 +15,6 @@
 
 namespace dsa {
 
-constexpr int kFinGroupThreads = 256;  // threads per row group (one named barrier each)
 constexpr int kFinMaxGroups = 4;       // row groups per CTA
 constexpr int kFinMaxSeg = 128;
 
@@ -34,99 +33,217 @@ struct FinalArgs {
   float* out_score;      // [rows, topk] or null
 };
 
-// Shared memory of one row group: [sort_cap] selected keys, then [stage_cap]
-// staged candidates.  NT threads per row group: 256 when a row has one key
-// chunk (about k candidates), 1024 for split-K rows (about C * k candidates).
-template <int NT>
-__global__ void __launch_bounds__(1024)
+constexpr int kFinBoundary = 1024;  // boundary-bin capacity per row group
+
+// Per-row-group scalars.
+struct FinGroup {
+  SelectScratch sc;
+  int staged, nwin, nbnd, fallback;
+  unsigned long long thr;
+};
+
+// Exact selection of the `need` largest of the n <= 256 keys in b[] by one
+// warp (register bitonic sort), appended to out[base..].
+__device__ __forceinline__ void warp_take_top(const uint64_t* b, int n, int need, uint64_t* out,
+                                              int base, int lane) {
+  uint64_t v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = lane * 8 + e;
+    v[e] = i < n ? b[i] : 0ull;
+  }
+  bitonic_regs_desc<32, 8>(v, nullptr, lane, 0);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = lane * 8 + e;
+    if (i < need) out[base + i] = v[e];
+  }
+}
+
+// Shared memory of one row group: [sort_cap] result keys, [stage_cap] staged
+// candidates, [kFinBoundary] boundary-bin candidates.  NT threads per row
+// group: 256 when a row has one key chunk (about k candidates), 1024 for
+// split-K rows (about C * k candidates).  E = sort_cap / NT keys per thread
+// for the optional ordering.
+//
+// Selection.  thr, the largest of the row's slot thresholds, bounds the row's
+// k-th best from below.  Candidates >= thr are staged and counted in 256 bins
+// of 16-bit score-key resolution above thr; the bin b* holding the k-th best
+// is found from the counts, every candidate in a higher bin is a winner, and
+// the (small) boundary bin b* is ranked exactly by one warp.  A boundary bin
+// too large for that, or a k-th best beyond the bin window, falls back to the
+// radix select.
+template <int NT, int E>
+__global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
     finalize_kernel(const FinalArgs a, int groups, int stage_cap) {
-  constexpr int kFinGroupThreads = NT;
   extern __shared__ __align__(16) uint64_t fin_smem[];
-  __shared__ SelectScratch sc_all[kFinMaxGroups];
+  __shared__ FinGroup fg_all[kFinMaxGroups];
   __shared__ const uint64_t* segp_all[kFinMaxGroups][kFinMaxSeg];
   __shared__ int segn_all[kFinMaxGroups][kFinMaxSeg];
   __shared__ unsigned long long segt_all[kFinMaxGroups][kFinMaxSeg];
-  __shared__ int staged_all[kFinMaxGroups];
-  const int grp = threadIdx.x / kFinGroupThreads;
-  const int tid = threadIdx.x % kFinGroupThreads;
+  const int grp = threadIdx.x / NT;
+  const int tid = threadIdx.x % NT;
+  const int lane = tid & 31;
   const int bar = 1 + grp;
   const int row = blockIdx.x * groups + grp;
   if (grp >= groups || row >= a.rows) return;   // whole groups leave together
-  uint64_t* fin_buf = fin_smem + (size_t)grp * (a.sort_cap + stage_cap);
-  uint64_t* stage = fin_buf + a.sort_cap;
-  SelectScratch* sc = &sc_all[grp];
+  uint64_t* out = fin_smem + (size_t)grp * (a.sort_cap + stage_cap + kFinBoundary);
+  uint64_t* stage = out + a.sort_cap;
+  uint64_t* bnd = stage + stage_cap;
+  FinGroup* G = &fg_all[grp];
   const uint64_t** segp = segp_all[grp];
   int* segn = segn_all[grp];
   unsigned long long* segt = segt_all[grp];
   const int nseg = a.C * a.nsub;
-  for (int g = tid; g < nseg; g += kFinGroupThreads) {
+  for (int g = tid; g < nseg; g += NT) {
     const int c = g / a.nsub, sb = g % a.nsub;
     const int64_t rs = (int64_t)row * a.C + c;
     segp[g] = a.logs + (rs * a.nsub + sb) * a.capw;
     segn[g] = a.log_cnt[rs * a.nsub + sb];
     segt[g] = a.log_thr[rs];
   }
-  if (tid == 0) staged_all[grp] = 0;
-  named_bar_sync(bar, kFinGroupThreads);
-  // stage the candidates at or above their slot's threshold (a superset of the
-  // row's top-k: each slot's threshold bounds that slot's own top-k from below)
-  // eight independent loads per thread in flight; one slot reservation per warp
-  const int lane = tid & 31;
-  for (int g = 0; g < nseg; ++g) {
+  for (int i = tid; i < 256; i += NT) G->sc.hist[i] = 0;
+  if (tid == 0) {
+    G->staged = G->nwin = G->nbnd = G->fallback = 0;
+    G->thr = 0ull;
+  }
+  named_bar_sync(bar, NT);
+  if (tid == 0) {
+    unsigned long long t = 0ull;
+    for (int g = 0; g < a.C; ++g) t = segt[g * a.nsub] > t ? segt[g * a.nsub] : t;
+    G->thr = t;
+  }
+  named_bar_sync(bar, NT);
+  const unsigned long long thr = G->thr;
+  const int thr16 = (int)(thr >> 48);
+  // ---- stage candidates >= thr and count them per 16-bit score-key bin above
+  // thr; segments are spread over the group's warps, eight loads per lane in flight
+  constexpr int NW = NT / 32;
+  const int wid = tid >> 5;
+  // fewer segments than warps: several warps share a segment (parts of 256)
+  const int parts = nseg >= NW ? 1 : NW / nseg;
+  const int g0 = nseg >= NW ? wid : (wid < parts * nseg ? wid % nseg : nseg);
+  const int gstep = nseg >= NW ? NW : nseg;
+  const int part = nseg >= NW ? 0 : wid / nseg;
+  for (int g = g0; g < nseg; g += gstep) {
     const uint64_t* p = segp[g];
     const int n = segn[g];
-    const unsigned long long t = segt[g];
-    for (int i0 = 0; i0 < n; i0 += 8 * kFinGroupThreads) {
+    for (int i0 = part * 256; i0 < n; i0 += parts * 256) {
       uint64_t v[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * kFinGroupThreads + tid;
+        const int i = i0 + j * 32 + lane;
         v[j] = i < n ? p[i] : 0ull;
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * kFinGroupThreads + tid;
-        const bool keep = i < n && v[j] >= t;
+        const int i = i0 + j * 32 + lane;
+        const bool keep = i < n && v[j] >= thr;
         const unsigned bal = __ballot_sync(0xffffffffu, keep);
         if (bal) {
           int base = 0;
-          if (lane == 0) base = atomicAdd(&staged_all[grp], __popc(bal));
+          if (lane == 0) base = atomicAdd(&G->staged, __popc(bal));
           base = __shfl_sync(0xffffffffu, base, 0);
-          const int slot = base + __popc(bal & ((1u << lane) - 1));
-          if (keep && slot < stage_cap) stage[slot] = v[j];
+          if (keep) {
+            const int slot = base + __popc(bal & ((1u << lane) - 1));
+            if (slot < stage_cap) stage[slot] = v[j];
+            const int bin = min(255, (int)(v[j] >> 48) - thr16);
+            const unsigned peers = __match_any_sync(bal, bin);
+            if (lane == __ffs(peers) - 1) atomicAdd(&G->sc.hist[bin], __popc(peers));
+          }
         }
       }
     }
   }
-  named_bar_sync(bar, kFinGroupThreads);
-  const int total = staged_all[grp];
-  const uint64_t* one[1];
-  int one_n[1];
-  const uint64_t* const* sp;
-  const int* sn;
-  int ns;
-  bool staged = total <= stage_cap;
-  if (staged) {
-    one[0] = stage;
-    one_n[0] = total;
-    sp = one;
-    sn = one_n;
-    ns = 1;
-  } else {  // too many to stage (long runs of tied scores): select from the logs
-    sp = segp;
-    sn = segn;
-    ns = nseg;
+  named_bar_sync(bar, NT);
+  const int total = G->staged;
+  int n;  // number of result keys in out[]
+  if (total <= stage_cap && total <= a.topk) {
+    // every candidate is a winner
+    for (int i = tid; i < total; i += NT) out[i] = stage[i];
+    n = total;
+  } else {
+    bool fb = total > stage_cap;
+    int bstar = 0, above = 0;
+    if (!fb) {
+      if (tid < 32) {
+        int ab;
+        const int b = hist_find(reinterpret_cast<const uint32_t*>(G->sc.hist), 0, a.topk, lane, &ab);
+        if (lane == 0) {
+          G->sc.sel[0] = b;
+          G->sc.sel[1] = ab;
+          if (b < 0 || b == 255) G->fallback = 1;
+        }
+      }
+      named_bar_sync(bar, NT);
+      fb = G->fallback != 0;
+      bstar = G->sc.sel[0];
+      above = G->sc.sel[1];
+    }
+    if (!fb) {
+      // winners above the boundary bin; the boundary bin's candidates aside
+      for (int i0 = 0; i0 < total; i0 += NT) {
+        const int i = i0 + tid;
+        const uint64_t v = i < total ? stage[i] : 0ull;
+        const int bin = i < total ? min(255, (int)(v >> 48) - thr16) : -1;
+        const bool win = bin > bstar, edge = bin == bstar;
+        const unsigned bw = __ballot_sync(0xffffffffu, win);
+        const unsigned be = __ballot_sync(0xffffffffu, edge);
+        int bwin = 0, bedge = 0;
+        if (lane == 0) {
+          if (bw) bwin = atomicAdd(&G->nwin, __popc(bw));
+          if (be) bedge = atomicAdd(&G->nbnd, __popc(be));
+        }
+        bwin = __shfl_sync(0xffffffffu, bwin, 0);
+        bedge = __shfl_sync(0xffffffffu, bedge, 0);
+        const unsigned lt = (1u << lane) - 1;
+        if (win) out[bwin + __popc(bw & lt)] = v;
+        if (edge) {
+          const int slot = bedge + __popc(be & lt);
+          if (slot < kFinBoundary) bnd[slot] = v;
+        }
+      }
+      named_bar_sync(bar, NT);
+      const int nb = G->nbnd;
+      const int need = a.topk - above;
+      if (nb <= 256) {
+        if (tid < 32) warp_take_top(bnd, nb, need, out, above, lane);
+        named_bar_sync(bar, NT);
+        n = a.topk;
+      } else if (nb <= kFinBoundary) {
+        const uint64_t* bs[1] = {bnd};
+        const int bn[1] = {nb};
+        const uint64_t t2 = radix_select<NT>(bs, bn, 1, need, &G->sc, tid, bar);
+        // append the boundary keys >= t2 after the winners
+        if (tid == 0) G->sc.newcnt = 0;
+        named_bar_sync(bar, NT);
+        for (int i = tid; i < nb; i += NT)
+          if (bnd[i] >= t2) out[above + atomicAdd(&G->sc.newcnt, 1)] = bnd[i];
+        named_bar_sync(bar, NT);
+        n = a.topk;
+      } else {
+        fb = true;
+      }
+    }
+    if (fb) {
+      // generic exact selection (long runs of ties): radix select over the
+      // staged set when it fits, else over the raw logs
+      const uint64_t* one[1] = {stage};
+      const int one_n[1] = {total};
+      const bool staged_ok = total <= stage_cap;
+      const uint64_t* const* sp = staged_ok ? one : segp;
+      const int* sn = staged_ok ? one_n : segn;
+      const int ns = staged_ok ? 1 : nseg;
+      const uint64_t t = radix_select<NT>(sp, sn, ns, a.topk, &G->sc, tid, bar);
+      n = compact_ge<NT>(sp, sn, ns, t, out, &G->sc, tid, bar, nullptr);
+    }
   }
-  uint64_t thr = 0ull;
-  if (!staged || total > a.topk)
-    thr = radix_select<kFinGroupThreads>(sp, sn, ns, a.topk, sc, tid, bar);
-  const int n = compact_ge<kFinGroupThreads>(sp, sn, ns, thr, fin_buf, sc, tid, bar, nullptr);
-  if (a.sorted) bitonic_sort_desc<kFinGroupThreads>(fin_buf, n, a.sort_cap, tid, bar);
+  if (a.sorted) sort_desc_regs<NT, E>(out, n, tid, bar);   // sort_cap == NT * E
   int32_t* oi = a.out_idx + (int64_t)row * a.topk;
   float* os = a.out_score ? a.out_score + (int64_t)row * a.topk : nullptr;
-  for (int i = tid; i < a.topk; i += kFinGroupThreads) {
+  for (int i = tid; i < a.topk; i += NT) {
     if (i < n) {
-      const uint64_t c = fin_buf[i];
+      const uint64_t c = out[i];
       oi[i] = comp_index(c);
       if (os) os[i] = comp_score(c);
     } else {

@@ -152,50 +152,6 @@ __device__ __forceinline__ int sched_item(int round, int cta, int grid) {
   return round * grid + ((round & 1) ? (grid - 1 - cta) : cta);
 }
 
-// Warp-wide search over 256 histogram bins (lane l owns bins 255-8l .. 248-8l):
-// the highest bin b with base + (count of bins >= b) >= need.  Returns the bin
-// (-1 when the total stays below need) and, in *above, base + count strictly
-// above it.
-__device__ __forceinline__ int hist_find(const uint32_t* h, int base, int need, int lane,
-                                         int* above) {
-  int c[8];
-  int tot = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    c[i] = (int)h[255 - 8 * lane - i];
-    tot += c[i];
-  }
-  int incl = tot;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int o = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += o;
-  }
-  const int excl = incl - tot;
-  const bool mine = base + excl < need && need <= base + incl;
-  const unsigned bal = __ballot_sync(0xffffffffu, mine);
-  if (!bal) {
-    *above = 0;
-    return -1;
-  }
-  const int src = __ffs(bal) - 1;
-  int bin = 0, ab = 0;
-  if (lane == src) {
-    int cum = base + excl;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (cum + c[i] >= need) {
-        bin = 255 - 8 * lane - i;
-        ab = cum;
-        break;
-      }
-      cum += c[i];
-    }
-  }
-  *above = __shfl_sync(0xffffffffu, ab, src);
-  return __shfl_sync(0xffffffffu, bin, src);
-}
-
 // In-place warp compaction of one sub-log: keep entries >= thr; returns the
 // count.  Eight independent loads per lane are in flight per round.
 __device__ __forceinline__ int compact_sublog(uint64_t* lg, int n, unsigned long long thr,
@@ -756,6 +712,25 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if (etid == 0) T->raise_any = 0;
         named_bar_sync(kBarEpi, kEpiThreads);
       }
+      // ---- item end (split-K): every warp trims its own sub-logs to the final
+      // threshold (the last step always ran a threshold update), so the select
+      // stage reads about k candidates per key chunk instead of every survivor
+      named_bar_sync(kBarEpi, kEpiThreads);
+      if (!stop && a.C > 1) {
+        for (int gg = 0; gg < a.G; ++gg) {
+          for (int qi = 0; qi < qhalf; ++qi) {
+            const int r = gg * a.QG + (modeB ? 0 : half * qhalf) + qi;
+            if (r >= g.nrows) continue;
+            const int n = T->subcnt[r][sub];
+            if (n == 0) continue;
+            uint64_t* lg = a.logs + ((slot0 + (int64_t)r * a.C) * a.nsub + sub) * a.capw;
+            const int kept = compact_sublog(lg, n, T->row_thr[r], lane);
+            if (lane == 0) T->subcnt[r][sub] = kept;
+            __syncwarp();
+          }
+        }
+      }
+      named_bar_sync(kBarEpi, kEpiThreads);
       // ---- item end: publish sub-log fills and thresholds
       for (int r = etid; r < g.nrows; r += kEpiThreads) {
         const int64_t rs = slot0 + (int64_t)r * a.C;

@@ -11,6 +11,50 @@
 
 namespace dsa {
 
+// Warp-wide search over 256 histogram bins (lane l owns bins 255-8l .. 248-8l):
+// the highest bin b with base + (count of bins >= b) >= need.  Returns the bin
+// (-1 when the total stays below need) and, in *above, base + count strictly
+// above it.
+__device__ __forceinline__ int hist_find(const uint32_t* h, int base, int need, int lane,
+                                         int* above) {
+  int c[8];
+  int tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    c[i] = (int)h[255 - 8 * lane - i];
+    tot += c[i];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += o;
+  }
+  const int excl = incl - tot;
+  const bool mine = base + excl < need && need <= base + incl;
+  const unsigned bal = __ballot_sync(0xffffffffu, mine);
+  if (!bal) {
+    *above = 0;
+    return -1;
+  }
+  const int src = __ffs(bal) - 1;
+  int bin = 0, ab = 0;
+  if (lane == src) {
+    int cum = base + excl;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (cum + c[i] >= need) {
+        bin = 255 - 8 * lane - i;
+        ab = cum;
+        break;
+      }
+      cum += c[i];
+    }
+  }
+  *above = __shfl_sync(0xffffffffu, ab, src);
+  return __shfl_sync(0xffffffffu, bin, src);
+}
+
 struct SelectScratch {
   int hist[256];
   int sel[4];
@@ -154,6 +198,79 @@ __device__ void bitonic_sort_desc(uint64_t* a, int n, int cap, int tid, int bar_
       named_bar_sync(bar_id, NTHR);
     }
   }
+}
+
+// Descending bitonic sort of N = NT * E keys held E per thread in registers
+// (thread t holds positions t*E .. t*E+E-1).  Strides below E compare inside a
+// thread, strides below 32*E across lanes with shuffles, and only strides of
+// 32*E and more go through shared memory `xs` (N keys) with a barrier.
+template <int NT, int E>
+__device__ __forceinline__ void bitonic_regs_desc(uint64_t (&v)[E], uint64_t* xs, int tid,
+                                                  int bar_id) {
+  constexpr int N = NT * E;
+  const int lane = tid & 31;
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      if (stride < E) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if ((e & stride) == 0) {
+            const int i = tid * E + e;
+            const bool desc = (i & size) == 0;
+            const uint64_t x = v[e], y = v[e + stride];
+            if ((x < y) == desc) {
+              v[e] = y;
+              v[e + stride] = x;
+            }
+          }
+        }
+      } else if (stride < 32 * E) {
+        const int ld = stride / E;  // lane distance of the partner
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const uint64_t o = __shfl_xor_sync(0xffffffffu, v[e], ld);
+          const bool lower = (lane & ld) == 0;      // this position is the pair's lower index
+          const bool desc = (i & size) == 0;
+          // the lower position keeps the larger key in a descending pair
+          const bool take_max = lower == desc;
+          v[e] = take_max ? (o > v[e] ? o : v[e]) : (o < v[e] ? o : v[e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) xs[tid * E + e] = v[e];
+        named_bar_sync(bar_id, NT);
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = tid * E + e;
+          const uint64_t o = xs[i ^ stride];
+          const bool lower = (i & stride) == 0;
+          const bool desc = (i & size) == 0;
+          const bool take_max = lower == desc;
+          v[e] = take_max ? (o > v[e] ? o : v[e]) : (o < v[e] ? o : v[e]);
+        }
+        named_bar_sync(bar_id, NT);
+      }
+    }
+  }
+}
+
+// Sort a[0, n) descending in place (n <= N = NT * E; slots up to N hold 0).
+template <int NT, int E>
+__device__ void sort_desc_regs(uint64_t* a, int n, int tid, int bar_id) {
+  uint64_t v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = tid * E + e;
+    v[e] = i < n ? a[i] : 0ull;
+  }
+  named_bar_sync(bar_id, NT);
+  bitonic_regs_desc<NT, E>(v, a, tid, bar_id);
+#pragma unroll
+  for (int e = 0; e < E; ++e) a[tid * E + e] = v[e];
+  named_bar_sync(bar_id, NT);
 }
 
 }  // namespace dsa

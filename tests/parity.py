@@ -20,6 +20,23 @@ import numpy as np
 import oracle
 
 
+def order_rows(idx, score):
+    """Order each row by (score desc, index asc), padding (-1, -inf) last."""
+    idx = np.asarray(idx)
+    score = np.asarray(score)
+    oi = np.empty_like(idx)
+    os_ = np.empty_like(score)
+    for r in range(idx.shape[0]):
+        valid = idx[r] >= 0
+        order = np.lexsort((idx[r][valid], -score[r][valid].astype(np.float64)))
+        nv = int(valid.sum())
+        oi[r, :nv] = idx[r][valid][order]
+        os_[r, :nv] = score[r][valid][order]
+        oi[r, nv:] = -1
+        os_[r, nv:] = -np.inf
+    return oi, os_
+
+
 def exact(gpu_idx, gpu_score, ref_idx, ref_score):
     gi, gs = np.asarray(gpu_idx), np.asarray(gpu_score)
     assert np.array_equal(gi, ref_idx), _first_diff(gi, ref_idx)

@@ -38,22 +38,28 @@ def dev(x):
 
 
 def run_dsa(B, p, q=None, k=None, q_scale=None, k_scale=None, flags=0):
+    """GPU top-k rows; without DSA_FLAG_SORTED the set is ordered on the host."""
     q = dev(p.q) if q is None else q
     k = dev(p.k) if k is None else k
     idx, sc = B.dsa_index(q, k, dev(p.w), p.topk, q_scale=q_scale, k_scale=k_scale,
                           q_pos0=dev(p.q_pos0), k_len=dev(p.k_len), flags=flags)
     import torch
     torch.cuda.synchronize()
-    return (idx.cpu().numpy().reshape(-1, p.topk), sc.cpu().numpy().reshape(-1, p.topk))
+    gi = idx.cpu().numpy().reshape(-1, p.topk)
+    gs = sc.cpu().numpy().reshape(-1, p.topk)
+    if not flags & B.DSA_FLAG_SORTED:
+        gi, gs = parity.order_rows(gi, gs)
+    return gi, gs
 
 
 # ------------------------------------------------------------------ exact ---
 
 @pytest.mark.parametrize("dtype", [gen.F32, gen.BF16])
 def test_integer_full_layer_bit_exact(B, dtype):
-    """L = 1024 causal, H = 64, d = 128, k = 128, integer q, k, w: bit-exact."""
+    """L = 1024 causal, H = 64, d = 128, k = 128, integer q, k, w: bit-exact,
+    including the (score desc, index asc) order requested by DSA_FLAG_SORTED."""
     p = gen.integer_problem(1, 1, 1024, 1024, 64, 128, 128, dtype=dtype)
-    gi, gs = run_dsa(B, p, flags=B.DSA_FLAG_CHECK)
+    gi, gs = run_dsa(B, p, flags=B.DSA_FLAG_CHECK | B.DSA_FLAG_SORTED)
     ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
     parity.exact(gi, gs, ri, rs)
 
@@ -84,10 +90,11 @@ def test_integer_topk_above_keys_pads(B):
     assert np.all(gi[:, 300:] == -1)
 
 
-def test_integer_many_ties_long_rows_bit_exact(B):
-    """Small value range => massive score ties; several threshold raises per row."""
+@pytest.mark.parametrize("flags", [0, 2])
+def test_integer_many_ties_long_rows_bit_exact(B, flags):
+    """Small value range => massive score ties; exact raises and the tie fallback."""
     p = gen.integer_problem(5, 1, 64, 20000, 64, 128, 1024, qk_max=1, w_max=1, dtype=gen.BF16)
-    gi, gs = run_dsa(B, p)
+    gi, gs = run_dsa(B, p, flags=flags)
     ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
     parity.exact(gi, gs, ri, rs)
 
