@@ -134,6 +134,24 @@ int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const v
               const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
               void* workspace, size_t workspace_bytes, void* stream);
 
+/* dsa_index without a caller-provided workspace, for callers that cannot
+ * allocate device memory when they call (a serving loop whose memory plan is
+ * fixed after start-up, or a host framework whose own allocator owns all
+ * device memory and forbids side allocations).  The pages describe no such
+ * call; it exists for those callers only.  Scratch is a fixed 64 MiB array in
+ * device memory inside the library (held on every GPU that loads the library,
+ * until the process exits); problems whose dsa_workspace_size() exceeds
+ * 64 MiB are rejected with DSA_ERR_WORKSPACE.  Nothing is allocated or freed.
+ * The first call on a device looks up that device's scratch address (a
+ * one-time set-up per device; make that first call before any stream
+ * capture).  Every call on a device shares the one scratch array, so calls
+ * whose executions overlap on the GPU (different streams, no ordering between
+ * them) race and corrupt each other's results; order them on one stream or
+ * with events.  Other arguments and results are as for dsa_index. */
+int dsa_index_noalloc(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+                      const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
+                      void* stream);
+
 /* The two stages of dsa_index, for callers that schedule (or time) them
  * separately: dsa_index is exactly dsa_index_scan followed by
  * dsa_index_select on the same workspace and stream.  The scan stage scores

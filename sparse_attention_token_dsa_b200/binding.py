@@ -54,13 +54,15 @@ def _load():
     lib.dsa_read_status.argtypes = [vp, vp]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_index_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.dsa_index_scan.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_index_select.argtypes = [P, vp, vp, vp, sz, vp]
     lib.misa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.misa_dagger_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
-    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "dsa_index_scan",
+    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "dsa_index_noalloc",
+              "dsa_index_scan",
               "dsa_index_select", "misa_index",
               "misa_dagger_index", "hisa_index", "dsa_quantize_e4m3"):
         getattr(lib, f).restype = C.c_int
@@ -140,6 +142,21 @@ def dsa_index(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_len=None
     idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
     _check(lib.dsa_index(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale), _ptr(w),
                          _ptr(idx), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream)), "dsa_index")
+    return idx, sc
+
+
+def dsa_index_noalloc(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_len=None,
+                      flags=0, out=None, stream=None):
+    """dsa_index on the library's fixed internal scratch (no workspace argument).
+
+    For callers that cannot allocate device memory at call time; problems that
+    need more than the library's 64 MiB scratch raise DsaError(DSA_ERR_WORKSPACE),
+    and calls that overlap on the GPU race on the shared scratch."""
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.dsa_index_noalloc(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale),
+                                 _ptr(w), _ptr(idx), _ptr(sc), _stream(stream)),
+           "dsa_index_noalloc")
     return idx, sc
 
 

@@ -340,6 +340,37 @@ int finish(const dsa_problem* p, void* ws, cudaStream_t st) {
   return DSA_OK;
 }
 
+// ----------------------------------------------------- allocation-free path --
+// Scratch of dsa_index_noalloc: a fixed 64 MiB array in device memory that
+// every GPU loading this library holds until the process exits.  Host code
+// must not use the name as an address; the device address comes from
+// cudaGetSymbolAddress, taken once per device with that device current.
+constexpr size_t kNoAllocScratchBytes = 64ull << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kNoAllocMaxDevices];  // per-device address, null until set up
+
+int noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    cudaGetLastError();
+    return DSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return DSA_ERR_CUDA;
+    }
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== ABI ==
@@ -477,6 +508,19 @@ int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const v
   int rc = dsa_index_scan(p, q, q_scale, k, k_scale, w, workspace, workspace_bytes, stream);
   if (rc != DSA_OK) return rc;
   return dsa_index_select(p, out_idx, out_score, workspace, workspace_bytes, stream);
+}
+
+int dsa_index_noalloc(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
+                      const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
+                      void* stream) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  if (dsa_layout(p).total > kNoAllocScratchBytes) return DSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  const int rc = noalloc_scratch_address(&scratch);
+  if (rc != DSA_OK) return rc;
+  return dsa_index(p, q, q_scale, k, k_scale, w, out_idx, out_score, scratch,
+                   kNoAllocScratchBytes, stream);
 }
 
 int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* out,

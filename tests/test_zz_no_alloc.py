@@ -1,0 +1,84 @@
+"""GPU test of dsa_index_noalloc, the entry point for callers that cannot
+allocate device memory when they call (fixed memory plans, host frameworks
+whose allocator owns all device memory).  It must return what dsa_index
+returns on the same inputs, call after call, while keeping its scratch inside
+the library; problems too large for that scratch are refused cleanly.
+
+This file is named so that pytest collects it last: a run that stops at the
+first failure has already run every other test.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from sparse_attention_token_dsa_b200 import inputs as gen
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def B():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    from sparse_attention_token_dsa_b200 import binding
+    return binding
+
+
+def _dev(x):
+    import torch
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).cuda().view(torch.bfloat16)
+    return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+
+
+def _call_noalloc(B, p, q, k, w, pos0, klen, flags):
+    """Call the C ABI directly (no Python-side workspace anywhere)."""
+    import torch
+    prob = B.problem(q, k, p.topk, pos0, klen, flags)
+    idx = torch.full((p.batch, p.n_q, p.topk), -7, dtype=torch.int32, device="cuda")
+    sc = torch.full((p.batch, p.n_q, p.topk), 7.0, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    rc = B.lib.dsa_index_noalloc(C.byref(prob), C.c_void_p(q.data_ptr()), None,
+                                 C.c_void_p(k.data_ptr()), None, C.c_void_p(w.data_ptr()),
+                                 C.c_void_p(idx.data_ptr()), C.c_void_p(sc.data_ptr()),
+                                 C.c_void_p(stream.cuda_stream))
+    torch.cuda.synchronize()
+    return rc, idx.cpu().numpy(), sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("kind", ["integer", "real"])
+def test_noalloc_matches_dsa_index_on_two_calls(B, kind):
+    import torch
+    if kind == "integer":
+        p = gen.integer_problem(41, 2, 150, 500, 64, 128, 96, q_pos0=[0, 300], k_len=[200, 500],
+                                dtype=gen.BF16)
+    else:
+        p = gen.normal_problem(42, 1, 384, 384, 64, 128, 128)
+    q, k, w = _dev(p.q), _dev(p.k), _dev(p.w)
+    pos0 = None if p.q_pos0 is None else _dev(p.q_pos0)
+    klen = None if p.k_len is None else _dev(p.k_len)
+    flags = B.DSA_FLAG_SORTED
+    ref_i, ref_s = B.dsa_index(q, k, w, p.topk, q_pos0=pos0, k_len=klen, flags=flags)
+    torch.cuda.synchronize()
+    ref_i, ref_s = ref_i.cpu().numpy(), ref_s.cpu().numpy()
+    for _ in range(2):   # the shared scratch keeps the previous call's contents
+        rc, gi, gs = _call_noalloc(B, p, q, k, w, pos0, klen, flags)
+        assert rc == B.DSA_OK, B.status_string(rc)
+        assert np.array_equal(gi, ref_i)
+        assert np.array_equal(gs, ref_s)   # same kernels: identical to the last bit
+
+
+def test_noalloc_refuses_problems_beyond_its_scratch(B):
+    import torch
+    # 32 sequences x 131072 keys of decode need far more than the fixed scratch
+    q = torch.zeros((32, 1, 64, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros((32, 131072, 128), dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros((32, 1, 64), dtype=torch.float32, device="cuda")
+    prob = B.problem(q, k, 2048)
+    assert B.dsa_workspace_size(prob) > 64 << 20
+    rc = B.lib.dsa_index_noalloc(C.byref(prob), C.c_void_p(q.data_ptr()), None,
+                                 C.c_void_p(k.data_ptr()), None, C.c_void_p(w.data_ptr()),
+                                 C.c_void_p(0x1000), C.c_void_p(0x1000), None)
+    assert rc == B.DSA_ERR_WORKSPACE
