@@ -149,10 +149,10 @@ bool make_map(CUtensorMap* m, const void* base, int esz, uint64_t rows, uint32_t
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <MmaKind K, bool S, int HT>
+template <MmaKind K, bool S, int HT, int GATHER = 0>
 cudaError_t launch_scan_t(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
                           const ScanArgs& a, cudaStream_t st) {
-  auto kern = scan_kernel<K, S, HT>;
+  auto kern = scan_kernel<K, S, HT, GATHER>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pl.smem);
   if (e != cudaSuccess) return e;
@@ -458,6 +458,11 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.n_k = p->n_k;
   a.H = p->heads;
   a.d = p->dim;
+  a.n_tok = p->n_k;
+  a.bs_shift = 0;
+  a.klist = nullptr;
+  a.klist_len = 0;
+  a.lb_shift = 0;
   a.keep = p->topk;
   a.QG = pl.QG;
   a.G = pl.G;

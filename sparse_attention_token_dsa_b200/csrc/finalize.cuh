@@ -29,8 +29,11 @@ struct FinalArgs {
   const uint64_t* logs;  // [rows * C][nsub][capw]
   const int32_t* log_cnt;               // [rows * C][nsub]
   const unsigned long long* log_thr;    // [rows * C]
-  int32_t* out_idx;      // [rows, topk]
-  float* out_score;      // [rows, topk] or null
+  int32_t nq_c;          // rows per sequence in this call (rows = batch * nq_c)
+  int32_t nq_total;      // rows per sequence of the outputs
+  int32_t q_off;         // row i of sequence b writes output row b * nq_total + q_off + i
+  int32_t* out_idx;      // [batch * nq_total, topk]
+  float* out_score;      // [batch * nq_total, topk] or null
 };
 
 constexpr int kFinBoundary = 1024;  // boundary-bin capacity per row group
@@ -239,8 +242,9 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
     }
   }
   if (a.sorted) sort_desc_regs<NT, E>(out, n, tid, bar);   // sort_cap == NT * E
-  int32_t* oi = a.out_idx + (int64_t)row * a.topk;
-  float* os = a.out_score ? a.out_score + (int64_t)row * a.topk : nullptr;
+  const int64_t orow = (int64_t)(row / a.nq_c) * a.nq_total + a.q_off + row % a.nq_c;
+  int32_t* oi = a.out_idx + orow * a.topk;
+  float* os = a.out_score ? a.out_score + orow * a.topk : nullptr;
   for (int i = tid; i < a.topk; i += NT) {
     if (i < n) {
       const uint64_t c = out[i];

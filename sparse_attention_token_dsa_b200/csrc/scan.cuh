@@ -42,6 +42,16 @@ namespace dsa {
 
 struct ScanArgs {
   int32_t batch, n_q, n_k, H, d;
+  int32_t q_stride;      // query rows per sequence in q / w / scales (>= q_off + n_q)
+  int32_t q_off;         // first query of this call: row i of sequence b is q / w row
+                         //   b * q_stride + q_off + i, at position pos0 + q_off + i
+  int32_t n_tok;         // token positions per sequence (default pos0 = n_tok - q_stride,
+                         //   k_len = n_tok)
+  int32_t bs_shift;      // > 0: keys are full-block representatives of 2^bs_shift tokens;
+                         //      a row sees block b iff (b + 1) << bs_shift <= min(pos + 1, k_len)
+  const int32_t* klist;  // gathered keys: per-row lists [rows, klist_len] (-1 = empty slot)
+  int32_t klist_len;
+  int32_t lb_shift;      // block lists: log2 tokens per listed block
   int32_t keep;          // entries each row must keep (top-k or k')
   int32_t QG;            // query rows per accumulator group (<= 256 / (H * parts))
   int32_t G;             // groups per work item (1 or 2)
@@ -50,7 +60,7 @@ struct ScanArgs {
   int32_t C;             // key chunks per row (split-K); 1 = whole prefix
   int32_t chunk;         // keys per chunk (multiple of 128) when C > 1
   int32_t n_items;       // batch * n_qt * C
-  const int32_t* q_pos0; // [batch] or null: n_k - n_q
+  const int32_t* q_pos0; // [batch] or null: n_tok - q_stride
   const int32_t* k_len;  // [batch] or null: n_k
   const float* w;        // [rows, H]
   const float* row_scale;   // [rows] or null: multiplies w (query dequant scale)
@@ -115,6 +125,7 @@ struct ItemGeom {
   int b, qt, c, row0, nrows, kbeg, kend, ntiles, t_hi;
 };
 
+template <int GATHER>
 __device__ __forceinline__ ItemGeom item_geom(const ScanArgs& a, int item) {
   ItemGeom g;
   const int qt_rev = item / (a.batch * a.C);
@@ -125,10 +136,19 @@ __device__ __forceinline__ ItemGeom item_geom(const ScanArgs& a, int item) {
   const int QT = a.QG * a.G;
   g.row0 = g.qt * QT;
   g.nrows = min(QT, a.n_q - g.row0);
-  const int pos0 = a.q_pos0 ? a.q_pos0[g.b] : a.n_k - a.n_q;
-  const int klen = a.k_len ? a.k_len[g.b] : a.n_k;
+  if constexpr (GATHER != 0) {
+    // one row per item; its keys come from its list, in list order
+    g.kbeg = 0;
+    g.kend = a.klist_len;
+    g.ntiles = g.nrows > 0 ? (a.klist_len + 127) >> 7 : 0;
+    g.t_hi = 0;
+    return g;
+  }
+  const int pos0 = (a.q_pos0 ? a.q_pos0[g.b] : a.n_tok - a.q_stride) + a.q_off;
+  const int klen = a.k_len ? a.k_len[g.b] : a.n_tok;
   const int maxpos = pos0 + g.row0 + g.nrows - 1;
   int kend = min(maxpos + 1, klen);
+  if (a.bs_shift > 0) kend = kend >> a.bs_shift;  // full blocks only
   int kbeg = 0;
   if (a.C > 1) {
     kbeg = g.c * a.chunk;
@@ -357,7 +377,7 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
 
 // 320 threads: ten warps over four sub-partitions of 16K registers each allow
 // at most 168 registers per thread.
-template <MmaKind KIND, bool SPLIT, int HT>
+template <MmaKind KIND, bool SPLIT, int HT, int GATHER>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const ScanArgs a) {
@@ -416,11 +436,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int round = 0; ok; ++round) {
         const int item = sched_item(round, blockIdx.x, grid);
         if (item >= a.n_items) break;
-        ItemGeom g = item_geom(a, item);
+        ItemGeom g = item_geom<GATHER>(a, item);
         if (g.ntiles == 0) continue;
         if (!mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1)) break;
         mbar_arrive_expect_tx(&T->q_full, q_bytes);
-        const int qrow0 = (g.b * a.n_q + g.row0) * a.H * PARTS;
+        const int qrow0 = (g.b * a.q_stride + a.q_off + g.row0) * a.H * PARTS;
         for (int gg = 0; gg < a.G; ++gg)
           for (int at = 0; at < Cfg::A; ++at)
             tma_load_2d(Qs + (gg * Cfg::A + at) * qcols * 128, &qmap, &T->q_full,
@@ -432,10 +452,43 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const uint32_t ph = (kcount / Cfg::KSTAGES) & 1;
           if (!mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2)) { ok = false; break; }
           mbar_arrive_expect_tx(&T->k_full[slot], Cfg::KTILE_BYTES);
-          const int tstart = (g.t_hi - t) << 7;
-          for (int at = 0; at < Cfg::A; ++at)
-            tma_load_2d(Ks + (slot * Cfg::A + at) * 16384, &kmap, &T->k_full[slot], at * Cfg::EPA,
-                        krow0 + tstart);
+          if constexpr (GATHER == 0) {
+            const int tstart = (g.t_hi - t) << 7;
+            for (int at = 0; at < Cfg::A; ++at)
+              tma_load_2d(Ks + (slot * Cfg::A + at) * 16384, &kmap, &T->k_full[slot],
+                          at * Cfg::EPA, krow0 + tstart);
+          } else {
+            const int32_t* lst = a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len;
+            if constexpr (GATHER == 1) {
+              // token list: four arbitrary key rows per gather (one-row-high boxes)
+              for (int r4 = 0; r4 < 128; r4 += 4) {
+                int rr[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                  const int e = t * 128 + r4 + j;
+                  const int kk = e < a.klist_len ? lst[e] : -1;
+                  rr[j] = krow0 + (kk >= 0 ? kk : 0);
+                }
+                for (int at = 0; at < Cfg::A; ++at)
+                  tma_gather4(Ks + (slot * Cfg::A + at) * 16384 + r4 * 128, &kmap, &T->k_full[slot],
+                              at * Cfg::EPA, rr[0], rr[1], rr[2], rr[3]);
+              }
+            } else {
+              // block list: runs of 2^lb_shift contiguous keys (box of min(bs, 128) rows)
+              const int bs = 1 << a.lb_shift;
+              const int box = bs < 128 ? bs : 128;
+              for (int r0 = 0; r0 < 128; r0 += box) {
+                const int e = t * 128 + r0;                 // token slot in the row's list
+                const int slot_b = e >> a.lb_shift;
+                const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
+                const int off = e & (bs - 1);
+                const int y = krow0 + (blk >= 0 ? blk * bs + off : 0);
+                for (int at = 0; at < Cfg::A; ++at)
+                  tma_load_2d(Ks + (slot * Cfg::A + at) * 16384 + r0 * 128, &kmap, &T->k_full[slot],
+                              at * Cfg::EPA, y);
+              }
+            }
+          }
           ++kcount;
         }
       }
@@ -455,7 +508,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       for (int round = 0; ok; ++round) {
         const int item = sched_item(round, blockIdx.x, grid);
         if (item >= a.n_items) break;
-        ItemGeom g = item_geom(a, item);
+        ItemGeom g = item_geom<GATHER>(a, item);
         if (g.ntiles == 0) continue;
         if (!mbar_wait(&T->q_full, it & 1, abort, a.status, 3)) break;
         ++it;
@@ -513,17 +566,26 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     for (int round = 0; !stop; ++round) {
       const int item = sched_item(round, blockIdx.x, grid);
       if (item >= a.n_items) break;
-      ItemGeom g = item_geom(a, item);
-      const int pos0 = a.q_pos0 ? a.q_pos0[g.b] : a.n_k - a.n_q;
-      const int klen = a.k_len ? a.k_len[g.b] : a.n_k;
+      ItemGeom g = item_geom<GATHER>(a, item);
+      const int pos0 = (a.q_pos0 ? a.q_pos0[g.b] : a.n_tok - a.q_stride) + a.q_off;
+      const int klen = a.k_len ? a.k_len[g.b] : a.n_tok;
       const int64_t slot0 = ((int64_t)g.b * a.n_q + g.row0) * a.C + g.c;  // slot of row 0
       // ---- item init: row states, histograms, head weights
       for (int r = etid; r < QT; r += kEpiThreads) {
         T->row_thr[r] = 0ull;
         T->row_b1[r] = -1;
         T->row_raise[r] = 0;
-        T->row_nleg[r] =
-            (r < g.nrows) ? max(0, min(min(pos0 + g.row0 + r, klen - 1), g.kend - 1) - g.kbeg + 1) : 0;
+        int nleg = 0;
+        if (r < g.nrows) {
+          const int pos = pos0 + g.row0 + r;
+          if (GATHER != 0)
+            nleg = max(0, min(pos, klen - 1) + 1);                     // key <= pos, key < k_len
+          else if (a.bs_shift > 0)
+            nleg = max(0, min(min(pos + 1, klen) >> a.bs_shift, g.kend) - g.kbeg);
+          else
+            nleg = max(0, min(min(pos, klen - 1), g.kend - 1) - g.kbeg + 1);
+        }
+        T->row_nleg[r] = nleg;
 #pragma unroll
         for (int w8 = 0; w8 < 8; ++w8) T->subcnt[r][w8] = 0;
       }
@@ -532,7 +594,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         const int r = i >> hshift, j = i & (H - 1);
         float wv = 0.f;
         if (r < g.nrows) {
-          const int64_t grow = (int64_t)g.b * a.n_q + g.row0 + r;
+          const int64_t grow = (int64_t)g.b * a.q_stride + a.q_off + g.row0 + r;
           wv = a.w[grow * H + j];
           if (a.row_scale) wv *= a.row_scale[grow];
           if (a.head_scale) wv *= a.head_scale[grow * H + j];
@@ -559,9 +621,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           tc_fence_after();
           const int gg = uu & (a.G - 1);
           const int t = uu >> (a.G - 1);
-          const int key = ((g.t_hi - t) << 7) + quad * 32 + lane;
+          int key;
+          if constexpr (GATHER == 0) {
+            key = ((g.t_hi - t) << 7) + quad * 32 + lane;
+          } else {
+            const int32_t* lst = a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len;
+            const int e = t * 128 + quad * 32 + lane;
+            if constexpr (GATHER == 1) {
+              key = e < a.klist_len ? lst[e] : -1;
+            } else {
+              const int slot_b = e >> a.lb_shift;
+              const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
+              key = blk >= 0 ? (blk << a.lb_shift) + (e & ((1 << a.lb_shift) - 1)) : -1;
+            }
+          }
           float ks = 1.f;
-          if (a.k_scale && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
+          if (a.k_scale && key >= 0 && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
           const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + s * a.stage_cols;
           // queries handled by this warp inside group gg
           const int qbeg = modeB ? 0 : half * qhalf;
