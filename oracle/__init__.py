@@ -58,6 +58,8 @@ def lib():
                                        vp, vp, vp]
         _lib.orc_hisa_rows.argtypes = [vp, i32, i32, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp,
                                        vp, vp, vp, vp]
+        _lib.orc_block_scores.restype = C.c_int64
+        _lib.orc_block_scores.argtypes = [vp, i64, i32, vp, i32, vp]
         _lib.orc_score_row.restype = C.c_int64
         _lib.orc_score_row.argtypes = [vp, i64, vp, i32, vp]
     return _lib
@@ -187,6 +189,16 @@ def score_row(inp: Inputs, row: int, heads=None):
     out = np.empty(max(n, 1), np.float64)
     h = None if heads is None else np.ascontiguousarray(heads, np.int32)
     got = lib().orc_score_row(inp.ref, int(row), _p(h), 0 if h is None else len(h), _p(out))
+    return out[:got]
+
+
+def block_scores(inp: Inputs, row: int, block: int, heads=None):
+    """HISA coarse scores J of every block of one row's legal prefix (fp64)."""
+    n = inp.prob.legal_count(row)
+    out = np.empty(max((n + block - 1) // block, 1), np.float64)
+    h = None if heads is None else np.ascontiguousarray(heads, np.int32)
+    got = lib().orc_block_scores(inp.ref, int(row), block, _p(h), 0 if h is None else len(h),
+                                 _p(out))
     return out[:got]
 
 

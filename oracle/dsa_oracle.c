@@ -629,6 +629,30 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
   return ORC_OK;
 }
 
+/* [HISA] coarse-stage scores of one row over every block of its legal prefix:
+ * J_{t,a} = sum_{x} w_{t,heads[x]} max(q_{t,heads[x]} . k~_a, 0) (heads NULL: all),
+ * the boundary block represented by the mean of its legal tokens.  Writes
+ * out[0 .. M^b_t) and returns M^b_t.  Used by tests to judge near-ties at the
+ * block cut-off. */
+int64_t orc_block_scores(const orc_inputs* in, int64_t row, int32_t blk, const int32_t* heads,
+                         int32_t nh, double* out) {
+  int32_t b = (int32_t)(row / in->n_q);
+  int64_t n = row_legal(in, row), m = 0;
+  double* reps = block_representatives(in, b, n, blk, &m);
+  for (int64_t a = 0; a < m; ++a) {
+    double J = 0.0;
+    int32_t cnt = heads ? nh : in->heads;
+    for (int32_t x = 0; x < cnt; ++x) {
+      int32_t j = heads ? heads[x] : x;
+      double z = dot_q_vec(in, row, j, reps + a * in->dim);
+      J += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+    }
+    out[a] = J;
+  }
+  free(reps);
+  return m;
+}
+
 /* Full fp64 score row (all legal s) of one query row for the listed heads
  * (NULL = all); returns |legal|.  Used by tests for margins and tie checks. */
 int64_t orc_score_row(const orc_inputs* in, int64_t row, const int32_t* heads, int32_t nh,

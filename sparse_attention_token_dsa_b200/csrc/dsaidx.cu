@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "finalize.cuh"
 #include "prep.cuh"
+#include "route.cuh"
 #include "scan.cuh"
 
 using namespace dsa;
@@ -112,6 +113,46 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   return pl;
 }
 
+// Plan of a gathered-key scan: every query row has its own key list, so a work
+// item is one row (QG = G = 1, no split-K) and the MMA N is its heads (at least 16).
+ScanPlan plan_gather(MmaKind kind, int batch, int n_q, int H, int keep) {
+  ScanPlan pl{};
+  pl.kind = kind;
+  pl.split = false;
+  pl.parts = 1;
+  pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
+  pl.atoms = pl.esz;
+  pl.kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
+  pl.QG = 1;
+  pl.G = 1;
+  pl.qcols = H < 16 ? 16 : H;
+  pl.stage_cols = pl.qcols > 128 ? 256 : 128;
+  pl.n_qt = n_q;
+  pl.rows = batch * n_q;
+  pl.smem = scan_smem_bytes(kind, 1, 1, pl.qcols);
+  const size_t per_sm = 228 * 1024;
+  int by_smem = (int)(per_sm / (pl.smem + 1024));
+  int by_tmem = 512 / (2 * pl.stage_cols);
+  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
+  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
+  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
+  pl.nsub = 8;
+  pl.C = 1;
+  pl.chunk = 0;
+  pl.n_items = batch * n_q;
+  pl.keep = keep;
+  pl.capw = 2 * keep + kCompactSlack + 128;
+  return pl;
+}
+
+// Log bytes of one planned stage (sub-logs, fills, thresholds).
+size_t log_bytes(const ScanPlan& pl) {
+  const size_t slots = (size_t)pl.rows * pl.C;
+  return align_up(slots * pl.nsub * pl.capw * sizeof(uint64_t)) +
+         align_up(slots * pl.nsub * sizeof(int32_t)) +
+         align_up(slots * sizeof(unsigned long long));
+}
+
 // ---------------------------------------------------------- TMA encoding --
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -178,8 +219,22 @@ cudaError_t launch_scan_h(const ScanPlan& pl, const CUtensorMap& qm, const CUten
   }
 }
 
+template <int GATHER>
+cudaError_t launch_scan_gather(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
+                               const ScanArgs& a, cudaStream_t st) {
+  switch (a.H) {  // routed / reranked stages run on bf16 operands
+    case 8: return launch_scan_t<MmaKind::BF16, false, 8, GATHER>(pl, qm, km, a, st);
+    case 16: return launch_scan_t<MmaKind::BF16, false, 16, GATHER>(pl, qm, km, a, st);
+    case 32: return launch_scan_t<MmaKind::BF16, false, 32, GATHER>(pl, qm, km, a, st);
+    case 64: return launch_scan_t<MmaKind::BF16, false, 64, GATHER>(pl, qm, km, a, st);
+    default: return launch_scan_t<MmaKind::BF16, false, 128, GATHER>(pl, qm, km, a, st);
+  }
+}
+
 cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
-                        const ScanArgs& a, cudaStream_t st) {
+                        const ScanArgs& a, cudaStream_t st, int gather = 0) {
+  if (gather == 1) return launch_scan_gather<1>(pl, qm, km, a, st);
+  if (gather == 2) return launch_scan_gather<2>(pl, qm, km, a, st);
   switch (pl.kind) {
     case MmaKind::TF32: return launch_scan_h<MmaKind::TF32, false>(pl, qm, km, a, st);
     case MmaKind::BF16: return launch_scan_h<MmaKind::BF16, false>(pl, qm, km, a, st);
@@ -205,11 +260,20 @@ cudaError_t launch_fin(const FinalArgs& f, int groups, int stage_cap, size_t sme
   return cudaGetLastError();
 }
 
+// Output mapping of a finalize call: row i of sequence b (of nq_c rows per
+// sequence in the logs) is written at row b * nq_total + q_off + i.
+struct OutMap {
+  int nq_c, nq_total, q_off;
+};
+
 cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint64_t* logs,
                             const int32_t* cnt, const unsigned long long* thr, int32_t* out_idx,
-                            float* out_score, cudaStream_t st) {
+                            float* out_score, OutMap om, cudaStream_t st) {
   FinalArgs f{};
   f.rows = pl.rows;
+  f.nq_c = om.nq_c;
+  f.nq_total = om.nq_total;
+  f.q_off = om.q_off;
   f.C = pl.C;
   f.nsub = pl.nsub;
   f.topk = topk;
@@ -371,6 +435,321 @@ int noalloc_scratch_address(void** out) {
   return DSA_OK;
 }
 
+// ------------------------------------------------------------- routed paths --
+// MISA, MISA-dagger and HISA chain scan stages over row chunks: every stage of
+// a chunk writes candidate logs into one shared log region, so the workspace
+// holds the logs of one chunk, bounded by kRouteLogBudget.
+constexpr size_t kRouteLogBudget = 8ull << 30;
+
+int log2_exact(int v) {
+  int s = 0;
+  while ((1 << s) < v) ++s;
+  return s;
+}
+
+struct RouteCfg {
+  int algo;
+  bool route;        // the MISA router runs (MISA, MISA-dagger, stacked HISA)
+  int h, bsR, nblkR, ncolsR;
+  bool hisa;
+  int bsH, nblkH, r;
+  int kp;            // MISA-dagger pool size
+  int hh;            // heads of the token stages
+  int list_len;      // per-row list of the second stage (pool or blocks), 0 for MISA
+};
+
+int route_cfg(const dsa_problem* p, int algo, const dsa_route_params* rp, RouteCfg* c) {
+  if (!rp) return DSA_ERR_INVALID;
+  if (algo != DSA_ALGO_MISA && algo != DSA_ALGO_MISA_DAGGER && algo != DSA_ALGO_HISA)
+    return DSA_ERR_INVALID;
+  if (p->q_dtype != DSA_BF16 || p->k_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
+  if (p->batch > 65535) return DSA_ERR_UNSUPPORTED;
+  *c = RouteCfg{};
+  c->algo = algo;
+  c->route = algo != DSA_ALGO_HISA || rp->misa_h > 0;
+  if (c->route) {
+    if (rp->misa_h < 1 || rp->misa_h > p->heads) return DSA_ERR_INVALID;
+    if (!pow2_in(rp->misa_h, 8, 128)) return DSA_ERR_UNSUPPORTED;
+    if (!pow2_in(rp->misa_block, 16, 4096)) return DSA_ERR_UNSUPPORTED;
+    c->h = rp->misa_h;
+    c->bsR = log2_exact(rp->misa_block);
+    c->nblkR = p->n_k >> c->bsR;
+    if (c->nblkR > kRouterBColsMax) return DSA_ERR_UNSUPPORTED;
+    c->ncolsR = c->nblkR <= 16 ? 16 : (c->nblkR + 15) / 16 * 16;
+  }
+  if (algo == DSA_ALGO_MISA_DAGGER) {
+    if (rp->k_prime < p->topk) return DSA_ERR_INVALID;
+    if (rp->k_prime > 8192) return DSA_ERR_UNSUPPORTED;
+    c->kp = rp->k_prime;
+    c->list_len = c->kp;
+  }
+  if (algo == DSA_ALGO_HISA) {
+    if (!pow2_in(rp->hisa_block, 16, 4096)) return DSA_ERR_UNSUPPORTED;
+    if (rp->hisa_r < 1) return DSA_ERR_INVALID;
+    if (rp->hisa_r > 8192) return DSA_ERR_UNSUPPORTED;
+    c->hisa = true;
+    c->bsH = log2_exact(rp->hisa_block);
+    c->nblkH = p->n_k >> c->bsH;
+    c->r = rp->hisa_r;
+    c->list_len = c->r;
+  }
+  c->hh = c->route ? c->h : p->heads;
+  return DSA_OK;
+}
+
+// Stage plans of one chunk of nq query rows per sequence.
+struct RouteStages {
+  ScanPlan s1;  // MISA: routed scan; MISA-dagger: routed scan keeping k'; HISA: coarse block scan
+  ScanPlan s2;  // MISA-dagger: rerank of the pool; HISA: rerank of the kept blocks' tokens
+  bool two;
+};
+
+RouteStages plan_route(const dsa_problem* p, const RouteCfg& c, int nq) {
+  RouteStages rs{};
+  if (c.algo == DSA_ALGO_MISA) {
+    rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, p->n_k, c.h, p->topk);
+  } else if (c.algo == DSA_ALGO_MISA_DAGGER) {
+    rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, p->n_k, c.h, c.kp);
+    rs.s2 = plan_gather(MmaKind::BF16, p->batch, nq, p->heads, p->topk);
+    rs.two = true;
+  } else {
+    rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, c.nblkH > 0 ? c.nblkH : 1, c.hh, c.r);
+    rs.s2 = plan_gather(MmaKind::BF16, p->batch, nq, c.hh, p->topk);
+    rs.two = true;
+  }
+  return rs;
+}
+
+size_t stages_log_bytes(const RouteStages& rs) {
+  size_t b = log_bytes(rs.s1);
+  if (rs.two) {
+    const size_t b2 = log_bytes(rs.s2);
+    if (b2 > b) b = b2;
+  }
+  return b;
+}
+
+struct RouteLayout {
+  RouteCfg c;
+  int nq_c, n_chunks;
+  size_t fullR_rows, fullH_rows;
+  size_t off_runR, off_fullR, off_heads, off_qg, off_wg, off_runH, off_fullH, off_list, off_logs;
+  size_t total;
+};
+
+RouteLayout route_layout(const dsa_problem* p, const RouteCfg& c) {
+  RouteLayout L{};
+  L.c = c;
+  const size_t rows = (size_t)p->batch * p->n_q;
+  // row chunk: halve until the candidate logs of one chunk fit the budget
+  int nq = p->n_q;
+  while (nq > 16 && stages_log_bytes(plan_route(p, c, nq)) > kRouteLogBudget) nq = (nq + 1) / 2;
+  L.nq_c = nq;
+  L.n_chunks = (p->n_q + nq - 1) / nq;
+  size_t logs = stages_log_bytes(plan_route(p, c, nq));
+  const int last = p->n_q - (L.n_chunks - 1) * nq;  // a short last chunk may split keys more
+  const size_t logs_last = stages_log_bytes(plan_route(p, c, last));
+  if (logs_last > logs) logs = logs_last;
+  size_t off = kWsHeaderBytes;
+  if (c.route) {
+    L.fullR_rows = (size_t)p->batch * (c.nblkR > 0 ? c.nblkR : 1) + 256;
+    L.off_runR = off;
+    off += align_up((size_t)p->batch * p->n_k * 128 * 2);
+    L.off_fullR = off;
+    off += align_up(L.fullR_rows * 128 * 2);
+    L.off_heads = off;
+    off += align_up(rows * c.h * sizeof(int32_t));
+    L.off_qg = off;
+    off += align_up(rows * c.h * 128 * 2);
+    L.off_wg = off;
+    off += align_up(rows * c.h * sizeof(float));
+  }
+  if (c.hisa) {
+    L.fullH_rows = (size_t)p->batch * (c.nblkH > 0 ? c.nblkH : 1) + 128;
+    L.off_runH = off;
+    off += align_up((size_t)p->batch * p->n_k * 128 * 2);
+    L.off_fullH = off;
+    off += align_up(L.fullH_rows * 128 * 2);
+  }
+  L.off_list = off;
+  off += align_up((size_t)p->batch * nq * c.list_len * sizeof(int32_t));
+  L.off_logs = off;
+  off += logs;
+  L.total = off;
+  return L;
+}
+
+struct LogPtrs {
+  uint64_t* logs;
+  int32_t* cnt;
+  unsigned long long* thr;
+};
+
+LogPtrs log_ptrs(const ScanPlan& pl, uint8_t* base) {
+  const size_t slots = (size_t)pl.rows * pl.C;
+  LogPtrs lp;
+  lp.logs = reinterpret_cast<uint64_t*>(base);
+  base += align_up(slots * pl.nsub * pl.capw * sizeof(uint64_t));
+  lp.cnt = reinterpret_cast<int32_t*>(base);
+  base += align_up(slots * pl.nsub * sizeof(int32_t));
+  lp.thr = reinterpret_cast<unsigned long long*>(base);
+  return lp;
+}
+
+// Operands of one bf16 scan stage.
+struct StageIO {
+  const void* q;          // [batch, q_stride, H, 128]
+  const float* w;         // [batch, q_stride, H]
+  int q_stride, H;
+  const void* k;          // key map rows (tokens or block representatives)
+  uint64_t k_rows;        // rows of the key map
+  uint32_t k_box;         // TMA box height of the key map
+  int n_kmap;             // key rows per sequence in the key map
+  int bs_shift;           // > 0: keys are full-block representatives
+  const int32_t* klist;   // gathered stages: per-row lists
+  int klist_len, lb_shift, gather;
+};
+
+int run_stage(const dsa_problem* p, const ScanPlan& pl, const StageIO& io, int q_off, int nq,
+              const LogPtrs& lp, int32_t* status, cudaStream_t st) {
+  CUtensorMap qm, km;
+  if (!make_map(&qm, io.q, 2, (uint64_t)p->batch * io.q_stride * io.H, (uint32_t)pl.qcols))
+    return DSA_ERR_CUDA;
+  if (!make_map(&km, io.k, 2, io.k_rows, io.k_box)) return DSA_ERR_CUDA;
+  ScanArgs a{};
+  a.batch = p->batch;
+  a.n_q = nq;
+  a.n_k = io.n_kmap;
+  a.H = io.H;
+  a.d = p->dim;
+  a.q_stride = io.q_stride;
+  a.q_off = q_off;
+  a.n_tok = p->n_k;
+  a.bs_shift = io.bs_shift;
+  a.klist = io.klist;
+  a.klist_len = io.klist_len;
+  a.lb_shift = io.lb_shift;
+  a.keep = pl.keep;
+  a.QG = pl.QG;
+  a.qcols = pl.qcols;
+  a.G = pl.G;
+  a.stage_cols = pl.stage_cols;
+  a.n_qt = pl.n_qt;
+  a.C = pl.C;
+  a.chunk = pl.chunk;
+  a.n_items = pl.n_items;
+  a.q_pos0 = p->q_pos0;
+  a.k_len = p->k_len;
+  a.w = io.w;
+  a.nsub = pl.nsub;
+  a.capw = pl.capw;
+  a.logs = lp.logs;
+  a.log_cnt = lp.cnt;
+  a.log_thr = lp.thr;
+  a.status = status;
+  return launch_scan(pl, qm, km, a, st, io.gather) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+int launch_pool(const void* k, const dsa_problem* p, int bs_shift, uint8_t* run, uint8_t* full,
+                int nblk, cudaStream_t st) {
+  const int nb = (p->n_k + (1 << bs_shift) - 1) >> bs_shift;
+  pool_prefix_kernel<false><<<dim3((unsigned)nb, (unsigned)p->batch), 128, 0, st>>>(
+      k, p->n_k, bs_shift, run, full, nblk);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+template <int H>
+cudaError_t launch_router_h(const CUtensorMap& am, const CUtensorMap& bm, const CUtensorMap& rm,
+                            const RouterArgs& a, cudaStream_t st) {
+  const int smem = (int)router_smem_bytes();
+  cudaError_t e =
+      cudaFuncSetAttribute(router_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int grid = a.n_tiles < sms ? a.n_tiles : sms;
+  if (grid < 1) grid = 1;
+  router_kernel<H><<<grid, kRouterThreads, smem, st>>>(am, bm, rm, a);
+  return cudaGetLastError();
+}
+
+// Pooling + router: heads, optional E, gathered q / w rows of every query.
+int run_router(const dsa_problem* p, const RouteLayout& L, const void* q, const void* k,
+               const float* w, int32_t* heads, float* E, uint8_t* ws, cudaStream_t st) {
+  const RouteCfg& c = L.c;
+  uint8_t* runR = ws + L.off_runR;
+  uint8_t* fullR = ws + L.off_fullR;
+  int rc = launch_pool(k, p, c.bsR, runR, fullR, c.nblkR, st);
+  if (rc != DSA_OK) return rc;
+  CUtensorMap am, bm, rm;
+  if (!make_map(&am, q, 2, (uint64_t)p->batch * p->n_q * p->heads, 128)) return DSA_ERR_CUDA;
+  if (!make_map(&bm, fullR, 2, L.fullR_rows, (uint32_t)c.ncolsR)) return DSA_ERR_CUDA;
+  if (!make_map(&rm, runR, 2, (uint64_t)p->batch * p->n_k, 1)) return DSA_ERR_CUDA;
+  RouterArgs a{};
+  a.batch = p->batch;
+  a.n_q = p->n_q;
+  a.n_tok = p->n_k;
+  a.H = p->heads;
+  a.h = c.h;
+  a.bs_shift = c.bsR;
+  a.nblk = c.nblkR;
+  a.ncols = c.ncolsR;
+  a.tiles_per_seq = (p->n_q * p->heads + 127) / 128;
+  a.n_tiles = p->batch * a.tiles_per_seq;
+  a.q_pos0 = p->q_pos0;
+  a.k_len = p->k_len;
+  a.q = reinterpret_cast<const uint16_t*>(q);
+  a.w = w;
+  a.heads = heads;
+  a.E = E;
+  a.qg = reinterpret_cast<uint16_t*>(ws + L.off_qg);
+  a.wg = reinterpret_cast<float*>(ws + L.off_wg);
+  a.status = reinterpret_cast<int32_t*>(ws);
+  cudaError_t e;
+  switch (p->heads) {
+    case 8: e = launch_router_h<8>(am, bm, rm, a, st); break;
+    case 16: e = launch_router_h<16>(am, bm, rm, a, st); break;
+    case 32: e = launch_router_h<32>(am, bm, rm, a, st); break;
+    case 64: e = launch_router_h<64>(am, bm, rm, a, st); break;
+    default: e = launch_router_h<128>(am, bm, rm, a, st); break;
+  }
+  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// Copy a chunk's per-row lists [batch, nq, len] into rows q_off.. of out [batch, n_q, len].
+int copy_lists(int32_t* out, const int32_t* lists, const dsa_problem* p, int q_off, int nq,
+               int len, cudaStream_t st) {
+  const size_t row = (size_t)len * sizeof(int32_t);
+  return cudaMemcpy2DAsync(out + (size_t)q_off * len, (size_t)p->n_q * row, lists, (size_t)nq * row,
+                           (size_t)nq * row, (size_t)p->batch, cudaMemcpyDeviceToDevice,
+                           st) == cudaSuccess
+             ? DSA_OK
+             : DSA_ERR_CUDA;
+}
+
+// Shared set-up of the routed entry points: validation, layout, status reset,
+// optional device checks.
+int route_begin(const dsa_problem* p, int algo, const dsa_route_params* rp, const void* q,
+                const void* k, const float* w, int32_t* out_idx, float* out_score, void* ws,
+                size_t ws_bytes, cudaStream_t st, RouteLayout* L) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  RouteCfg c;
+  v = route_cfg(p, algo, rp, &c);
+  if (v != DSA_OK) return v;
+  if (!q || !k || !w || !out_idx || !out_score) return DSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID;
+  *L = route_layout(p, c);
+  if (!ws || ws_bytes < L->total) return DSA_ERR_WORKSPACE;
+  uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
+  if (cudaMemsetAsync(w8, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (p->flags & DSA_FLAG_CHECK)
+    check_inputs_kernel<<<64, 256, 0, st>>>(nullptr, 0, nullptr, 0, p->q_pos0, p->k_len, p->batch,
+                                            p->n_k, reinterpret_cast<int32_t*>(w8));
+  return DSA_OK;
+}
+
 }  // namespace
 
 // ===================================================================== ABI ==
@@ -404,12 +783,15 @@ int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_param
   if (!bytes) return DSA_ERR_INVALID;
   int v = validate_problem(p);
   if (v != DSA_OK) return v;
-  (void)rp;
   if (algo == DSA_ALGO_DSA) {
     *bytes = dsa_layout(p).total;
     return DSA_OK;
   }
-  return DSA_ERR_UNSUPPORTED;
+  RouteCfg c;
+  v = route_cfg(p, algo, rp, &c);
+  if (v != DSA_OK) return v;
+  *bytes = route_layout(p, c).total;
+  return DSA_OK;
 }
 
 int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
@@ -458,6 +840,8 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.n_k = p->n_k;
   a.H = p->heads;
   a.d = p->dim;
+  a.q_stride = p->n_q;
+  a.q_off = 0;
   a.n_tok = p->n_k;
   a.bs_shift = 0;
   a.klist = nullptr;
@@ -465,6 +849,7 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.lb_shift = 0;
   a.keep = p->topk;
   a.QG = pl.QG;
+  a.qcols = pl.qcols;
   a.G = pl.G;
   a.stage_cols = pl.stage_cols;
   a.n_qt = pl.n_qt;
@@ -501,7 +886,7 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
   if (launch_finalize(pl, p->topk, sorted, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
                       reinterpret_cast<const int32_t*>(ws + L.off_cnt),
                       reinterpret_cast<const unsigned long long*>(ws + L.off_thr), out_idx,
-                      out_score, st) != cudaSuccess)
+                      out_score, OutMap{p->n_q, p->n_q, 0}, st) != cudaSuccess)
     return DSA_ERR_CUDA;
   return finish(p, workspace, st);
 }
@@ -542,26 +927,198 @@ int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
 int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
                const float* w, int32_t* out_idx, float* out_score, int32_t* out_heads,
                float* out_E, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
-  (void)out_heads; (void)out_E; (void)workspace; (void)workspace_bytes; (void)stream;
-  return DSA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RouteLayout L;
+  int rc = route_begin(p, DSA_ALGO_MISA, rp, q, k, w, out_idx, out_score, workspace,
+                       workspace_bytes, st, &L);
+  if (rc != DSA_OK) return rc;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
+  rc = run_router(p, L, q, k, w, heads, out_E, ws, st);
+  if (rc != DSA_OK) return rc;
+  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  for (int ci = 0; ci < L.n_chunks; ++ci) {
+    const int q_off = ci * L.nq_c;
+    const int nq = p->n_q - q_off < L.nq_c ? p->n_q - q_off : L.nq_c;
+    const RouteStages rs = plan_route(p, L.c, nq);
+    const LogPtrs lp = log_ptrs(rs.s1, ws + L.off_logs);
+    StageIO io{};
+    io.q = ws + L.off_qg;
+    io.w = reinterpret_cast<const float*>(ws + L.off_wg);
+    io.q_stride = p->n_q;
+    io.H = L.c.h;
+    io.k = k;
+    io.k_rows = (uint64_t)p->batch * p->n_k;
+    io.k_box = 128;
+    io.n_kmap = p->n_k;
+    rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (launch_finalize(rs.s1, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
+                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return finish(p, workspace, st);
 }
 
 int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
                       const void* k, const float* w, int32_t* out_idx, float* out_score,
                       int32_t* out_heads, int32_t* out_pool, void* workspace,
                       size_t workspace_bytes, void* stream) {
-  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
-  (void)out_heads; (void)out_pool; (void)workspace; (void)workspace_bytes; (void)stream;
-  return DSA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RouteLayout L;
+  int rc = route_begin(p, DSA_ALGO_MISA_DAGGER, rp, q, k, w, out_idx, out_score, workspace,
+                       workspace_bytes, st, &L);
+  if (rc != DSA_OK) return rc;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
+  rc = run_router(p, L, q, k, w, heads, nullptr, ws, st);
+  if (rc != DSA_OK) return rc;
+  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  int32_t* pool = reinterpret_cast<int32_t*>(ws + L.off_list);
+  for (int ci = 0; ci < L.n_chunks; ++ci) {
+    const int q_off = ci * L.nq_c;
+    const int nq = p->n_q - q_off < L.nq_c ? p->n_q - q_off : L.nq_c;
+    const RouteStages rs = plan_route(p, L.c, nq);
+    // pass 1: routed heads, keep k' candidates
+    LogPtrs lp = log_ptrs(rs.s1, ws + L.off_logs);
+    StageIO io{};
+    io.q = ws + L.off_qg;
+    io.w = reinterpret_cast<const float*>(ws + L.off_wg);
+    io.q_stride = p->n_q;
+    io.H = L.c.h;
+    io.k = k;
+    io.k_rows = (uint64_t)p->batch * p->n_k;
+    io.k_box = 128;
+    io.n_kmap = p->n_k;
+    rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (launch_finalize(rs.s1, L.c.kp, 0, lp.logs, lp.cnt, lp.thr, pool, nullptr,
+                        OutMap{nq, nq, 0}, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (out_pool) {
+      rc = copy_lists(out_pool, pool, p, q_off, nq, L.c.kp, st);
+      if (rc != DSA_OK) return rc;
+    }
+    // pass 2: every head on the pool's tokens
+    lp = log_ptrs(rs.s2, ws + L.off_logs);
+    StageIO io2{};
+    io2.q = q;
+    io2.w = w;
+    io2.q_stride = p->n_q;
+    io2.H = p->heads;
+    io2.k = k;
+    io2.k_rows = (uint64_t)p->batch * p->n_k;
+    io2.k_box = 1;                      // gather4 rows
+    io2.n_kmap = p->n_k;
+    io2.klist = pool;
+    io2.klist_len = L.c.kp;
+    io2.gather = 1;
+    rc = run_stage(p, rs.s2, io2, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (launch_finalize(rs.s2, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
+                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return finish(p, workspace, st);
 }
 
 int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
                const float* w, int32_t* out_idx, float* out_score, int32_t* out_blocks,
                int32_t* out_heads, void* workspace, size_t workspace_bytes, void* stream) {
-  (void)p; (void)rp; (void)q; (void)k; (void)w; (void)out_idx; (void)out_score;
-  (void)out_blocks; (void)out_heads; (void)workspace; (void)workspace_bytes; (void)stream;
-  return DSA_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RouteLayout L;
+  int rc = route_begin(p, DSA_ALGO_HISA, rp, q, k, w, out_idx, out_score, workspace,
+                       workspace_bytes, st, &L);
+  if (rc != DSA_OK) return rc;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  const RouteCfg& c = L.c;
+  const void* qs = q;
+  const float* wsrc = w;
+  if (c.route) {
+    int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
+    rc = run_router(p, L, q, k, w, heads, nullptr, ws, st);
+    if (rc != DSA_OK) return rc;
+    qs = ws + L.off_qg;
+    wsrc = reinterpret_cast<const float*>(ws + L.off_wg);
+  }
+  uint8_t* runH = ws + L.off_runH;
+  uint8_t* fullH = ws + L.off_fullH;
+  rc = launch_pool(k, p, c.bsH, runH, fullH, c.nblkH, st);
+  if (rc != DSA_OK) return rc;
+  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  int32_t* blocks = reinterpret_cast<int32_t*>(ws + L.off_list);
+  for (int ci = 0; ci < L.n_chunks; ++ci) {
+    const int q_off = ci * L.nq_c;
+    const int nq = p->n_q - q_off < L.nq_c ? p->n_q - q_off : L.nq_c;
+    const RouteStages rs = plan_route(p, c, nq);
+    // coarse: the full blocks' representatives scored like keys, keep r
+    LogPtrs lp = log_ptrs(rs.s1, ws + L.off_logs);
+    StageIO io{};
+    io.q = qs;
+    io.w = wsrc;
+    io.q_stride = p->n_q;
+    io.H = c.hh;
+    io.k = fullH;
+    io.k_rows = L.fullH_rows;
+    io.k_box = 128;
+    io.n_kmap = c.nblkH > 0 ? c.nblkH : 1;
+    io.bs_shift = c.bsH;
+    rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    // the boundary block of every row joins its candidates
+    BoundaryArgs ba{};
+    ba.batch = p->batch;
+    ba.n_q = nq;
+    ba.q_stride = p->n_q;
+    ba.q_off = q_off;
+    ba.n_tok = p->n_k;
+    ba.H = c.hh;
+    ba.bs_shift = c.bsH;
+    ba.q_pos0 = p->q_pos0;
+    ba.k_len = p->k_len;
+    ba.q = reinterpret_cast<const uint16_t*>(qs);
+    ba.w = wsrc;
+    ba.run = reinterpret_cast<const uint16_t*>(runH);
+    ba.C = rs.s1.C;
+    ba.nsub = rs.s1.nsub;
+    ba.capw = rs.s1.capw;
+    ba.logs = lp.logs;
+    ba.log_cnt = lp.cnt;
+    const long long rows = (long long)p->batch * nq;
+    boundary_candidate_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(ba);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    if (launch_finalize(rs.s1, c.r, 0, lp.logs, lp.cnt, lp.thr, blocks, nullptr,
+                        OutMap{nq, nq, 0}, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (out_blocks) {
+      rc = copy_lists(out_blocks, blocks, p, q_off, nq, c.r, st);
+      if (rc != DSA_OK) return rc;
+    }
+    // fine: the kept blocks' legal tokens with the full formula
+    lp = log_ptrs(rs.s2, ws + L.off_logs);
+    StageIO io2{};
+    io2.q = qs;
+    io2.w = wsrc;
+    io2.q_stride = p->n_q;
+    io2.H = c.hh;
+    io2.k = k;
+    io2.k_rows = (uint64_t)p->batch * p->n_k;
+    io2.k_box = c.bsH < 7 ? (1u << c.bsH) : 128u;
+    io2.n_kmap = p->n_k;
+    io2.klist = blocks;
+    io2.klist_len = c.r;
+    io2.lb_shift = c.bsH;
+    io2.gather = 2;
+    rc = run_stage(p, rs.s2, io2, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (launch_finalize(rs.s2, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
+                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
+  return finish(p, workspace, st);
 }
 
 }  // extern "C"

@@ -54,6 +54,7 @@ struct ScanArgs {
   int32_t lb_shift;      // block lists: log2 tokens per listed block
   int32_t keep;          // entries each row must keep (top-k or k')
   int32_t QG;            // query rows per accumulator group (<= 256 / (H * parts))
+  int32_t qcols;         // MMA N per group: max(16, QG * H * parts) query-head columns
   int32_t G;             // groups per work item (1 or 2)
   int32_t stage_cols;    // TMEM columns per accumulator stage (128 or 256)
   int32_t n_qt;          // query tiles per sequence (ceil(n_q / (QG*G)))
@@ -137,10 +138,12 @@ __device__ __forceinline__ ItemGeom item_geom(const ScanArgs& a, int item) {
   g.row0 = g.qt * QT;
   g.nrows = min(QT, a.n_q - g.row0);
   if constexpr (GATHER != 0) {
-    // one row per item; its keys come from its list, in list order
+    // one row per item; its keys come from its list, in list order (a block
+    // list expands each entry into 2^lb_shift consecutive tokens)
+    const int nkeys = GATHER == 2 ? (a.klist_len << a.lb_shift) : a.klist_len;
     g.kbeg = 0;
-    g.kend = a.klist_len;
-    g.ntiles = g.nrows > 0 ? (a.klist_len + 127) >> 7 : 0;
+    g.kend = nkeys;
+    g.ntiles = g.nrows > 0 ? (nkeys + 127) >> 7 : 0;
     g.t_hi = 0;
     return g;
   }
@@ -343,11 +346,12 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
   } else {
     // HT in {8, 16}: one 32-column chunk holds 32 / HT query rows
     constexpr int QPC = 32 / HT;
-    const int nchunk = nq / QPC;
+    const int nchunk = (nq + QPC - 1) / QPC;
     uint32_t va[1][32], vb[1][32];
     auto chunk = [&](const uint32_t (&v)[1][32], int c) {
 #pragma unroll
       for (int qq = 0; qq < QPC; ++qq) {
+        if (c * QPC + qq >= nq) break;
         float b[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int jj = 0; jj < HT; jj += 4) {
@@ -387,7 +391,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   // 1024-byte aligned base; plain pointer arithmetic on the __shared__ array
   // keeps the shared address space visible to the compiler (LDS/ATOMS, not generic)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int qcols = a.QG * a.H * PARTS;                     // MMA N per group
+  const int qcols = a.qcols;                                // MMA N per group
   const int QT = a.QG * a.G;
   uint8_t* Qs = smem;                                       // [G][A][qcols x 128B]
   const int q_bytes = a.G * Cfg::A * qcols * 128;

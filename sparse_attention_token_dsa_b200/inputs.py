@@ -88,6 +88,33 @@ def integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, d
                    None if k_len is None else np.asarray(k_len, np.int32), name="integer")
 
 
+def segment_integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int,
+                            dim: int, topk: int, seg: int, q_pos0=None, k_len=None) -> Problem:
+    """Integer problem whose keys are constant on aligned segments of `seg` tokens.
+
+    q uniform integers in [-3, 3], w in [-2, 2]; every key of segment i equals
+    an integer vector c_i in [-2, 2]^d except the segment's last token, which
+    is c_i + e_i with e_i integers in [-1, 1]^d (bf16 storage, exact).  Any
+    mean over a prefix of a power-of-two block aligned inside a segment is
+    either c_i or c_i + e_i / (block size): a dyadic number with a small
+    numerator, so pooled keys, their dot products with q and the sums over
+    heads and blocks stay exactly representable in fp32 at the test sizes.
+    """
+    q = _rng(workload, 1).integers(-3, 4, size=(batch, n_q, heads, dim)).astype(np.float32)
+    r = _rng(workload, 2)
+    nseg = (n_k + seg - 1) // seg
+    c = r.integers(-2, 3, size=(batch, nseg, dim)).astype(np.float32)
+    e = r.integers(-1, 2, size=(batch, nseg, dim)).astype(np.float32)
+    k = np.repeat(c, seg, axis=1)[:, :n_k].copy()
+    last = np.arange(seg - 1, n_k, seg)
+    k[:, last] += e[:, : len(last)]
+    w = _rng(workload, 3).integers(-2, 3, size=(batch, n_q, heads)).astype(np.float32)
+    return Problem(batch, n_q, n_k, heads, dim, topk, BF16, BF16, f32_to_bf16_bits(q),
+                   f32_to_bf16_bits(k), w,
+                   None if q_pos0 is None else np.asarray(q_pos0, np.int32),
+                   None if k_len is None else np.asarray(k_len, np.int32), name="segments")
+
+
 def normal_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, dim: int,
                    topk: int, q_pos0=None, k_len=None, n_needles: int = 0,
                    key_structure: str = "iid", n_centres: int = 256,

@@ -91,3 +91,72 @@ def test_quantize_rejects(bind):
     assert f(None, 1, 4, 128, fake, fake, None) == -1
     assert f(fake, 2, 4, 128, fake, fake, None) == -2
     assert f(fake, 1, 4, 0, fake, fake, None) == -1
+
+
+def _ws(bind, p, algo, rp):
+    n = C.c_size_t(0)
+    rc = bind.lib.dsa_workspace_size(C.byref(p), algo, None if rp is None else C.byref(rp),
+                                     C.byref(n))
+    return rc, n.value
+
+
+@pytest.mark.parametrize("algo,rp,status", [
+    (1, None, -1),                                                  # route params required
+    (1, dict(misa_block=128, misa_h=8), 0),
+    (1, dict(misa_block=100, misa_h=8), -2),                         # block not a power of two
+    (1, dict(misa_block=128, misa_h=12), -2),                        # h not a power of two
+    (1, dict(misa_block=128, misa_h=128), -1),                       # h > heads
+    (1, dict(misa_block=8, misa_h=8), -2),                           # block below 16
+    (2, dict(misa_block=128, misa_h=8, k_prime=4), -1),              # k' < topk
+    (2, dict(misa_block=128, misa_h=8, k_prime=9000), -2),           # k' above 8192
+    (2, dict(misa_block=128, misa_h=8, k_prime=64), 0),
+    (3, dict(hisa_block=64, hisa_r=0), -1),                          # r < 1
+    (3, dict(hisa_block=64, hisa_r=16), 0),
+    (3, dict(hisa_block=64, hisa_r=16, misa_block=128, misa_h=8), 0),  # stacked
+    (3, dict(hisa_block=48, hisa_r=16), -2),
+    (7, dict(hisa_block=64, hisa_r=16), -1),                         # unknown algorithm
+])
+def test_route_workspace_validation(bind, algo, rp, status):
+    p = _prob(bind, n_q=256, n_k=1024)
+    rc, n = _ws(bind, p, algo, None if rp is None else bind.route_params(**rp))
+    assert rc == status
+    if status == 0:
+        assert n > 0
+
+
+def test_route_rejects_unsupported_operands(bind):
+    rp = bind.route_params(misa_block=128, misa_h=8)
+    assert _ws(bind, _prob(bind, q_dtype=0, k_dtype=0), 1, rp)[0] == -2      # fp32: bf16 only
+    assert _ws(bind, _prob(bind, q_dtype=1, k_dtype=2), 1, rp)[0] == -2      # e4m3 keys
+    # more than 224 full router blocks per sequence
+    assert _ws(bind, _prob(bind, n_k=225 * 16), 1, bind.route_params(misa_block=16, misa_h=8))[0] == -2
+    assert _ws(bind, _prob(bind, n_k=224 * 16), 1, bind.route_params(misa_block=16, misa_h=8))[0] == 0
+
+
+def test_route_workspace_is_bounded_by_row_chunks(bind):
+    """The candidate logs of 128K prefill rows are chunked: the workspace stays far
+    below rows x per-row log size."""
+    p = _prob(bind, n_q=131072, n_k=131072, topk=2048)
+    rc, n = _ws(bind, p, 2, bind.route_params(misa_block=1024, misa_h=8, k_prime=8192))
+    assert rc == 0
+    per_row_pass1 = 4 * (2 * 8192 + 768) * 8
+    assert n < 131072 * per_row_pass1 / 4
+    rc, n2 = _ws(bind, p, 3, bind.route_params(hisa_block=64, hisa_r=128))
+    assert rc == 0 and n2 > 0
+
+
+def test_route_entry_points_reject_before_launch(bind):
+    p = _prob(bind, n_q=256, n_k=1024)
+    rp = bind.route_params(misa_block=128, misa_h=8, k_prime=64, hisa_block=64, hisa_r=16)
+    fake = C.c_void_p(0x1000)
+    L = bind.lib
+    assert L.misa_index(C.byref(p), None, fake, fake, fake, fake, fake, None, None, fake,
+                        1 << 40, None) == -1
+    assert L.misa_index(C.byref(p), C.byref(rp), None, fake, fake, fake, fake, None, None, fake,
+                        1 << 40, None) == -1
+    assert L.misa_index(C.byref(p), C.byref(rp), fake, fake, fake, fake, fake, None, None, fake,
+                        16, None) == -3
+    assert L.misa_dagger_index(C.byref(p), C.byref(rp), fake, fake, fake, None, fake, None, None,
+                               fake, 1 << 40, None) == -1
+    assert L.hisa_index(C.byref(p), C.byref(rp), fake, fake, fake, fake, fake, None, None, None,
+                        0, None) == -3

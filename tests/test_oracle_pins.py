@@ -273,6 +273,46 @@ def test_hisa_coarse_closed_form(oracle_mod):
     assert list(h["idx"][0]) == list(range(16, 22))
 
 
+def test_block_scores_closed_form(oracle_mod):
+    """Same block-constant keys: J_b = w q c_b for every block, in block order."""
+    d, blk, nblk = 4, 8, 10
+    c = np.array([3, -1, 7, 7, 2, 0, 5, 1, 6, 4], np.float32)
+    k = np.zeros((1, blk * nblk, d), np.float32)
+    k[0, :, 0] = np.repeat(c, blk)
+    q = np.zeros((1, 1, 8, d), np.float32)
+    q[0, 0, 0, 0] = 1.0
+    w = np.zeros((1, 1, 8), np.float32)
+    w[0, 0, 0] = 2.0
+    p = make(q, k, w, topk=6)
+    J = oracle_mod.block_scores(oracle_mod.Inputs(p), 0, blk)
+    assert np.array_equal(J, 2.0 * np.maximum(c, 0))
+
+
+def test_block_scores_with_unit_blocks_are_token_scores(oracle_mod):
+    """b = 1: every block is one token, so J is the DSA score row (any head list)."""
+    p = gen.normal_problem(61, 1, 40, 40, 16, 128, 8)
+    inp = oracle_mod.Inputs(p)
+    for row in (0, 17, 39):
+        assert np.array_equal(oracle_mod.block_scores(inp, row, 1), oracle_mod.score_row(inp, row))
+        hs = np.array([1, 4, 9], np.int32)
+        assert np.array_equal(oracle_mod.block_scores(inp, row, 1, hs),
+                              oracle_mod.score_row(inp, row, hs))
+
+
+def test_segment_problem_pooled_keys_are_exact(oracle_mod):
+    """Segment-structured integer keys: every pooled key (full or boundary block,
+    block sizes dividing the segment) is c or c + e / blocksize exactly."""
+    p = gen.segment_integer_problem(62, 1, 200, 200, 8, 128, 8, seg=64)
+    inp = oracle_mod.Inputs(p)
+    k = gen.bf16_bits_to_f32(p.k)[0].astype(np.float64)
+    for blk in (16, 64):
+        for n in (37, 64, 150, 200):
+            reps = oracle_mod.pool(inp, 0, n, blk)
+            for a in range(reps.shape[0]):
+                lo, hi = a * blk, min((a + 1) * blk, n)
+                assert np.array_equal(reps[a], k[lo:hi].mean(0))
+
+
 # ----------------------------------------------------------------- E4M3 codec --
 
 def test_e4m3_ocp_values(oracle_mod):
