@@ -111,11 +111,18 @@ typedef struct {
 
 /* Routing / hierarchy parameters (ignored fields may be zero).
  *   misa_block  B  : tokens per pooled key of the MISA router (e.g. 1024)
- *   misa_h      h  : routed heads kept per query (e.g. 8), 1 <= h <= heads
- *   k_prime     k' : MISA-dagger candidate pool (e.g. 8192), k' >= topk
+ *   misa_h      h  : routed heads kept per query (e.g. 8); a power of two in
+ *                    [8, heads]
+ *   k_prime     k' : MISA-dagger candidate pool (e.g. 8192), topk <= k' <= 8192
  *   hisa_block  b  : tokens per HISA block (e.g. 64)
- *   hisa_r      r  : HISA blocks kept per query (e.g. 128)
- * Block sizes must be powers of two in [16, 4096]. */
+ *   hisa_r      r  : HISA blocks kept per query (e.g. 128), 1 <= r <= 8192
+ * Block sizes must be powers of two in [16, 4096], and the router sees at
+ * most 224 full blocks: n_k / B <= 224 (B = 1024 covers 229,376 tokens).
+ * The routed entry points take bf16 q and k only (q_dtype == k_dtype ==
+ * DSA_BF16; anything else returns DSA_ERR_UNSUPPORTED) and batch <= 65535.
+ * Their workspace holds the pooled keys, the routed query rows and the
+ * candidate logs of one chunk of query rows; long prefills run in several
+ * row chunks so that the logs stay within 8 GiB. */
 typedef struct {
   int32_t misa_block;
   int32_t misa_h;
@@ -128,6 +135,12 @@ typedef struct {
  * may be NULL for DSA_ALGO_DSA).  Writes *bytes; returns a status. */
 int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
                        size_t* bytes);
+
+/* Query rows per sequence that a routed entry point (algo MISA, MISA_DAGGER or
+ * HISA) processes per row chunk for problem p: its scan and select launches
+ * repeat once per chunk of *rows rows.  Host only; returns a status. */
+int dsa_route_chunk_rows(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
+                         int32_t* rows);
 
 /* DSA lightning-indexer top-k: score -> causal mask -> token top-k. */
 int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
@@ -167,7 +180,10 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
 /* MISA: block-pooled router picks rp->misa_h heads per query, those heads score
  * every legal token, token top-k.  out_heads [batch,n_q,h] int32 (ascending head
  * order) and out_E [batch,n_q,heads] fp32 (the router importance E) are optional
- * (NULL skips them).  Supports q_dtype == k_dtype in {F32, BF16}. */
+ * (NULL skips them).  Router: full blocks of the legal prefix plus the boundary
+ * block (the mean of its legal tokens); heads ranked by
+ * S_{t,j} = sum_b |w_{t,j}| ReLU(q_{t,j} . k~_b) = M_t E_{t,j}, ties to the
+ * lower head index. */
 int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
                const void* k, const float* w, int32_t* out_idx, float* out_score,
                int32_t* out_heads, float* out_E, void* workspace, size_t workspace_bytes,

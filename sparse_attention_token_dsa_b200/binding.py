@@ -54,6 +54,7 @@ def _load():
     lib.dsa_read_status.argtypes = [vp, vp]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_route_chunk_rows.argtypes = [P, i32, R, C.POINTER(i32)]
     lib.dsa_index_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.dsa_index_scan.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_index_select.argtypes = [P, vp, vp, vp, sz, vp]
@@ -61,7 +62,8 @@ def _load():
     lib.misa_dagger_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
-    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_index", "dsa_index_noalloc",
+    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
+              "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
               "misa_dagger_index", "hisa_index", "dsa_quantize_e4m3"):
@@ -118,6 +120,14 @@ def dsa_workspace_size(p: DsaProblem, algo: int = DSA_ALGO_DSA, rp: DsaRoutePara
     n = C.c_size_t(0)
     _check(lib.dsa_workspace_size(C.byref(p), algo, None if rp is None else C.byref(rp),
                                   C.byref(n)), "dsa_workspace_size")
+    return n.value
+
+
+def dsa_route_chunk_rows(p: DsaProblem, algo: int, rp: DsaRouteParams) -> int:
+    """Query rows per sequence of one row chunk of a routed entry point."""
+    n = C.c_int32(0)
+    _check(lib.dsa_route_chunk_rows(C.byref(p), algo, C.byref(rp), C.byref(n)),
+           "dsa_route_chunk_rows")
     return n.value
 
 

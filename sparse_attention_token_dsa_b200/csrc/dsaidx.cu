@@ -794,6 +794,18 @@ int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_param
   return DSA_OK;
 }
 
+int dsa_route_chunk_rows(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
+                         int32_t* rows) {
+  if (!rows) return DSA_ERR_INVALID;
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  RouteCfg c;
+  v = route_cfg(p, algo, rp, &c);
+  if (v != DSA_OK) return v;
+  *rows = route_layout(p, c).nq_c;
+  return DSA_OK;
+}
+
 int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
                    const float* k_scale, const float* w, void* workspace, size_t workspace_bytes,
                    void* stream) {
