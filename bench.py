@@ -55,6 +55,15 @@ WORKLOADS = {
         desc="DSA indexer decode, 32 sequences x 131072 cached keys, one query each, H_I=64, "
              "d=128, e4m3 K with per-token fp32 scale, bf16 q, fp32 w, top-k=2048",
         kind="decode", batch=32, L=131072, H=64, topk=2048, fp8=True, seed=3, needles=0),
+    "misa_prefill_16k": dict(
+        desc="MISA prefill, batch 1, L=16384 causal, H_I=64, d=128, B=1024, h=8, top-k=2048, "
+             "bf16 (small case of the 128K workload, sized for ncu captures)",
+        kind="misa", batch=1, L=16384, H=64, topk=2048, seed=4, block=1024, h=8),
+    "hisa_prefill_16k": dict(
+        desc="HISA prefill, batch 1, L=16384 causal, H_I=64, d=128, b=64, r=128, top-k=2048, "
+             "bf16, clustered keys (small case of the 128K workload, sized for ncu captures)",
+        kind="hisa", batch=1, L=16384, H=64, topk=2048, seed=5, hb=64, r=128, h=0,
+        block=1024, keys="clusters"),
     "dsa_prefill_128k": dict(
         desc="DSA indexer prefill, batch 1, L=131072 causal, H_I=64, d=128, top-k=2048, "
              "bf16 q,k ~N(0,1), w ~N(0,1/64) (the dense scan MISA and HISA reduce)",

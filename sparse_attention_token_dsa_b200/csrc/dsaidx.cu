@@ -32,7 +32,7 @@ bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1))
 struct ScanPlan {
   MmaKind kind;
   bool split;
-  int parts, esz, atoms, kstages;
+  int parts, esz, atoms, kstages, tstages;
   int QG, G, qcols, stage_cols, n_qt, C, chunk, n_items, keep, nsub, capw;
   int rows;
   size_t smem;
@@ -41,14 +41,40 @@ struct ScanPlan {
 
 constexpr size_t kSmemBudget = 227 * 1024;
 
-size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols) {
+// Dynamic shared memory of the scan: alignment slack, Q tiles, K stages, then
+// the per-row histograms (streaming rows) or the candidate array (gathered rows).
+size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols, int kstages, bool gather) {
   const int esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   const int atoms = esz;  // d = 128
-  const int kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
   size_t q = align_up((size_t)G * atoms * qcols * 128, 1024);
   size_t k = (size_t)kstages * atoms * 128 * 128;
-  size_t h = (size_t)G * QG * kHistWords * sizeof(uint32_t);
+  size_t h = gather ? (size_t)kMaxGatherKeys * sizeof(uint64_t) +
+                          (size_t)kGatherBins * sizeof(uint32_t) +
+                          (size_t)kGatherBoundary * sizeof(uint64_t)
+                    : (size_t)G * QG * kHistWords * sizeof(uint32_t);
   return 1024 + q + k + h + sizeof(ScanSmemTail);
+}
+
+// Residency and pipeline depths of a planned scan: CTAs per SM from shared
+// memory and TMEM; a CTA alone on its SM deepens its K pipeline into the
+// spare shared memory, and the TMEM accumulator stages fill 512 columns.
+void finish_plan(ScanPlan& pl, bool gather) {
+  const size_t per_sm = 228 * 1024;
+  pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather);
+  int by_smem = (int)(per_sm / (pl.smem + 1024));
+  int by_tmem = 512 / (2 * pl.stage_cols);
+  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
+  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
+  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
+  if (pl.ctas_per_sm == 1) {
+    while (pl.kstages < 6 &&
+           scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages + 1, gather) <= kSmemBudget)
+      ++pl.kstages;
+    pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather);
+  }
+  pl.tstages = 512 / (pl.ctas_per_sm * pl.stage_cols);
+  if (pl.tstages > kMaxTStages) pl.tstages = kMaxTStages;
+  if (pl.tstages < 2) pl.tstages = 2;
 }
 
 // H: heads scanned; n_q / n_k / batch: geometry; keep: entries kept per row.
@@ -59,7 +85,7 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.parts = split ? 2 : 1;
   pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   pl.atoms = pl.esz;
-  pl.kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
+  pl.kstages = kind == MmaKind::E4M3 ? 4 : 2;
   const int ncols_max = kind == MmaKind::TF32 ? 128 : 256;
   const int hp = H * pl.parts;
   int QG = ncols_max / hp;
@@ -70,7 +96,8 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   G = 1;
 #endif
   // fit the shared-memory budget and the per-item row limit
-  while (G * QG > kMaxRows || scan_smem_bytes(kind, G, QG, QG * hp) > kSmemBudget) {
+  while (G * QG > kMaxRows ||
+         scan_smem_bytes(kind, G, QG, QG * hp, pl.kstages, false) > kSmemBudget) {
     if (G == 2) G = 1;
     else if (QG > qg_min) QG /= 2;
     else break;
@@ -81,13 +108,7 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.stage_cols = pl.qcols > 128 ? 256 : 128;
   pl.n_qt = (n_q + QG * G - 1) / (QG * G);
   pl.rows = batch * n_q;
-  pl.smem = scan_smem_bytes(kind, G, QG, pl.qcols);
-  const size_t per_sm = 228 * 1024;
-  int by_smem = (int)(per_sm / (pl.smem + 1024));
-  int by_tmem = 512 / (2 * pl.stage_cols);
-  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
-  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
-  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
+  finish_plan(pl, false);
   pl.nsub = QG == 1 ? 8 : 4;
   // split-K over keys when there are too few query tiles to fill the GPU
   const long long tiles = (long long)batch * pl.n_qt;
@@ -122,26 +143,21 @@ ScanPlan plan_gather(MmaKind kind, int batch, int n_q, int H, int keep) {
   pl.parts = 1;
   pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   pl.atoms = pl.esz;
-  pl.kstages = kind == MmaKind::E4M3 ? 4 : (kind == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
+  pl.kstages = 2;
   pl.QG = 1;
   pl.G = 1;
   pl.qcols = H < 16 ? 16 : H;
   pl.stage_cols = pl.qcols > 128 ? 256 : 128;
   pl.n_qt = n_q;
   pl.rows = batch * n_q;
-  pl.smem = scan_smem_bytes(kind, 1, 1, pl.qcols);
-  const size_t per_sm = 228 * 1024;
-  int by_smem = (int)(per_sm / (pl.smem + 1024));
-  int by_tmem = 512 / (2 * pl.stage_cols);
-  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
-  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
-  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
-  pl.nsub = 8;
+  finish_plan(pl, true);
+  // the row's exact top-keep is selected in the kernel: one sub-log of keep entries
+  pl.nsub = 1;
   pl.C = 1;
   pl.chunk = 0;
   pl.n_items = batch * n_q;
   pl.keep = keep;
-  pl.capw = 2 * keep + kCompactSlack + 128;
+  pl.capw = keep;
   return pl;
 }
 
@@ -492,6 +508,7 @@ int route_cfg(const dsa_problem* p, int algo, const dsa_route_params* rp, RouteC
     c->nblkH = p->n_k >> c->bsH;
     c->r = rp->hisa_r;
     c->list_len = c->r;
+    if (((long long)c->r << c->bsH) > kMaxGatherKeys) return DSA_ERR_UNSUPPORTED;
   }
   c->hh = c->route ? c->h : p->heads;
   return DSA_OK;
@@ -632,6 +649,8 @@ int run_stage(const dsa_problem* p, const ScanPlan& pl, const StageIO& io, int q
   a.keep = pl.keep;
   a.QG = pl.QG;
   a.qcols = pl.qcols;
+  a.kstages = pl.kstages;
+  a.tstages = pl.tstages;
   a.G = pl.G;
   a.stage_cols = pl.stage_cols;
   a.n_qt = pl.n_qt;
@@ -862,6 +881,8 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.keep = p->topk;
   a.QG = pl.QG;
   a.qcols = pl.qcols;
+  a.kstages = pl.kstages;
+  a.tstages = pl.tstages;
   a.G = pl.G;
   a.stage_cols = pl.stage_cols;
   a.n_qt = pl.n_qt;

@@ -45,24 +45,6 @@ struct FinGroup {
   unsigned long long thr;
 };
 
-// Exact selection of the `need` largest of the n <= 256 keys in b[] by one
-// warp (register bitonic sort), appended to out[base..].
-__device__ __forceinline__ void warp_take_top(const uint64_t* b, int n, int need, uint64_t* out,
-                                              int base, int lane) {
-  uint64_t v[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = lane * 8 + e;
-    v[e] = i < n ? b[i] : 0ull;
-  }
-  bitonic_regs_desc<32, 8>(v, nullptr, lane, 0);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = lane * 8 + e;
-    if (i < need) out[base + i] = v[e];
-  }
-}
-
 // Shared memory of one row group: [sort_cap] result keys, [stage_cap] staged
 // candidates, [kFinBoundary] boundary-bin candidates.  NT threads per row
 // group: 256 when a row has one key chunk (about k candidates), 1024 for

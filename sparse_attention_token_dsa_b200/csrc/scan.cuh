@@ -22,14 +22,15 @@
 // Streaming top-k.  A candidate (score, key) is kept while its composite key
 // (order-preserving score bits, then ~index) is >= the row's threshold thr.
 // thr is always a lower bound of the row's final keep-th best composite, so no
-// winner is ever dropped.  It is raised every step from per-row histograms of
-// the kept candidates: h1 counts them by the top byte of the 32-bit score key;
-// h2[0] / h2[1] count those whose top byte equals b1 / b1 + 1 by the second
-// byte, where b1 is the top-byte bin holding the keep-th best.  The pair gives
-// thr at 16-bit score-key resolution (bf16 precision) without rescanning the
-// logs (a first threshold, or a jump of b1 by more than one, rebuilds h2 from
-// the logs).  Counts can only be low (never high) in the bins the search
-// reaches, which can only make thr looser, never invalid.  Each epilogue warp
+// winner is ever dropped.  It is raised every kUpdateSteps steps from per-row
+// histograms of the kept candidates: h1 counts them by the top byte of the
+// 32-bit score key; h2[0] / h2[1] count those whose top byte equals b1 / b1 + 1
+// by the second byte, where b1 is the top-byte bin holding the keep-th best.
+// The pair gives thr at 16-bit score-key resolution (bf16 precision) without
+// rescanning the logs; a first threshold, or a jump of b1 by more than one,
+// restarts h2 empty (thr then has top-byte resolution until h2 has counted
+// enough new candidates).  Counts can only be low (never high) in the bins the
+// search reaches, which can only make thr looser, never invalid.  Each epilogue warp
 // appends to its own sub-log per row (no atomics) and compacts it in place
 // (keep >= thr) when it nears capacity; if that is not enough (long runs of
 // tied scores) an exact radix-select raise sets thr to the keep-th best
@@ -57,6 +58,8 @@ struct ScanArgs {
   int32_t qcols;         // MMA N per group: max(16, QG * H * parts) query-head columns
   int32_t G;             // groups per work item (1 or 2)
   int32_t stage_cols;    // TMEM columns per accumulator stage (128 or 256)
+  int32_t tstages;       // accumulator stages in TMEM (2 or 4; tstages * stage_cols <= 512)
+  int32_t kstages;       // K-tile pipeline depth (2 .. 8)
   int32_t n_qt;          // query tiles per sequence (ceil(n_q / (QG*G)))
   int32_t C;             // key chunks per row (split-K); 1 = whole prefix
   int32_t chunk;         // keys per chunk (multiple of 128) when C > 1
@@ -84,29 +87,29 @@ constexpr int kMaxRows = 16;          // rows per work item
 constexpr int kMaxItemCols = 512;     // rows x heads per item
 constexpr int kBarEpi = 1;            // named barrier among the epilogue warps
 constexpr int kHistWords = 768;       // h1[256] + h2[2][256] per row
-constexpr int kUpdateSteps = 4;       // steps (key tiles) between threshold updates
+constexpr int kUpdateSteps = 16;      // steps (key tiles) between threshold updates
 // Sub-log slack: a step appends at most 64 entries per row to one sub-log, and a
-// flagged row waits at most two update periods (8 steps) for its exact raise.
-constexpr int kCompactSlack = 640;
-
-#ifndef DSA_BF16_KSTAGES
-#define DSA_BF16_KSTAGES 2   // K-tile pipeline depth for bf16 operands
-#endif
+// flagged row waits at most two update periods for its exact raise.
+constexpr int kCompactSlack = 64 * 2 * kUpdateSteps + 128;
+// Gathered-key rows keep every candidate of their list in shared memory and
+// select once at the end of the row.
+constexpr int kMaxGatherKeys = 8192;
+constexpr int kGatherBins = 4096;     // linear score bins of the end-of-row selection
+constexpr int kGatherBoundary = 256;  // boundary-bin candidates ranked by one warp
+constexpr int kMaxTStages = 4;
 
 template <MmaKind KIND>
 struct ScanCfg {
   static constexpr int ESZ = KIND == MmaKind::TF32 ? 4 : (KIND == MmaKind::BF16 ? 2 : 1);
   static constexpr int A = 128 * ESZ / 128;   // 128-byte atoms per key row (d = 128)
   static constexpr int EPA = 128 / ESZ;       // elements per atom
-  static constexpr int KSTAGES =
-      KIND == MmaKind::E4M3 ? 4 : (KIND == MmaKind::BF16 ? DSA_BF16_KSTAGES : 2);
   static constexpr int KTILE_BYTES = A * 128 * 128;
 };
 
 struct ScanSmemTail {
   uint64_t k_full[8], k_empty[8];
   uint64_t q_full, q_empty;
-  uint64_t t_full[2], t_empty[2];
+  uint64_t t_full[kMaxTStages], t_empty[kMaxTStages];
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -116,8 +119,12 @@ struct ScanSmemTail {
   int32_t row_b1[kMaxRows];    // top-byte bin of the keep-th best (-1: fewer kept)
   int32_t row_raise[kMaxRows]; // a sub-log could not be compacted enough
   int32_t raise_any;           // some row needs an exact raise
+  int32_t gather_legal;        // gathered row: legal candidates seen
+  int32_t gather_nwin, gather_nbnd;
+  float gather_lo[kEpiWarps], gather_hi[kEpiWarps];
   int32_t subcnt[kMaxRows][8]; // sub-log fill, written only by the owning warp
   unsigned long long row_thr[kMaxRows];
+  int32_t item_min_nleg;       // smallest row_nleg of the item's rows
   alignas(16) float wsm[kMaxItemCols];
   SelectScratch sel;
 };
@@ -201,25 +208,6 @@ __device__ __forceinline__ int compact_sublog(uint64_t* lg, int n, unsigned long
   return wpos;
 }
 
-// Fine-histogram rebuild from one sub-log (entries whose top byte is b1 or b1+1).
-__device__ __forceinline__ void rebuild_fine(uint32_t* h, const uint64_t* lg, int n, int b1,
-                                             int lane) {
-  for (int i0 = 0; i0 < n; i0 += 256) {
-    uint32_t sk[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = i0 + j * 32 + lane;
-      sk[j] = i < n ? (uint32_t)(lg[i] >> 32) : 0u;
-    }
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int i = i0 + j * 32 + lane;
-      const int d1 = (int)(sk[j] >> 24) - b1;
-      if (i < n && (d1 == 0 || d1 == 1)) atomicAdd(&h[256 + d1 * 256 + ((sk[j] >> 16) & 255)], 1u);
-    }
-  }
-}
-
 // Per-unit context of the filter: the lane's key, its dequant scale, and where
 // this warp's sub-logs and the row histograms live.
 struct FilterCtx {
@@ -229,26 +217,30 @@ struct FilterCtx {
   int lane;
   unsigned lanemask_lt;
   int sub;
+  bool all_legal;        // every key of this unit is legal for every row of the item
   uint64_t* logs;        // this warp's sub-log of item row 0
-  int64_t row_stride;    // entries between consecutive rows' sub-logs
+  uint32_t row_stride;   // entries between consecutive rows' sub-logs
   uint32_t* hist;
   ScanSmemTail* T;
 };
 
 // Legality, composite key, threshold filter and append for one query row.
-// The common path (no lane survives) costs one limit load, one threshold load,
+// The common path (no lane survives) costs the key arithmetic, one threshold
+// load and a vote (the legality test is skipped for units inside every row's
+// legal range).
 // the key arithmetic and a vote.
 __device__ __forceinline__ void filter_append(const FilterCtx& f, int r, float acc) {
   ScanSmemTail* T = f.T;
+  const bool legal = f.all_legal || (unsigned)(f.key - f.kbeg) < (unsigned)T->row_nleg[r];
   const uint32_t sk = score_key(acc * f.ks);
   const uint64_t comp = ((uint64_t)sk << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)f.key);
-  const bool surv = (unsigned)(f.key - f.kbeg) < (unsigned)T->row_nleg[r] && comp >= T->row_thr[r];
+  const bool surv = legal && comp >= T->row_thr[r];
   const unsigned bal = __ballot_sync(0xffffffffu, surv);
   if (bal) {
     int* cnt = &T->subcnt[r][f.sub];
     const int base = *cnt;
     if (surv) {
-      f.logs[r * f.row_stride + base + __popc(bal & f.lanemask_lt)] = comp;
+      f.logs[(uint32_t)r * f.row_stride + (uint32_t)(base + __popc(bal & f.lanemask_lt))] = comp;
       uint32_t* h = f.hist + r * kHistWords;
       const int b1 = (int)(sk >> 24);
       atomicAdd(&h[b1], 1u);
@@ -379,6 +371,44 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
   }
 }
 
+// sum_j w_j ReLU(D_j) over the HT accumulator columns of one query row (TMEM
+// columns [0, HT) at taddr), for the gathered-key epilogue.
+template <int HT>
+__device__ __forceinline__ float row_acc(uint32_t taddr, const float* w) {
+  if constexpr (HT >= 32) {
+    constexpr int NC = HT / 32;
+    unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+    uint32_t va[1][32], vb[1][32];
+    tmem_ld_chunks<1>(taddr, va);
+    tmem_wait_chunks<1>(va);
+#pragma unroll
+    for (int c = 0; c < NC; c += 2) {
+      if (c + 1 < NC) tmem_ld_chunks<1>(taddr + (c + 1) * 32, vb);
+      relu_dot<1>(va, w + c * 32, acc);
+      if (c + 1 >= NC) break;
+      tmem_wait_chunks<1>(vb);
+      if (c + 2 < NC) tmem_ld_chunks<1>(taddr + (c + 2) * 32, va);
+      relu_dot<1>(vb, w + (c + 1) * 32, acc);
+      if (c + 2 < NC) tmem_wait_chunks<1>(va);
+    }
+    return sum8(acc);
+  } else {
+    uint32_t v[1][32];
+    tmem_ld_chunks<1>(taddr, v);
+    tmem_wait_chunks<1>(v);
+    float b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int jj = 0; jj < HT; jj += 4) {
+      const float4 wv = *reinterpret_cast<const float4*>(w + jj);
+      b[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[0][jj + 0]), 0.f), b[0]);
+      b[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[0][jj + 1]), 0.f), b[1]);
+      b[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[0][jj + 2]), 0.f), b[2]);
+      b[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[0][jj + 3]), 0.f), b[3]);
+    }
+    return (b[0] + b[1]) + (b[2] + b[3]);
+  }
+}
+
 // 320 threads: ten warps over four sub-partitions of 16K registers each allow
 // at most 168 registers per thread.
 template <MmaKind KIND, bool SPLIT, int HT, int GATHER>
@@ -395,22 +425,30 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   const int QT = a.QG * a.G;
   uint8_t* Qs = smem;                                       // [G][A][qcols x 128B]
   const int q_bytes = a.G * Cfg::A * qcols * 128;
-  uint8_t* Ks = smem + ((q_bytes + 1023) & ~1023);          // [KSTAGES][A][128 x 128B]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + Cfg::KSTAGES * Cfg::KTILE_BYTES);  // [QT][768]
-  ScanSmemTail* T = reinterpret_cast<ScanSmemTail*>(hist + QT * kHistWords);
+  const int KS = a.kstages, NS = a.tstages;
+  uint8_t* Ks = smem + ((q_bytes + 1023) & ~1023);          // [KS][A][128 x 128B]
+  // streaming rows: per-row histograms [QT][768]; gathered rows: the row's
+  // candidate composites [kMaxGatherKeys]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + KS * Cfg::KTILE_BYTES);
+  uint64_t* cand = reinterpret_cast<uint64_t*>(hist);                 // [kMaxGatherKeys]
+  uint32_t* ghist = reinterpret_cast<uint32_t*>(cand + kMaxGatherKeys);  // [kGatherBins]
+  uint64_t* gbnd = reinterpret_cast<uint64_t*>(ghist + kGatherBins);   // [kGatherBoundary]
+  ScanSmemTail* T = reinterpret_cast<ScanSmemTail*>(
+      GATHER != 0 ? reinterpret_cast<uint8_t*>(gbnd + kGatherBoundary)
+                  : reinterpret_cast<uint8_t*>(hist + QT * kHistWords));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool modeB = (a.QG == 1);  // one query per group: halves take alternate stages
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < Cfg::KSTAGES; ++i) {
+    for (int i = 0; i < KS; ++i) {
       mbar_init(&T->k_full[i], 1);
       mbar_init(&T->k_empty[i], 1);
     }
     mbar_init(&T->q_full, 1);
     mbar_init(&T->q_empty, 1);
     mbar_init(&T->drain, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NS; ++s) {
       mbar_init(&T->t_full[s], 1);
       mbar_init(&T->t_empty[s], modeB ? 4 : 8);
     }
@@ -418,7 +456,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
-    tmem_alloc(&T->tmem_base, 2 * a.stage_cols);
+    tmem_alloc(&T->tmem_base, NS * a.stage_cols);
     tmem_relinquish();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -434,74 +472,90 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer --
-    if (lane == 0) {
-      uint32_t kcount = 0, it = 0;
-      bool ok = true;
-      for (int round = 0; ok; ++round) {
-        const int item = sched_item(round, blockIdx.x, grid);
-        if (item >= a.n_items) break;
-        ItemGeom g = item_geom<GATHER>(a, item);
-        if (g.ntiles == 0) continue;
-        if (!mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1)) break;
-        mbar_arrive_expect_tx(&T->q_full, q_bytes);
-        const int qrow0 = (g.b * a.q_stride + a.q_off + g.row0) * a.H * PARTS;
-        for (int gg = 0; gg < a.G; ++gg)
-          for (int at = 0; at < Cfg::A; ++at)
-            tma_load_2d(Qs + (gg * Cfg::A + at) * qcols * 128, &qmap, &T->q_full,
-                        at * Cfg::EPA, qrow0 + gg * a.QG * a.H * PARTS);
-        ++it;
-        const int krow0 = g.b * a.n_k;
-        for (int t = 0; t < g.ntiles && ok; ++t) {
-          const int slot = kcount % Cfg::KSTAGES;
-          const uint32_t ph = (kcount / Cfg::KSTAGES) & 1;
-          if (!mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2)) { ok = false; break; }
-          mbar_arrive_expect_tx(&T->k_full[slot], Cfg::KTILE_BYTES);
-          if constexpr (GATHER == 0) {
+    // Lane 0 owns the barriers; for gathered keys the whole warp reads the
+    // row's list (four entries or one block per lane) and issues the copies.
+    uint32_t kcount = 0, it = 0;
+    bool ok = true;
+    for (int round = 0; ok; ++round) {
+      const int item = sched_item(round, blockIdx.x, grid);
+      if (item >= a.n_items) break;
+      ItemGeom g = item_geom<GATHER>(a, item);
+      if (g.ntiles == 0) continue;
+      if (lane == 0) {
+        ok = mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1);
+        if (ok) {
+          mbar_arrive_expect_tx(&T->q_full, q_bytes);
+          const int qrow0 = (g.b * a.q_stride + a.q_off + g.row0) * a.H * PARTS;
+          for (int gg = 0; gg < a.G; ++gg)
+            for (int at = 0; at < Cfg::A; ++at)
+              tma_load_2d(Qs + (gg * Cfg::A + at) * qcols * 128, &qmap, &T->q_full,
+                          at * Cfg::EPA, qrow0 + gg * a.QG * a.H * PARTS);
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      ++it;
+      const int krow0 = g.b * a.n_k;
+      const int32_t* lst = GATHER != 0
+          ? a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len : nullptr;
+      for (int t = 0; t < g.ntiles; ++t) {
+        const int slot = kcount % KS;
+        const uint32_t ph = (kcount / KS) & 1;
+        // list entries of this tile (loaded before the wait so their latency overlaps it)
+        int rr[4] = {0, 0, 0, 0};
+        int ybox = -1;
+        if constexpr (GATHER == 1) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int e = t * 128 + lane * 4 + j;
+            const int kk = e < a.klist_len ? lst[e] : -1;
+            rr[j] = krow0 + (kk >= 0 ? kk : 0);
+          }
+        } else if constexpr (GATHER == 2) {
+          const int bs = 1 << a.lb_shift;
+          const int box = bs < 128 ? bs : 128;
+          if (lane < 128 / box) {
+            const int e = t * 128 + lane * box;            // token slot in the row's list
+            const int slot_b = e >> a.lb_shift;
+            const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
+            ybox = krow0 + (blk >= 0 ? blk * bs + (e & (bs - 1)) : 0);
+          }
+        }
+        if (lane == 0) {
+          ok = mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2);
+          if (ok) mbar_arrive_expect_tx(&T->k_full[slot], Cfg::KTILE_BYTES);
+        }
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if constexpr (GATHER == 0) {
+          if (lane == 0) {
             const int tstart = (g.t_hi - t) << 7;
             for (int at = 0; at < Cfg::A; ++at)
               tma_load_2d(Ks + (slot * Cfg::A + at) * 16384, &kmap, &T->k_full[slot],
                           at * Cfg::EPA, krow0 + tstart);
-          } else {
-            const int32_t* lst = a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len;
-            if constexpr (GATHER == 1) {
-              // token list: four arbitrary key rows per gather (one-row-high boxes)
-              for (int r4 = 0; r4 < 128; r4 += 4) {
-                int rr[4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                  const int e = t * 128 + r4 + j;
-                  const int kk = e < a.klist_len ? lst[e] : -1;
-                  rr[j] = krow0 + (kk >= 0 ? kk : 0);
-                }
-                for (int at = 0; at < Cfg::A; ++at)
-                  tma_gather4(Ks + (slot * Cfg::A + at) * 16384 + r4 * 128, &kmap, &T->k_full[slot],
-                              at * Cfg::EPA, rr[0], rr[1], rr[2], rr[3]);
-              }
-            } else {
-              // block list: runs of 2^lb_shift contiguous keys (box of min(bs, 128) rows)
-              const int bs = 1 << a.lb_shift;
-              const int box = bs < 128 ? bs : 128;
-              for (int r0 = 0; r0 < 128; r0 += box) {
-                const int e = t * 128 + r0;                 // token slot in the row's list
-                const int slot_b = e >> a.lb_shift;
-                const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
-                const int off = e & (bs - 1);
-                const int y = krow0 + (blk >= 0 ? blk * bs + off : 0);
-                for (int at = 0; at < Cfg::A; ++at)
-                  tma_load_2d(Ks + (slot * Cfg::A + at) * 16384 + r0 * 128, &kmap, &T->k_full[slot],
-                              at * Cfg::EPA, y);
-              }
-            }
           }
-          ++kcount;
+        } else if constexpr (GATHER == 1) {
+          // four arbitrary key rows per copy (one-row-high boxes), 32 copies per atom
+          for (int at = 0; at < Cfg::A; ++at)
+            tma_gather4(Ks + (slot * Cfg::A + at) * 16384 + lane * 4 * 128, &kmap,
+                        &T->k_full[slot], at * Cfg::EPA, rr[0], rr[1], rr[2], rr[3]);
+        } else {
+          // runs of 2^lb_shift consecutive keys (box of min(bs, 128) rows)
+          const int bs = 1 << a.lb_shift;
+          const int box = bs < 128 ? bs : 128;
+          if (lane < 128 / box)
+            for (int at = 0; at < Cfg::A; ++at)
+              tma_load_2d(Ks + (slot * Cfg::A + at) * 16384 + lane * box * 128, &kmap,
+                          &T->k_full[slot], at * Cfg::EPA, ybox);
         }
+        ++kcount;
       }
-      if (*abort) {
-        // abort path: let this CTA's own copies in flight land before exit
-        if (it > 0) mbar_wait_drain(&T->q_full, (it - 1) & 1);
-        for (uint32_t i = kcount > Cfg::KSTAGES ? kcount - Cfg::KSTAGES : 0; i < kcount; ++i)
-          mbar_wait_drain(&T->k_full[i % Cfg::KSTAGES], (i / Cfg::KSTAGES) & 1);
-      }
+    }
+    if (lane == 0 && *abort) {
+      // abort path: let this CTA's own copies in flight land before exit
+      if (it > 0) mbar_wait_drain(&T->q_full, (it - 1) & 1);
+      for (uint32_t i = kcount > (uint32_t)KS ? kcount - KS : 0; i < kcount; ++i)
+        mbar_wait_drain(&T->k_full[i % KS], (i / KS) & 1);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA --
@@ -520,12 +574,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         const int nunits = g.ntiles * a.G;
         for (int u = 0; u < nunits; ++u) {
           const int gg = u & (a.G - 1);
-          const int slot = kcount % Cfg::KSTAGES;
+          const int slot = kcount % KS;
           if (gg == 0) {
-            if (!mbar_wait(&T->k_full[slot], (kcount / Cfg::KSTAGES) & 1, abort, a.status, 4)) { ok = false; break; }
+            if (!mbar_wait(&T->k_full[slot], (kcount / KS) & 1, abort, a.status, 4)) { ok = false; break; }
           }
-          const int s = ucount & 1;
-          if (!mbar_wait(&T->t_empty[s], ((ucount >> 1) & 1) ^ 1, abort, a.status, 5)) { ok = false; break; }
+          const int s = ucount % NS;
+          if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d = tmem_base + s * a.stage_cols;
           const uint32_t kbase = smem_u32(Ks + slot * Cfg::A * 16384);
@@ -555,6 +609,185 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         mbar_wait_drain(&T->drain, 0);
       }
     }
+  } else if constexpr (GATHER != 0) {
+    // ------------------------------------------ epilogue, gathered keys --
+    // One query row per item; the halves take alternate accumulator stages.
+    // Every candidate's composite goes to shared memory (list position e);
+    // at the end of the row one exact selection keeps its top `keep`, written
+    // to the row's first sub-log.
+    const int etid = threadIdx.x;
+    const int quad = warp & 3;
+    const int half = warp >> 2;
+    uint32_t ucount = 0;
+    int step_par = 0;
+    for (int round = 0;; ++round) {
+      const int item = sched_item(round, blockIdx.x, grid);
+      if (item >= a.n_items) break;
+      ItemGeom g = item_geom<GATHER>(a, item);
+      const int pos0 = (a.q_pos0 ? a.q_pos0[g.b] : a.n_tok - a.q_stride) + a.q_off;
+      const int klen = a.k_len ? a.k_len[g.b] : a.n_tok;
+      const int64_t slot0 = (int64_t)g.b * a.n_q + g.row0;     // one key chunk
+      const int nkeys = g.kend;                                 // list length in tokens
+      const int nleg = g.nrows > 0 ? max(0, min(pos0 + g.row0, klen - 1) + 1) : 0;
+      const int32_t* lst = a.klist + slot0 * a.klist_len;
+      const int64_t grow = (int64_t)g.b * a.q_stride + a.q_off + g.row0;
+      for (int i = etid; i < HT; i += kEpiThreads) T->wsm[i] = g.nrows > 0 ? a.w[grow * HT + i] : 0.f;
+      for (int i = etid; i < kGatherBins; i += kEpiThreads) ghist[i] = 0u;
+      if (etid == 0) {
+        T->gather_legal = 0;
+        T->gather_nwin = 0;
+        T->gather_nbnd = 0;
+      }
+      named_bar_sync(kBarEpi, kEpiThreads);
+      int legal_cnt = 0;
+      float lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
+      for (int u = 0; u < g.ntiles; ++u) {
+        const uint32_t uc = ucount + u;
+        if ((int)(uc & 1) != half) continue;
+        const int s = uc % NS;
+        // this lane's key (list lookup issued before the wait)
+        const int e = u * 128 + quad * 32 + lane;
+        int key;
+        if constexpr (GATHER == 1) {
+          key = e < a.klist_len ? lst[e] : -1;
+        } else {
+          const int sb = e >> a.lb_shift;
+          const int blk = sb < a.klist_len ? lst[sb] : -1;
+          key = blk >= 0 ? (blk << a.lb_shift) + (e & ((1 << a.lb_shift) - 1)) : -1;
+        }
+        const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
+        __syncwarp();
+        if (!__all_sync(0xffffffffu, got)) continue;
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + s * a.stage_cols;
+        const float acc = row_acc<HT>(taddr, T->wsm);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&T->t_empty[s]);
+        const bool legal = (unsigned)key < (unsigned)nleg;
+        legal_cnt += legal ? 1 : 0;
+        if (legal) {
+          lo = fminf(lo, acc);
+          hi = fmaxf(hi, acc);
+        }
+        if (e < nkeys) cand[e] = legal ? make_comp(acc, key) : 0ull;
+      }
+      ucount += g.ntiles;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        legal_cnt += __shfl_xor_sync(0xffffffffu, legal_cnt, off);
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+      }
+      if (lane == 0) {
+        if (legal_cnt) atomicAdd(&T->gather_legal, legal_cnt);
+        T->gather_lo[warp] = lo;
+        T->gather_hi[warp] = hi;
+      }
+      if (etid == 0) T->epi_stop[step_par] = *abort;   // uniform stop decision
+      named_bar_sync(kBarEpi, kEpiThreads);
+      const bool stop = T->epi_stop[step_par] != 0;
+      step_par ^= 1;
+      if (stop) break;
+      const int n_legal = T->gather_legal;
+      const int ncand = nkeys < kMaxGatherKeys ? nkeys : kMaxGatherKeys;
+      uint64_t* out = a.logs + slot0 * a.nsub * a.capw;
+      int cnt = 0;
+      bool radix = false;
+      if (n_legal > a.keep) {
+        // linear score bins over [lo, hi]: count, locate the bin of the keep-th best,
+        // emit every candidate above it and rank that bin's few candidates exactly
+        float lo2 = T->gather_lo[0], hi2 = T->gather_hi[0];
+#pragma unroll
+        for (int w = 1; w < kEpiWarps; ++w) {
+          lo2 = fminf(lo2, T->gather_lo[w]);
+          hi2 = fmaxf(hi2, T->gather_hi[w]);
+        }
+        const float span = hi2 - lo2;
+        const float scale = span > 0.f ? (float)(kGatherBins - 1) / span : 0.f;
+        auto bin_of = [&](uint64_t c) {
+          const int b = __float2int_rz((key_score((uint32_t)(c >> 32)) - lo2) * scale);
+          return min(kGatherBins - 1, max(0, b));
+        };
+        for (int e = etid; e < ncand; e += kEpiThreads) {
+          const uint64_t c = cand[e];
+          if (c != 0ull) atomicAdd(&ghist[bin_of(c)], 1u);
+        }
+        named_bar_sync(kBarEpi, kEpiThreads);
+        // thread t owns the 16 bins from 4095 - 16 t downwards; scan in that order
+        uint32_t own = 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) own += ghist[kGatherBins - 1 - 16 * etid - i];
+        uint32_t incl = own;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += o;
+        }
+        uint32_t* wsum = reinterpret_cast<uint32_t*>(T->sel.hist);
+        if (lane == 31) wsum[warp] = incl;
+        named_bar_sync(kBarEpi, kEpiThreads);
+        uint32_t wbase = 0;
+        for (int w = 0; w < warp; ++w) wbase += wsum[w];
+        const uint32_t excl = wbase + incl - own;
+        const uint32_t need = (uint32_t)a.keep;
+        if (excl < need && need <= excl + own) {
+          uint32_t cum = excl;
+          for (int i = 0; i < 16; ++i) {
+            const int b = kGatherBins - 1 - 16 * etid - i;
+            const uint32_t c = ghist[b];
+            if (cum + c >= need) {
+              T->sel.sel[2] = b;
+              T->sel.sel[3] = (int)cum;            // candidates strictly above bin b
+              break;
+            }
+            cum += c;
+          }
+        }
+        named_bar_sync(kBarEpi, kEpiThreads);
+        const int bstar = T->sel.sel[2], above = T->sel.sel[3];
+        for (int e0 = 0; e0 < ncand; e0 += kEpiThreads) {
+          const int e = e0 + etid;
+          const uint64_t c = e < ncand ? cand[e] : 0ull;
+          const int b = c != 0ull ? bin_of(c) : -1;
+          const bool win = b > bstar, edge = b == bstar;
+          const unsigned bw = __ballot_sync(0xffffffffu, win);
+          const unsigned be = __ballot_sync(0xffffffffu, edge);
+          int pw = 0, pe = 0;
+          if (lane == 0) {
+            if (bw) pw = atomicAdd(&T->gather_nwin, __popc(bw));
+            if (be) pe = atomicAdd(&T->gather_nbnd, __popc(be));
+          }
+          pw = __shfl_sync(0xffffffffu, pw, 0);
+          pe = __shfl_sync(0xffffffffu, pe, 0);
+          const unsigned lt = (1u << lane) - 1u;
+          if (win) out[pw + __popc(bw & lt)] = c;
+          if (edge) {
+            const int sl = pe + __popc(be & lt);
+            if (sl < kGatherBoundary) gbnd[sl] = c;
+          }
+        }
+        named_bar_sync(kBarEpi, kEpiThreads);
+        const int nb = T->gather_nbnd;
+        if (nb <= kGatherBoundary) {
+          if (warp == 0) warp_take_top(gbnd, nb, a.keep - above, out, above, lane);
+          cnt = a.keep;
+        } else {
+          radix = true;                                  // a crowded bin (ties): exact radix
+        }
+      }
+      if (n_legal > 0 && (n_legal <= a.keep || radix)) {
+        const uint64_t* segs[1] = {cand};
+        const int segn[1] = {ncand};
+        uint64_t thr = 1ull;                          // every legal composite is >= 1
+        if (n_legal > a.keep)
+          thr = radix_select<kEpiThreads>(segs, segn, 1, a.keep, &T->sel, etid, kBarEpi);
+        cnt = compact_ge<kEpiThreads>(segs, segn, 1, thr, out, &T->sel, etid, kBarEpi, nullptr);
+      }
+      if (etid < a.nsub) a.log_cnt[slot0 * a.nsub + etid] = etid == 0 ? cnt : 0;
+      if (etid == 0) a.log_thr[slot0] = 0ull;
+      named_bar_sync(kBarEpi, kEpiThreads);             // cand is reused by the next row
+    }
   } else {
     // ------------------------------------------------------------ epilogue --
     const int etid = threadIdx.x;              // 0..255
@@ -582,14 +815,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         int nleg = 0;
         if (r < g.nrows) {
           const int pos = pos0 + g.row0 + r;
-          if (GATHER != 0)
-            nleg = max(0, min(pos, klen - 1) + 1);                     // key <= pos, key < k_len
-          else if (a.bs_shift > 0)
+          if (a.bs_shift > 0)
             nleg = max(0, min(min(pos + 1, klen) >> a.bs_shift, g.kend) - g.kbeg);
           else
             nleg = max(0, min(min(pos, klen - 1), g.kend - 1) - g.kbeg + 1);
         }
         T->row_nleg[r] = nleg;
+        // positions grow with the row, so row 0 has the item's smallest legal
+        // count; an item with unused row slots (nleg 0) has none that is always legal
+        if (r == 0) T->item_min_nleg = g.nrows < QT ? 0 : nleg;
 #pragma unroll
         for (int w8 = 0; w8 < 8; ++w8) T->subcnt[r][w8] = 0;
       }
@@ -616,31 +850,19 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         for (int v = 0; v < nstep; ++v) {
           const int uu = u + v;
           const uint32_t uc = ucount + v;
-          const int s = uc & 1;
-          const bool mine = modeB ? (half == s) : true;
+          const int s = uc % NS;
+          const bool mine = modeB ? (half == (int)(uc & 1)) : true;
           if (!mine) continue;
-          const bool got = mbar_wait(&T->t_full[s], (uc >> 1) & 1, abort, a.status, 6);
+          const int gg = uu & (a.G - 1);
+          const int t = uu >> (a.G - 1);
+          const int key = ((g.t_hi - t) << 7) + quad * 32 + lane;
+          // key dequant scale, loaded before the wait so its latency overlaps it
+          float ks = 1.f;
+          if (a.k_scale && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
+          const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
           tc_fence_after();
-          const int gg = uu & (a.G - 1);
-          const int t = uu >> (a.G - 1);
-          int key;
-          if constexpr (GATHER == 0) {
-            key = ((g.t_hi - t) << 7) + quad * 32 + lane;
-          } else {
-            const int32_t* lst = a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len;
-            const int e = t * 128 + quad * 32 + lane;
-            if constexpr (GATHER == 1) {
-              key = e < a.klist_len ? lst[e] : -1;
-            } else {
-              const int slot_b = e >> a.lb_shift;
-              const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
-              key = blk >= 0 ? (blk << a.lb_shift) + (e & ((1 << a.lb_shift) - 1)) : -1;
-            }
-          }
-          float ks = 1.f;
-          if (a.k_scale && key >= 0 && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
           const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + s * a.stage_cols;
           // queries handled by this warp inside group gg
           const int qbeg = modeB ? 0 : half * qhalf;
@@ -653,7 +875,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           fc.lanemask_lt = (1u << lane) - 1u;
           fc.sub = sub;
           fc.logs = a.logs + (slot0 * a.nsub + sub) * a.capw;
-          fc.row_stride = (int64_t)a.C * a.nsub * a.capw;
+          fc.row_stride = (uint32_t)(a.C * a.nsub * a.capw);
+          fc.all_legal = key - (int)(quad * 32 + lane) >= g.kbeg &&
+                         key - (int)(quad * 32 + lane) + 127 - g.kbeg < T->item_min_nleg;
           fc.hist = hist;
           fc.T = T;
           if constexpr (SPLIT) {
@@ -737,12 +961,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                 h[512 + i] = 0u;
               }
             } else {
-              // first threshold or a jump: rebuild both fine histograms from the sub-logs
+              // first threshold or a jump: the fine histograms restart empty and count
+              // the candidates kept from now on (low counts: a looser, valid threshold)
               for (int i = lane; i < 512; i += 32) h[256 + i] = 0u;
-              __syncwarp();
-              const int64_t rs = slot0 + (int64_t)r * a.C;
-              for (int sb = 0; sb < a.nsub; ++sb)
-                rebuild_fine(h, a.logs + (rs * a.nsub + sb) * a.capw, T->subcnt[r][sb], nb1, lane);
             }
             __syncwarp();
             if (lane == 0) T->row_b1[r] = nb1;
@@ -750,9 +971,12 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           __syncwarp();
           int above2;
           const int b2 = hist_find(h + 256, above1, a.keep, lane, &above2);
-          if (b2 >= 0 && lane == 0) {
-            const unsigned long long thr =
-                (unsigned long long)(((uint32_t)nb1 << 24) | ((uint32_t)b2 << 16)) << 32;
+          if (lane == 0) {
+            // the keep-th best lies in top-byte bin nb1, and in its fine bin b2 when the
+            // fine counts reach it
+            const uint32_t hi = b2 >= 0 ? (((uint32_t)nb1 << 24) | ((uint32_t)b2 << 16))
+                                        : ((uint32_t)nb1 << 24);
+            const unsigned long long thr = (unsigned long long)hi << 32;
             if (thr > T->row_thr[r]) T->row_thr[r] = thr;
           }
           __syncwarp();
@@ -827,7 +1051,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * a.stage_cols);
+    tmem_dealloc(tmem_base, NS * a.stage_cols);
   }
 }
 

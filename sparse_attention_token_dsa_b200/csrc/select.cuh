@@ -258,8 +258,10 @@ __device__ __forceinline__ void bitonic_regs_desc(uint64_t (&v)[E], uint64_t* xs
 }
 
 // Sort a[0, n) descending in place (n <= N = NT * E; slots up to N hold 0).
+// Thread t reads slots written by other threads: the group synchronises first.
 template <int NT, int E>
 __device__ void sort_desc_regs(uint64_t* a, int n, int tid, int bar_id) {
+  named_bar_sync(bar_id, NT);
   uint64_t v[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
@@ -271,6 +273,24 @@ __device__ void sort_desc_regs(uint64_t* a, int n, int tid, int bar_id) {
 #pragma unroll
   for (int e = 0; e < E; ++e) a[tid * E + e] = v[e];
   named_bar_sync(bar_id, NT);
+}
+
+// Exact selection of the `need` largest of the n <= 256 keys in b[] by one
+// warp (register bitonic sort), appended to out[base..].
+__device__ __forceinline__ void warp_take_top(const uint64_t* b, int n, int need, uint64_t* out,
+                                              int base, int lane) {
+  uint64_t v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = lane * 8 + e;
+    v[e] = i < n ? b[i] : 0ull;
+  }
+  bitonic_regs_desc<32, 8>(v, nullptr, lane, 0);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int i = lane * 8 + e;
+    if (i < need) out[base + i] = v[e];
+  }
 }
 
 }  // namespace dsa

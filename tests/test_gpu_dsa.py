@@ -99,6 +99,16 @@ def test_integer_many_ties_long_rows_bit_exact(B, flags):
     parity.exact(gi, gs, ri, rs)
 
 
+@pytest.mark.parametrize("topk", [2048, 4096, 8192])
+def test_integer_sorted_large_topk_bit_exact(B, topk):
+    """Ordered output with several keys per select thread: rows just below and
+    just above topk legal keys (every candidate a winner / a real selection)."""
+    p = gen.integer_problem(7, 1, 64, 12000, 64, 128, topk, q_pos0=[topk - 32], dtype=gen.BF16)
+    gi, gs = run_dsa(B, p, flags=B.DSA_FLAG_SORTED)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
 def test_single_key_and_single_query(B):
     p = gen.integer_problem(6, 2, 1, 1, 64, 128, 4, dtype=gen.F32)
     gi, gs = run_dsa(B, p)
