@@ -303,26 +303,23 @@ cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint
   f.log_thr = thr;
   f.out_idx = out_idx;
   f.out_score = out_score;
-  if (pl.C == 1) {
+  if (pl.C == 1 && sc <= 2048) {
     // one key chunk per row: about k candidates; up to four rows per CTA
     const int stage_cap = sc + sc / 2;
     const size_t per_group = ((size_t)sc + stage_cap + kFinBoundary) * sizeof(uint64_t);
     const int e_per = sc / 256;
     int groups = (int)((160 * 1024) / per_group);
     if (groups > kFinMaxGroups) groups = kFinMaxGroups;
-    if (e_per > 8) groups = 1;
     if (groups < 1) groups = 1;
     const size_t smem = per_group * groups;
     switch (e_per) {
       case 1: return launch_fin<256, 1>(f, groups, stage_cap, smem, st);
       case 2: return launch_fin<256, 2>(f, groups, stage_cap, smem, st);
       case 4: return launch_fin<256, 4>(f, groups, stage_cap, smem, st);
-      case 8: return launch_fin<256, 8>(f, groups, stage_cap, smem, st);
-      case 16: return launch_fin<256, 16>(f, groups, stage_cap, smem, st);
-      default: return launch_fin<256, 32>(f, groups, stage_cap, smem, st);
+      default: return launch_fin<256, 8>(f, groups, stage_cap, smem, st);
     }
   }
-  // split-K rows: about C * k candidates; one row per 1024-thread CTA
+  // split-K rows (about C * k candidates) and large k: one row per 1024-thread CTA
   const size_t budget = 200 * 1024;
   int stage_cap = (int)(budget / sizeof(uint64_t)) - sc - kFinBoundary;
   if (stage_cap < sc) stage_cap = sc;

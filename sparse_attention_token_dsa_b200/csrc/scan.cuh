@@ -641,20 +641,27 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       named_bar_sync(kBarEpi, kEpiThreads);
       int legal_cnt = 0;
       float lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
-      for (int u = 0; u < g.ntiles; ++u) {
-        const uint32_t uc = ucount + u;
-        if ((int)(uc & 1) != half) continue;
-        const int s = uc % NS;
-        // this lane's key (list lookup issued before the wait)
+      // this lane's key at list position e of unit u (a global load)
+      auto key_at = [&](int u) -> int {
         const int e = u * 128 + quad * 32 + lane;
-        int key;
         if constexpr (GATHER == 1) {
-          key = e < a.klist_len ? lst[e] : -1;
+          return e < a.klist_len ? lst[e] : -1;
         } else {
           const int sb = e >> a.lb_shift;
           const int blk = sb < a.klist_len ? lst[sb] : -1;
-          key = blk >= 0 ? (blk << a.lb_shift) + (e & ((1 << a.lb_shift) - 1)) : -1;
+          return blk >= 0 ? (blk << a.lb_shift) + (e & ((1 << a.lb_shift) - 1)) : -1;
         }
+      };
+      // this half takes every other unit; the key of its next unit is loaded one
+      // unit ahead so the list lookup never waits on memory
+      const int u0 = (int)((ucount + half) & 1);
+      int key_next = u0 < g.ntiles ? key_at(u0) : -1;
+      for (int u = u0; u < g.ntiles; u += 2) {
+        const uint32_t uc = ucount + u;
+        const int s = uc % NS;
+        const int e = u * 128 + quad * 32 + lane;
+        const int key = key_next;
+        if (u + 2 < g.ntiles) key_next = key_at(u + 2);
         const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) continue;
@@ -842,6 +849,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       if (etid == 0) T->raise_any = 0;
       named_bar_sync(kBarEpi, kEpiThreads);
       const int nunits = g.ntiles * a.G;
+      auto ks_at = [&](int uu) -> float {
+        if (!a.k_scale) return 1.f;
+        const int key = ((g.t_hi - (uu >> (a.G - 1))) << 7) + quad * 32 + lane;
+        return key < a.n_k ? a.k_scale[(int64_t)g.b * a.n_k + key] : 1.f;
+      };
+      const int ustep = modeB ? 2 : 1;                  // this warp's units: every / every other
+      const int ufirst = modeB ? (int)((ucount + half) & 1) : 0;
+      float ks_next = ufirst < nunits ? ks_at(ufirst) : 1.f;
       int u = 0;
       int steps = 0;
       while (u < nunits) {
@@ -856,9 +871,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const int gg = uu & (a.G - 1);
           const int t = uu >> (a.G - 1);
           const int key = ((g.t_hi - t) << 7) + quad * 32 + lane;
-          // key dequant scale, loaded before the wait so its latency overlaps it
-          float ks = 1.f;
-          if (a.k_scale && key < a.n_k) ks = a.k_scale[(int64_t)g.b * a.n_k + key];
+          // key dequant scale: loaded one unit of this warp ahead
+          const float ks = ks_next;
+          if (uu + ustep < nunits) ks_next = ks_at(uu + ustep);
           const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
