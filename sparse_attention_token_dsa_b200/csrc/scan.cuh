@@ -318,7 +318,7 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
     for (int sg = 0; sg < nseg; sg += 2) {
       const bool has_b = sg + 1 < nseg;
       if (has_b) tmem_ld_chunks<SEGC>(col + (sg + 1) * 32 * SEGC, vb);
-      relu_dot<SEGC>(va, w + sg * 32 * SEGC, acc);
+      relu_dot<1>(va, w + sg * 32 * SEGC, acc);
       if ((sg + 1) % SPQ == 0) {
         filter_append(f, rbase + sg / SPQ, sum8(acc));
 #pragma unroll
@@ -327,7 +327,7 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
       if (!has_b) break;
       tmem_wait_chunks<SEGC>(vb);
       if (sg + 2 < nseg) tmem_ld_chunks<SEGC>(col + (sg + 2) * 32 * SEGC, va);
-      relu_dot<SEGC>(vb, w + (sg + 1) * 32 * SEGC, acc);
+      relu_dot<1>(vb, w + (sg + 1) * 32 * SEGC, acc);
       if ((sg + 2) % SPQ == 0) {
         filter_append(f, rbase + (sg + 1) / SPQ, sum8(acc));
 #pragma unroll
@@ -368,6 +368,32 @@ __device__ __forceinline__ void unit_heads(const FilterCtx& f, uint32_t col, con
       chunk(vb, c + 1);
       if (c + 2 < nchunk) tmem_wait_chunks<1>(va);
     }
+  }
+}
+
+// unit_heads with the row count known at compile time (HT >= 32): the whole
+// unit is one straight-line sequence of 32-column segments, the load of
+// segment i+1 in flight while segment i is reduced.
+template <int HT, int NQ>
+__device__ __forceinline__ void unit_heads_n(const FilterCtx& f, uint32_t col, const float* w,
+                                             int rbase) {
+  static_assert(HT >= 32, "32-column segments");
+  constexpr int SPQ = HT / 32;                 // segments per query row
+  constexpr int NSEG = NQ * SPQ;
+  uint32_t v[2][1][32];
+  unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+  tmem_ld_chunks<1>(col, v[0]);
+  tmem_wait_chunks<1>(v[0]);
+#pragma unroll
+  for (int sg = 0; sg < NSEG; ++sg) {
+    if (sg + 1 < NSEG) tmem_ld_chunks<1>(col + (sg + 1) * 32, v[(sg + 1) & 1]);
+    relu_dot<1>(v[sg & 1], w + sg * 32, acc);
+    if ((sg + 1) % SPQ == 0) {
+      filter_append(f, rbase + sg / SPQ, sum8(acc));
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = 0ull;
+    }
+    if (sg + 1 < NSEG) tmem_wait_chunks<1>(v[(sg + 1) & 1]);
   }
 }
 
@@ -920,7 +946,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               filter_append(fc, r, (acc0 + acc1) + (acc2 + acc3));
             }
           } else {
-            unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+            if constexpr (HT >= 32) {
+              if (qhalf == 2)
+                unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+              else if (qhalf == 1)
+                unit_heads_n<HT, 1>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+              else
+                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+            } else {
+              unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+            }
           }
           tc_fence_before();
           __syncwarp();
