@@ -98,7 +98,12 @@ ROUTED = ("misa", "dagger", "hisa")
 # dram__bytes_read.sum + dram__bytes_write.sum of one scan-kernel launch, from the
 # ncu captures summarised under profiles/, valid only while the kernel sources
 # hash to `src`; otherwise the traffic is reported as null.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/scan_kernel_dsa_prefill_32k.md: 601.86 MB read + 1.91 GB written
+    "dsa_prefill_32k": {"bytes": 601_860_000 + 1_910_000_000, "src": "28bdbb0a5c27bd8b"},
+    # profiles/scan_kernel_dsa_decode_128k.md: 557.22 MB read + 24.83 MB written
+    "dsa_decode_128k": {"bytes": 557_220_000 + 24_830_000, "src": "28bdbb0a5c27bd8b"},
+}
 
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
 
