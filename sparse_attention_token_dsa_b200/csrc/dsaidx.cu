@@ -147,7 +147,8 @@ ScanPlan plan_gather(MmaKind kind, int batch, int n_q, int H, int keep) {
   pl.QG = 1;
   pl.G = 1;
   pl.qcols = H < 16 ? 16 : H;
-  pl.stage_cols = pl.qcols > 128 ? 256 : 128;
+  // narrow accumulators: more TMEM stages let the MMA run further ahead
+  pl.stage_cols = pl.qcols > 128 ? 256 : (pl.qcols > 64 ? 128 : 64);
   pl.n_qt = n_q;
   pl.rows = batch * n_q;
   finish_plan(pl, true);

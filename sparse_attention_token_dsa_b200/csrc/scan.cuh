@@ -57,8 +57,8 @@ struct ScanArgs {
   int32_t QG;            // query rows per accumulator group (<= 256 / (H * parts))
   int32_t qcols;         // MMA N per group: max(16, QG * H * parts) query-head columns
   int32_t G;             // groups per work item (1 or 2)
-  int32_t stage_cols;    // TMEM columns per accumulator stage (128 or 256)
-  int32_t tstages;       // accumulator stages in TMEM (2 or 4; tstages * stage_cols <= 512)
+  int32_t stage_cols;    // TMEM columns per accumulator stage (64, 128 or 256)
+  int32_t tstages;       // accumulator stages in TMEM (2 .. 8; tstages * stage_cols <= 512)
   int32_t kstages;       // K-tile pipeline depth (2 .. 8)
   int32_t n_qt;          // query tiles per sequence (ceil(n_q / (QG*G)))
   int32_t C;             // key chunks per row (split-K); 1 = whole prefix
@@ -96,7 +96,7 @@ constexpr int kCompactSlack = 64 * 2 * kUpdateSteps + 128;
 constexpr int kMaxGatherKeys = 8192;
 constexpr int kGatherBins = 4096;     // linear score bins of the end-of-row selection
 constexpr int kGatherBoundary = 256;  // boundary-bin candidates ranked by one warp
-constexpr int kMaxTStages = 4;
+constexpr int kMaxTStages = 8;
 
 template <MmaKind KIND>
 struct ScanCfg {
