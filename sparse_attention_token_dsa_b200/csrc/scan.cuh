@@ -728,8 +728,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       int cnt = 0;
       bool radix = false;
       if (n_legal > a.keep) {
-        // linear score bins over [lo, hi]: count, locate the bin of the keep-th best,
-        // emit every candidate above it and rank that bin's few candidates exactly
+        // Linear score bins over [lo, hi]: count, locate the bin holding the keep-th
+        // best, emit every candidate above it and rank that bin's candidates exactly.
+        // A crowded bin is split once more into its own linear bins; only a bin that
+        // stays crowded (long runs of equal scores) falls back to the radix select.
         float lo2 = T->gather_lo[0], hi2 = T->gather_hi[0];
 #pragma unroll
         for (int w = 1; w < kEpiWarps; ++w) {
@@ -737,76 +739,101 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           hi2 = fmaxf(hi2, T->gather_hi[w]);
         }
         const float span = hi2 - lo2;
-        const float scale = span > 0.f ? (float)(kGatherBins - 1) / span : 0.f;
-        auto bin_of = [&](uint64_t c) {
-          const int b = __float2int_rz((key_score((uint32_t)(c >> 32)) - lo2) * scale);
+        const float scale0 = span > 0.f ? (float)(kGatherBins - 1) / span : 0.f;
+        auto bin_at = [&](uint64_t c, float base, float sc) {
+          const int b = __float2int_rz((key_score((uint32_t)(c >> 32)) - base) * sc);
           return min(kGatherBins - 1, max(0, b));
         };
-        for (int e = etid; e < ncand; e += kEpiThreads) {
-          const uint64_t c = cand[e];
-          if (c != 0ull) atomicAdd(&ghist[bin_of(c)], 1u);
-        }
-        named_bar_sync(kBarEpi, kEpiThreads);
-        // thread t owns the 16 bins from 4095 - 16 t downwards; scan in that order
-        uint32_t own = 0;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) own += ghist[kGatherBins - 1 - 16 * etid - i];
-        uint32_t incl = own;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
-          if (lane >= off) incl += o;
-        }
-        uint32_t* wsum = reinterpret_cast<uint32_t*>(T->sel.hist);
-        if (lane == 31) wsum[warp] = incl;
-        named_bar_sync(kBarEpi, kEpiThreads);
-        uint32_t wbase = 0;
-        for (int w = 0; w < warp; ++w) wbase += wsum[w];
-        const uint32_t excl = wbase + incl - own;
-        const uint32_t need = (uint32_t)a.keep;
-        if (excl < need && need <= excl + own) {
-          uint32_t cum = excl;
-          for (int i = 0; i < 16; ++i) {
-            const int b = kGatherBins - 1 - 16 * etid - i;
-            const uint32_t c = ghist[b];
-            if (cum + c >= need) {
-              T->sel.sel[2] = b;
-              T->sel.sel[3] = (int)cum;            // candidates strictly above bin b
-              break;
+        int need = a.keep;          // still to emit
+        int emitted = 0;            // winners already in out[]
+        int scope_bin = -1;         // level 1: only candidates of this level-0 bin
+        float base = lo2, scale = scale0;
+        bool done = false;
+        for (int level = 0; level < 2 && !done && !radix; ++level) {
+          if (level == 1) {
+            for (int i = etid; i < kGatherBins; i += kEpiThreads) ghist[i] = 0u;
+            if (etid == 0) {
+              T->gather_nwin = 0;
+              T->gather_nbnd = 0;
             }
-            cum += c;
+            named_bar_sync(kBarEpi, kEpiThreads);
           }
-        }
-        named_bar_sync(kBarEpi, kEpiThreads);
-        const int bstar = T->sel.sel[2], above = T->sel.sel[3];
-        for (int e0 = 0; e0 < ncand; e0 += kEpiThreads) {
-          const int e = e0 + etid;
-          const uint64_t c = e < ncand ? cand[e] : 0ull;
-          const int b = c != 0ull ? bin_of(c) : -1;
-          const bool win = b > bstar, edge = b == bstar;
-          const unsigned bw = __ballot_sync(0xffffffffu, win);
-          const unsigned be = __ballot_sync(0xffffffffu, edge);
-          int pw = 0, pe = 0;
-          if (lane == 0) {
-            if (bw) pw = atomicAdd(&T->gather_nwin, __popc(bw));
-            if (be) pe = atomicAdd(&T->gather_nbnd, __popc(be));
+          auto in_scope = [&](uint64_t c) {
+            return c != 0ull && (scope_bin < 0 || bin_at(c, lo2, scale0) == scope_bin);
+          };
+          for (int e = etid; e < ncand; e += kEpiThreads) {
+            const uint64_t c = cand[e];
+            if (in_scope(c)) atomicAdd(&ghist[bin_at(c, base, scale)], 1u);
           }
-          pw = __shfl_sync(0xffffffffu, pw, 0);
-          pe = __shfl_sync(0xffffffffu, pe, 0);
-          const unsigned lt = (1u << lane) - 1u;
-          if (win) out[pw + __popc(bw & lt)] = c;
-          if (edge) {
-            const int sl = pe + __popc(be & lt);
-            if (sl < kGatherBoundary) gbnd[sl] = c;
+          named_bar_sync(kBarEpi, kEpiThreads);
+          // thread t owns the 16 bins from 4095 - 16 t downwards; scan in that order
+          uint32_t own = 0;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) own += ghist[kGatherBins - 1 - 16 * etid - i];
+          uint32_t incl = own;
+#pragma unroll
+          for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
           }
-        }
-        named_bar_sync(kBarEpi, kEpiThreads);
-        const int nb = T->gather_nbnd;
-        if (nb <= kGatherBoundary) {
-          if (warp == 0) warp_take_top(gbnd, nb, a.keep - above, out, above, lane);
-          cnt = a.keep;
-        } else {
-          radix = true;                                  // a crowded bin (ties): exact radix
+          uint32_t* wsum = reinterpret_cast<uint32_t*>(T->sel.hist);
+          if (lane == 31) wsum[warp] = incl;
+          named_bar_sync(kBarEpi, kEpiThreads);
+          uint32_t wbase = 0;
+          for (int w = 0; w < warp; ++w) wbase += wsum[w];
+          const uint32_t excl = wbase + incl - own;
+          if (excl < (uint32_t)need && (uint32_t)need <= excl + own) {
+            uint32_t cum = excl;
+            for (int i = 0; i < 16; ++i) {
+              const int b = kGatherBins - 1 - 16 * etid - i;
+              const uint32_t c = ghist[b];
+              if (cum + c >= (uint32_t)need) {
+                T->sel.sel[2] = b;
+                T->sel.sel[3] = (int)cum;          // in-scope candidates strictly above bin b
+                break;
+              }
+              cum += c;
+            }
+          }
+          named_bar_sync(kBarEpi, kEpiThreads);
+          const int bstar = T->sel.sel[2], above = T->sel.sel[3];
+          for (int e0 = 0; e0 < ncand; e0 += kEpiThreads) {
+            const int e = e0 + etid;
+            const uint64_t c = e < ncand ? cand[e] : 0ull;
+            const int b = in_scope(c) ? bin_at(c, base, scale) : -1;
+            const bool win = b > bstar, edge = b == bstar;
+            const unsigned bw = __ballot_sync(0xffffffffu, win);
+            const unsigned be = __ballot_sync(0xffffffffu, edge);
+            int pw = 0, pe = 0;
+            if (lane == 0) {
+              if (bw) pw = atomicAdd(&T->gather_nwin, __popc(bw));
+              if (be) pe = atomicAdd(&T->gather_nbnd, __popc(be));
+            }
+            pw = __shfl_sync(0xffffffffu, pw, 0);
+            pe = __shfl_sync(0xffffffffu, pe, 0);
+            const unsigned lt = (1u << lane) - 1u;
+            if (win) out[emitted + pw + __popc(bw & lt)] = c;
+            if (edge) {
+              const int sl = pe + __popc(be & lt);
+              if (sl < kGatherBoundary) gbnd[sl] = c;
+            }
+          }
+          named_bar_sync(kBarEpi, kEpiThreads);
+          const int nb = T->gather_nbnd;
+          emitted += above;
+          need -= above;
+          if (nb <= kGatherBoundary) {
+            if (warp == 0) warp_take_top(gbnd, nb, need, out, emitted, lane);
+            cnt = a.keep;
+            done = true;
+          } else if (level == 0 && scale0 > 0.f) {
+            // split the crowded bin: its scores lie in [lo + b / scale, lo + (b + 1) / scale)
+            scope_bin = bstar;
+            base = lo2 + (float)bstar / scale0;
+            scale = scale0 * (float)(kGatherBins - 1);
+          } else {
+            radix = true;                                // equal scores: exact radix
+          }
         }
       }
       if (n_legal > 0 && (n_legal <= a.keep || radix)) {
