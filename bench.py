@@ -39,6 +39,11 @@ METRIC = "indexer ms/layer @128K prefill; decode µs/query; % of tensor-pipe / H
 
 _L128 = 131072
 WORKLOADS = {
+    "dsa_prefill_1k_int": dict(
+        desc="DSA indexer prefill, batch 1, L=1024 causal, H_I=64, d=128, top-k=128, "
+             "integer q,k in [-3,3] and w in [-2,2] (bf16 storage, exact)",
+        kind="prefill", batch=1, L=1024, H=64, topk=128, fp8=False, seed=1, needles=0,
+        integer=True),
     "dsa_prefill_32k": dict(
         desc="DSA indexer prefill, batch 1, L=32768 causal, H_I=64, d=128, top-k=2048, "
              "bf16 q,k ~N(0,1), w ~N(0,1/64), 32 planted needles",
@@ -127,6 +132,9 @@ def peaks():
 
 
 def make_problem(w):
+    if w.get("integer"):
+        return gen.integer_problem(w["seed"], w["batch"], w["L"], w["L"], w["H"], 128, w["topk"],
+                                   dtype=gen.BF16)
     if w["kind"] == "decode":
         p, _ = gen.decode_problem(w["seed"], w["batch"], w["L"], w["H"], 128, w["topk"])
         return p
@@ -330,6 +338,17 @@ def run_reference(args, w, p):
 
 # ------------------------------------------------------------------ GPU arm --
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -453,10 +472,7 @@ def main():
     st = B.dsa_read_status(ws)
     if st != 0:
         raise RuntimeError(f"device status {st}: {B.status_string(st)}")
-    if world > 1:
-        t = torch.tensor([elapsed], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
+    elapsed = max_over_ranks(elapsed, dev)
 
     # end to end through the public call with host buffers (pinned), copies inside
     qp, kp, wp = qh.pin_memory(), kh.pin_memory(), wh.pin_memory()
@@ -493,10 +509,7 @@ def main():
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = qh.numel() * qh.element_size() + kh.numel() * kh.element_size() + wh.numel() * 4
     d2h = idx.numel() * 4 + sc.numel() * 4
 
