@@ -110,36 +110,36 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
   const int g0 = nseg >= NW ? wid : (wid < parts * nseg ? wid % nseg : nseg);
   const int gstep = nseg >= NW ? NW : nseg;
   const int part = nseg >= NW ? 0 : wid / nseg;
-  for (int g = g0; g < nseg; g += gstep) {
-    const uint64_t* p = segp[g];
-    const int n = segn[g];
-    for (int i0 = part * 256; i0 < n; i0 += parts * 256) {
-      uint64_t v[8];
+  // every candidate >= thr of the row's logs, warp-uniformly: fn(v, is_candidate)
+  auto for_each_candidate = [&](auto&& fn) {
+    for (int g = g0; g < nseg; g += gstep) {
+      const uint64_t* p = segp[g];
+      const int n = segn[g];
+      for (int i0 = part * 256; i0 < n; i0 += parts * 256) {
+        uint64_t v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * 32 + lane;
-        v[j] = i < n ? p[i] : 0ull;
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = i0 + j * 32 + lane;
-        const bool keep = i < n && v[j] >= thr;
-        const unsigned bal = __ballot_sync(0xffffffffu, keep);
-        if (bal) {
-          int base = 0;
-          if (lane == 0) base = atomicAdd(&G->staged, __popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          if (keep) {
-            const int slot = base + __popc(bal & ((1u << lane) - 1));
-            if (slot < stage_cap) stage[slot] = v[j];
-            const int bin = min(255, (int)(v[j] >> 48) - thr16);
-            const unsigned peers = __match_any_sync(bal, bin);
-            if (lane == __ffs(peers) - 1) atomicAdd(&G->sc.hist[bin], __popc(peers));
-          }
+        for (int j = 0; j < 8; ++j) {
+          const int i = i0 + j * 32 + lane;
+          v[j] = i < n ? p[i] : 0ull;
         }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) fn(v[j], i0 + j * 32 + lane < n && v[j] >= thr);
       }
     }
-  }
+  };
+  for_each_candidate([&](uint64_t v, bool keep) {
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (bal) {
+      int base = 0;
+      if (lane == 0) base = atomicAdd(&G->staged, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (keep) {
+        const int slot = base + __popc(bal & ((1u << lane) - 1));
+        if (slot < stage_cap) stage[slot] = v;
+        atomicAdd(&G->sc.hist[min(255, (int)(v >> 48) - thr16)], 1);
+      }
+    }
+  });
   named_bar_sync(bar, NT);
   const int total = G->staged;
   int n;  // number of result keys in out[]
@@ -148,9 +148,12 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
     for (int i = tid; i < total; i += NT) out[i] = stage[i];
     n = total;
   } else {
-    bool fb = total > stage_cap;
+    // more candidates than the stage holds: the histogram is still complete, so
+    // winners and the boundary bin are taken from the logs in a second read
+    const bool overflow = total > stage_cap;
+    bool fb = false;
     int bstar = 0, above = 0;
-    if (!fb) {
+    {
       if (tid < 32) {
         int ab;
         const int b = hist_find(reinterpret_cast<const uint32_t*>(G->sc.hist), 0, a.topk, lane, &ab);
@@ -167,10 +170,8 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
     }
     if (!fb) {
       // winners above the boundary bin; the boundary bin's candidates aside
-      for (int i0 = 0; i0 < total; i0 += NT) {
-        const int i = i0 + tid;
-        const uint64_t v = i < total ? stage[i] : 0ull;
-        const int bin = i < total ? min(255, (int)(v >> 48) - thr16) : -1;
+      auto sort_out = [&](uint64_t v, bool cand) {
+        const int bin = cand ? min(255, (int)(v >> 48) - thr16) : -1;
         const bool win = bin > bstar, edge = bin == bstar;
         const unsigned bw = __ballot_sync(0xffffffffu, win);
         const unsigned be = __ballot_sync(0xffffffffu, edge);
@@ -187,6 +188,14 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
           const int slot = bedge + __popc(be & lt);
           if (slot < kFinBoundary) bnd[slot] = v;
         }
+      };
+      if (!overflow) {
+        for (int i0 = 0; i0 < total; i0 += NT) {
+          const int i = i0 + tid;
+          sort_out(i < total ? stage[i] : 0ull, i < total);
+        }
+      } else {
+        for_each_candidate(sort_out);
       }
       named_bar_sync(bar, NT);
       const int nb = G->nbnd;

@@ -275,21 +275,16 @@ __device__ void sort_desc_regs(uint64_t* a, int n, int tid, int bar_id) {
   named_bar_sync(bar_id, NT);
 }
 
-// Exact selection of the `need` largest of the n <= 256 keys in b[] by one
-// warp (register bitonic sort), appended to out[base..].
+// Exact selection of the `need` largest of the n <= 256 distinct keys in b[]
+// by one warp, appended to out[base..] in descending order: each key's rank is
+// the number of larger keys (n compares per key, read as smem broadcasts).
 __device__ __forceinline__ void warp_take_top(const uint64_t* b, int n, int need, uint64_t* out,
                                               int base, int lane) {
-  uint64_t v[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = lane * 8 + e;
-    v[e] = i < n ? b[i] : 0ull;
-  }
-  bitonic_regs_desc<32, 8>(v, nullptr, lane, 0);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int i = lane * 8 + e;
-    if (i < need) out[base + i] = v[e];
+  for (int i = lane; i < n; i += 32) {
+    const uint64_t v = b[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += b[j] > v ? 1 : 0;
+    if (rank < need) out[base + rank] = v;
   }
 }
 
