@@ -397,6 +397,37 @@ __device__ __forceinline__ void unit_heads_n(const FilterCtx& f, uint32_t col, c
   }
 }
 
+// unit_heads for HT in {8, 16} with the row count known at compile time: each
+// 32-column chunk holds 32 / HT rows; straight-line, next chunk's load in flight.
+template <int HT, int NQ>
+__device__ __forceinline__ void unit_heads_small(const FilterCtx& f, uint32_t col, const float* w,
+                                                 int rbase) {
+  static_assert(HT < 32 && NQ % (32 / HT) == 0, "whole chunks");
+  constexpr int QPC = 32 / HT;
+  constexpr int NCH = NQ / QPC;
+  uint32_t v[2][1][32];
+  tmem_ld_chunks<1>(col, v[0]);
+  tmem_wait_chunks<1>(v[0]);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c + 1 < NCH) tmem_ld_chunks<1>(col + (c + 1) * 32, v[(c + 1) & 1]);
+#pragma unroll
+    for (int qq = 0; qq < QPC; ++qq) {
+      float b[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int jj = 0; jj < HT; jj += 4) {
+        const float4 wv = *reinterpret_cast<const float4*>(w + c * 32 + qq * HT + jj);
+        b[0] = fmaf(wv.x, fmaxf(__uint_as_float(v[c & 1][0][qq * HT + jj + 0]), 0.f), b[0]);
+        b[1] = fmaf(wv.y, fmaxf(__uint_as_float(v[c & 1][0][qq * HT + jj + 1]), 0.f), b[1]);
+        b[2] = fmaf(wv.z, fmaxf(__uint_as_float(v[c & 1][0][qq * HT + jj + 2]), 0.f), b[2]);
+        b[3] = fmaf(wv.w, fmaxf(__uint_as_float(v[c & 1][0][qq * HT + jj + 3]), 0.f), b[3]);
+      }
+      filter_append(f, rbase + c * QPC + qq, (b[0] + b[1]) + (b[2] + b[3]));
+    }
+    if (c + 1 < NCH) tmem_wait_chunks<1>(v[(c + 1) & 1]);
+  }
+}
+
 // sum_j w_j ReLU(D_j) over the HT accumulator columns of one query row (TMEM
 // columns [0, HT) at taddr), for the gathered-key epilogue.
 template <int HT>
@@ -981,7 +1012,10 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               else
                 unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
             } else {
-              unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+              if (qhalf == 8)
+                unit_heads_small<HT, 8>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+              else
+                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
             }
           }
           tc_fence_before();
