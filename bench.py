@@ -513,6 +513,43 @@ def main():
     h2d = qh.numel() * qh.element_size() + kh.numel() * kh.element_size() + wh.numel() * 4
     d2h = idx.numel() * 4 + sc.numel() * 4
 
+    # quality of the selection (outside every timed region): needle recall at the
+    # probe rows; for routed methods the overlap with the exact DSA top-k of the
+    # same rows (both on the GPU) and the dense layer's time for the speed-up
+    quality = {}
+    if rank == 0:
+        gi = idx.reshape(p.batch * p.n_q, p.topk)
+        if p.needles:
+            found = 0
+            for b, t, s_ in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
+                found += int((gi[b * p.n_q + t] == s_).any().item())
+            quality["needle_recall"] = found / len(p.needles["s"])
+        if kind in ROUTED:
+            dprob = B.problem(q, k, p.topk)
+            dws = torch.empty(B.dsa_workspace_size(dprob), dtype=torch.uint8, device=dev)
+            didx = torch.empty_like(idx)
+            dsc = torch.empty_like(sc)
+            B.dsa_index(q, k, wt, p.topk, out=(didx, dsc), workspace=dws)
+            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            d0.record(stream)
+            B.dsa_index(q, k, wt, p.topk, out=(didx, dsc), workspace=dws)
+            d1.record(stream)
+            torch.cuda.synchronize()
+            dense_ms = d0.elapsed_time(d1)
+            rows = torch.linspace(p.n_q // 16, p.n_q - 1, 512).long().to(dev)
+            a_ = gi[rows].sort(dim=1).values
+            b_ = didx.reshape(-1, p.topk)[rows].sort(dim=1).values
+            inter = torch.zeros(len(rows), device=dev)
+            for j in range(0, p.topk, 256):          # |A ∩ B| by membership of A's entries
+                blk = a_[:, j:j + 256]
+                pos = torch.searchsorted(b_, blk).clamp(max=p.topk - 1)
+                inter += ((torch.gather(b_, 1, pos) == blk) & (blk >= 0)).sum(1).float()
+            nv = (a_ >= 0).sum(1).float()
+            iou = (inter / (2 * nv - inter)).mean().item()
+            quality.update({"iou_vs_dsa": iou, "dsa_ms": dense_ms,
+                            "speedup_vs_dsa": dense_ms / (elapsed / args.steps)})
+            del dws
+
     if rank == 0:
         unit, scale = unit_of(w)
         ms_per_step = elapsed / args.steps
@@ -556,6 +593,7 @@ def main():
             cfg["select_ms"] = ms_per_step - stage_ms
         else:
             cfg["row_chunks"] = chunks
+        cfg.update(quality)
         line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
                 "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
