@@ -153,25 +153,43 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
     const bool overflow = total > stage_cap;
     bool fb = false;
     int bstar = 0, above = 0;
-    {
+    // the 256 bins cover score-key prefixes base16 .. base16 + 254 (bin 255 holds
+    // everything higher); a k-th best beyond that window moves the window up and
+    // recounts (the candidates below the new base cannot be among the top k)
+    int base16 = thr16;
+    for (int window = 0;; ++window) {
       if (tid < 32) {
         int ab;
         const int b = hist_find(reinterpret_cast<const uint32_t*>(G->sc.hist), 0, a.topk, lane, &ab);
         if (lane == 0) {
           G->sc.sel[0] = b;
           G->sc.sel[1] = ab;
-          if (b < 0 || b == 255) G->fallback = 1;
+          G->fallback = (b < 0 || (b == 255 && window == 7)) ? 1 : 0;
         }
       }
       named_bar_sync(bar, NT);
       fb = G->fallback != 0;
       bstar = G->sc.sel[0];
       above = G->sc.sel[1];
+      if (fb || bstar < 255) break;
+      base16 += 255;
+      for (int i = tid; i < 256; i += NT) G->sc.hist[i] = 0;
+      named_bar_sync(bar, NT);
+      auto recount = [&](uint64_t v, bool cand) {
+        const int bin = cand ? min(255, (int)(v >> 48) - base16) : -1;
+        if (bin >= 0) atomicAdd(&G->sc.hist[bin], 1);
+      };
+      if (!overflow) {
+        for (int i = tid; i < total; i += NT) recount(stage[i], true);
+      } else {
+        for_each_candidate(recount);
+      }
+      named_bar_sync(bar, NT);
     }
     if (!fb) {
       // winners above the boundary bin; the boundary bin's candidates aside
       auto sort_out = [&](uint64_t v, bool cand) {
-        const int bin = cand ? min(255, (int)(v >> 48) - thr16) : -1;
+        const int bin = cand ? min(255, (int)(v >> 48) - base16) : -1;
         const bool win = bin > bstar, edge = bin == bstar;
         const unsigned bw = __ballot_sync(0xffffffffu, win);
         const unsigned be = __ballot_sync(0xffffffffu, edge);
