@@ -21,7 +21,7 @@ using namespace dsa;
 
 namespace {
 
-constexpr int kTargetCtas = 296;  // 148 SMs x 2: sizing target for split-K decode
+constexpr int kTargetCtas = 296;  // split-K decode: about two work items per SM (persistent CTAs)
 constexpr size_t kAlign = 256;
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
@@ -59,14 +59,11 @@ size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols, int kstages, bool
 // memory and TMEM; a CTA alone on its SM deepens its K pipeline into the
 // spare shared memory, and the TMEM accumulator stages fill 512 columns.
 void finish_plan(ScanPlan& pl, bool gather) {
-  const size_t per_sm = 228 * 1024;
   pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather);
-  int by_smem = (int)(per_sm / (pl.smem + 1024));
-  int by_tmem = 512 / (2 * pl.stage_cols);
-  pl.ctas_per_sm = by_smem < by_tmem ? by_smem : by_tmem;
-  if (pl.ctas_per_sm > 2) pl.ctas_per_sm = 2;
-  if (pl.ctas_per_sm < 1) pl.ctas_per_sm = 1;
-  if (pl.ctas_per_sm == 1) {
+  // 320 threads at up to 168 registers take more than half the register file:
+  // one CTA per SM, whatever shared memory and TMEM would allow
+  pl.ctas_per_sm = 1;
+  {
     while (pl.kstages < 6 &&
            scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages + 1, gather) <= kSmemBudget)
       ++pl.kstages;
