@@ -985,20 +985,37 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               const float* wr = &T->wsm[r * HT];
               const uint32_t cb = taddr + (qbeg + qi) * HT * PARTS;
               float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+              // hi / lo parts of 16 heads at a time, the next 16 in flight
+              auto part16 = [&](const uint32_t (&hi)[16], const uint32_t (&lo)[16], int c0) {
 #pragma unroll
-              for (int c0 = 0; c0 < HT; c0 += 32) {
-                uint32_t v0[32], v1[32];
-                tmem_ld32(cb + c0, v0);
-                tmem_ld32(cb + HT + c0, v1);
-                tmem_ld_wait(v0);
-                tmem_ld_wait(v1);
-#pragma unroll
-                for (int jj = 0; jj < 32; jj += 4) {
+                for (int jj = 0; jj < 16; jj += 4) {
                   const float4 wv = *reinterpret_cast<const float4*>(wr + c0 + jj);
-                  acc0 = fmaf(wv.x, fmaxf(fmaf(__uint_as_float(v1[jj + 0]), 0.0625f, __uint_as_float(v0[jj + 0])), 0.f), acc0);
-                  acc1 = fmaf(wv.y, fmaxf(fmaf(__uint_as_float(v1[jj + 1]), 0.0625f, __uint_as_float(v0[jj + 1])), 0.f), acc1);
-                  acc2 = fmaf(wv.z, fmaxf(fmaf(__uint_as_float(v1[jj + 2]), 0.0625f, __uint_as_float(v0[jj + 2])), 0.f), acc2);
-                  acc3 = fmaf(wv.w, fmaxf(fmaf(__uint_as_float(v1[jj + 3]), 0.0625f, __uint_as_float(v0[jj + 3])), 0.f), acc3);
+                  acc0 = fmaf(wv.x, fmaxf(fmaf(__uint_as_float(lo[jj + 0]), 0.0625f, __uint_as_float(hi[jj + 0])), 0.f), acc0);
+                  acc1 = fmaf(wv.y, fmaxf(fmaf(__uint_as_float(lo[jj + 1]), 0.0625f, __uint_as_float(hi[jj + 1])), 0.f), acc1);
+                  acc2 = fmaf(wv.z, fmaxf(fmaf(__uint_as_float(lo[jj + 2]), 0.0625f, __uint_as_float(hi[jj + 2])), 0.f), acc2);
+                  acc3 = fmaf(wv.w, fmaxf(fmaf(__uint_as_float(lo[jj + 3]), 0.0625f, __uint_as_float(hi[jj + 3])), 0.f), acc3);
+                }
+              };
+              constexpr int NCH = HT / 16;
+              uint32_t ha[16], la[16], hb[16], lb[16];
+              tmem_ld16(cb, ha);
+              tmem_ld16(cb + HT, la);
+              tmem_ld_wait(ha, la);
+#pragma unroll
+              for (int c = 0; c < NCH; c += 2) {
+                if (c + 1 < NCH) {
+                  tmem_ld16(cb + (c + 1) * 16, hb);
+                  tmem_ld16(cb + HT + (c + 1) * 16, lb);
+                }
+                part16(ha, la, c * 16);
+                if (c + 1 < NCH) {
+                  tmem_ld_wait(hb, lb);
+                  if (c + 2 < NCH) {
+                    tmem_ld16(cb + (c + 2) * 16, ha);
+                    tmem_ld16(cb + HT + (c + 2) * 16, la);
+                  }
+                  part16(hb, lb, (c + 1) * 16);
+                  if (c + 2 < NCH) tmem_ld_wait(ha, la);
                 }
               }
               filter_append(fc, r, (acc0 + acc1) + (acc2 + acc3));
