@@ -115,7 +115,7 @@ typedef struct {
  *                    [8, heads]
  *   k_prime     k' : MISA-dagger candidate pool (e.g. 8192), topk <= k' <= 8192
  *   hisa_block  b  : tokens per HISA block (e.g. 64)
- *   hisa_r      r  : HISA blocks kept per query (e.g. 128), 1 <= r <= 8192
+ *   hisa_r      r  : HISA blocks kept per query (e.g. 128), r * b <= 8192
  * Block sizes must be powers of two in [16, 4096], and the router sees at
  * most 224 full blocks: n_k / B <= 224 (B = 1024 covers 229,376 tokens).
  * The routed entry points take bf16 q and k only (q_dtype == k_dtype ==

@@ -7,17 +7,21 @@
 // kernel fuses score, causal mask and top-k so the n^2 score matrix never
 // reaches memory, section 2.2 "kernel boundary").  Restricted to a routed
 // head subset this is MISA's step 4 ("MISA: Mixture of Indexer Sparse
-// Attention", method step 4): the caller passes gathered q / w rows.
+// Attention", method step 4): the caller passes gathered q / w rows.  The
+// keys of a work item are a contiguous range, full-block representatives
+// (HISA's coarse stage), or a per-row list gathered by TMA (the MISA-dagger and
+// HISA reranks, whose rows select once at the end instead of streaming).
 //
-// Layout of one CTA (persistent, one work item at a time):
+// Layout of one CTA (persistent, one per SM, one work item at a time):
 //   warps 0-7  epilogue: TMEM -> registers, ReLU, * w, sum over heads, causal
 //              mask, composite key, threshold filter, append to warp-owned
 //              candidate sub-logs, per-row threshold maintenance
 //   warp 8     TMA producer: Q tile of the item (resident), K tiles streamed
+//              through 2-6 stages
 //   warp 9     MMA issuer (one thread) + TMEM allocator
 // MMA: M = 128 keys (TMEM lane = key), N = query rows x heads (x 2 for the
-// split-query fp8 form), K = d; fp32 accumulate in TMEM, two accumulator
-// stages so the epilogue of one unit overlaps the MMA of the next.
+// split-query fp8 form), K = d; fp32 accumulate in TMEM, 2-8 accumulator
+// stages so the epilogue of one unit overlaps the MMAs of the next.
 //
 // Streaming top-k.  A candidate (score, key) is kept while its composite key
 // (order-preserving score bits, then ~index) is >= the row's threshold thr.
