@@ -104,10 +104,10 @@ ROUTED = ("misa", "dagger", "hisa")
 # ncu captures summarised under profiles/, valid only while the kernel sources
 # hash to `src`; otherwise the traffic is reported as null.
 TRAFFIC = {
-    # profiles/scan_kernel_dsa_prefill_32k.md: 601.86 MB read + 1.91 GB written
-    "dsa_prefill_32k": {"bytes": 601_860_000 + 1_910_000_000, "src": "28bdbb0a5c27bd8b"},
-    # profiles/scan_kernel_dsa_decode_128k.md: 557.22 MB read + 24.83 MB written
-    "dsa_decode_128k": {"bytes": 557_220_000 + 24_830_000, "src": "28bdbb0a5c27bd8b"},
+    # profiles/scan_kernel_dsa_prefill_32k.md: 600.78 MB read + 1.91 GB written
+    "dsa_prefill_32k": {"bytes": 600_780_000 + 1_910_000_000, "src": "eca0cc460ca22400"},
+    # profiles/scan_kernel_dsa_decode_128k.md: 559.46 MB read + 24.39 MB written
+    "dsa_decode_128k": {"bytes": 559_460_000 + 24_390_000, "src": "eca0cc460ca22400"},
 }
 
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
