@@ -104,10 +104,10 @@ ROUTED = ("misa", "dagger", "hisa")
 # ncu captures summarised under profiles/, valid only while the kernel sources
 # hash to `src`; otherwise the traffic is reported as null.
 TRAFFIC = {
-    # profiles/scan_kernel_dsa_prefill_32k.md: 600.78 MB read + 1.91 GB written
-    "dsa_prefill_32k": {"bytes": 600_780_000 + 1_910_000_000, "src": "eca0cc460ca22400"},
-    # profiles/scan_kernel_dsa_decode_128k.md: 559.46 MB read + 24.39 MB written
-    "dsa_decode_128k": {"bytes": 559_460_000 + 24_390_000, "src": "eca0cc460ca22400"},
+    # profiles/scan_kernel_dsa_prefill_32k.md: 601.29 MB read + 1.91 GB written
+    "dsa_prefill_32k": {"bytes": 601_290_000 + 1_910_000_000, "src": "23b61bde9a857492"},
+    # profiles/scan_kernel_dsa_decode_128k.md: 559.32 MB read + 26.36 MB written
+    "dsa_decode_128k": {"bytes": 559_320_000 + 26_360_000, "src": "23b61bde9a857492"},
 }
 
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]

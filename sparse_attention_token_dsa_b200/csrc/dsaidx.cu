@@ -102,7 +102,10 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.QG = QG;
   pl.G = G;
   pl.qcols = QG * hp;
-  pl.stage_cols = pl.qcols > 128 ? 256 : 128;
+  {
+    const int n = QG * H;  // MMA N: the split-query parts share one accumulator
+    pl.stage_cols = n > 128 ? 256 : (n > 64 ? 128 : 64);
+  }
   pl.n_qt = (n_q + QG * G - 1) / (QG * G);
   pl.rows = batch * n_q;
   finish_plan(pl, false);
@@ -857,7 +860,8 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   }
   CUtensorMap qm, km;
   const int qesz = pl.split ? 1 : pl.esz;
-  if (!make_map(&qm, qop, qesz, (uint64_t)pl.rows * p->heads * pl.parts, (uint32_t)pl.qcols))
+  if (!make_map(&qm, qop, qesz, (uint64_t)pl.rows * p->heads * pl.parts,
+                (uint32_t)(pl.qcols / pl.parts)))
     return DSA_ERR_CUDA;
   if (!make_map(&km, k, pl.esz, (uint64_t)p->batch * p->n_k, 128)) return DSA_ERR_CUDA;
   ScanArgs a{};

@@ -43,12 +43,14 @@ __global__ void quantize_rows_kernel(const void* __restrict__ x, int dtype, int6
 }
 
 // Split of a bf16 / fp32 query head into two e4m3 parts for the e4m3-key MMA:
-//   s = amax(q_j) / 448,  hi = e4m3(q_j / s),  lo = e4m3(16 * (q_j / s - hi)),
-//   q_j ~= s * (hi + lo / 16).
-// The residual of a round-to-nearest e4m3 code is at most half its spacing, so
-// 16x the residual stays inside the e4m3 range; the pair carries about eight
-// significant bits, the precision of the bf16 input.  Output layout
-// [rows][2][H][d] (hi block then lo block per row) and the scale s per
+//   s = amax(q_j) / 448,  hi = e4m3(q_j / s),  lo = e4m3(q_j / s - hi),
+//   q_j ~= s * (hi + lo).
+// The residual of a round-to-nearest e4m3 code is at most half its spacing and
+// is itself coded with e4m3's four significant bits (its subnormal steps of
+// 2^-9 below 2^-6), so the pair carries about eight significant bits, the
+// precision of the bf16 input.  As hi + lo is a plain sum, the scan runs the
+// two parts as two MMAs into one accumulator.  Output layout [2][rows][H][d]
+// (every row's hi part, then every row's lo part) and the scale s per
 // (row, head), which the scan folds into the head weight.
 __global__ void split_query_kernel(const void* __restrict__ q, int dtype, int64_t rows, int H,
                                    int d, uint8_t* __restrict__ parts,
@@ -56,8 +58,6 @@ __global__ void split_query_kernel(const void* __restrict__ q, int dtype, int64_
   const int64_t rh = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (rh >= rows * H) return;
-  const int64_t row = rh / H;
-  const int j = (int)(rh % H);
   const int64_t src = rh * d;
   float amax = 0.f;
   for (int c = lane; c < d; c += 32) amax = fmaxf(amax, fabsf(load_as_f32(q, dtype, src + c)));
@@ -65,14 +65,13 @@ __global__ void split_query_kernel(const void* __restrict__ q, int dtype, int64_
   for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
   const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
   if (lane == 0) head_scale[rh] = s;
-  uint8_t* hi = parts + (row * 2 * H + j) * (int64_t)d;
-  uint8_t* lo = parts + (row * 2 * H + H + j) * (int64_t)d;
+  uint8_t* hi = parts + rh * (int64_t)d;
+  uint8_t* lo = parts + (rows * H + rh) * (int64_t)d;
   for (int c = lane; c < d; c += 32) {
     const float v = __fdiv_rn(load_as_f32(q, dtype, src + c), s);
     const uint8_t ch = e4m3_rn_sat(v);
-    const float r = v - e4m3_value(ch);
     hi[c] = ch;
-    lo[c] = e4m3_rn_sat(r * 16.0f);
+    lo[c] = e4m3_rn_sat(v - e4m3_value(ch));
   }
 }
 

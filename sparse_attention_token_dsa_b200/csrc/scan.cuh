@@ -19,9 +19,10 @@
 //   warp 8     TMA producer: Q tile of the item (resident), K tiles streamed
 //              through 2-6 stages
 //   warp 9     MMA issuer (one thread) + TMEM allocator
-// MMA: M = 128 keys (TMEM lane = key), N = query rows x heads (x 2 for the
-// split-query fp8 form), K = d; fp32 accumulate in TMEM, 2-8 accumulator
-// stages so the epilogue of one unit overlaps the MMAs of the next.
+// MMA: M = 128 keys (TMEM lane = key), N = query rows x heads, K = d (the
+// split-query fp8 form issues its hi and lo query parts as two MMAs into the
+// same accumulator); fp32 accumulate in TMEM, 2-8 accumulator stages so the
+// epilogue of one unit overlaps the MMAs of the next.
 //
 // Streaming top-k.  A candidate (score, key) is kept while its composite key
 // (order-preserving score bits, then ~index) is >= the row's threshold thr.
@@ -59,7 +60,7 @@ struct ScanArgs {
   int32_t lb_shift;      // block lists: log2 tokens per listed block
   int32_t keep;          // entries each row must keep (top-k or k')
   int32_t QG;            // query rows per accumulator group (<= 256 / (H * parts))
-  int32_t qcols;         // MMA N per group: max(16, QG * H * parts) query-head columns
+  int32_t qcols;         // Q-tile rows per group: max(16, QG * H) x parts; MMA N = qcols / parts
   int32_t G;             // groups per work item (1 or 2)
   int32_t stage_cols;    // TMEM columns per accumulator stage (64, 128 or 256)
   int32_t tstages;       // accumulator stages in TMEM (2 .. 8; tstages * stage_cols <= 512)
@@ -72,7 +73,7 @@ struct ScanArgs {
   const int32_t* k_len;  // [batch] or null: n_k
   const float* w;        // [rows, H]
   const float* row_scale;   // [rows] or null: multiplies w (query dequant scale)
-  const float* head_scale;  // [rows, H] or null: multiplies w (split-query part scale)
+  const float* head_scale;  // [rows, H] or null: multiplies w (split-query scale)
   const float* k_scale;     // [batch * n_k] or null: multiplies the score (key dequant scale)
   int32_t nsub;          // sub-logs per row slot (4: one per lane quadrant; 8: one per warp)
   int32_t capw;          // entries per sub-log (>= keep + 256)
@@ -482,7 +483,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   // 1024-byte aligned base; plain pointer arithmetic on the __shared__ array
   // keeps the shared address space visible to the compiler (LDS/ATOMS, not generic)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  const int qcols = a.qcols;                                // MMA N per group
+  const int qcols = a.qcols;                                // Q-tile rows per group
   const int QT = a.QG * a.G;
   uint8_t* Qs = smem;                                       // [G][A][qcols x 128B]
   const int q_bytes = a.G * Cfg::A * qcols * 128;
@@ -546,11 +547,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         ok = mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1);
         if (ok) {
           mbar_arrive_expect_tx(&T->q_full, q_bytes);
-          const int qrow0 = (g.b * a.q_stride + a.q_off + g.row0) * a.H * PARTS;
+          // split-query rows: the hi parts of all rows come first, then the lo parts
+          const int qrow0 = (g.b * a.q_stride + a.q_off + g.row0) * a.H;
+          const int lo_rows = a.batch * a.q_stride * a.H;
+          const int part_cols = qcols / PARTS;
           for (int gg = 0; gg < a.G; ++gg)
             for (int at = 0; at < Cfg::A; ++at)
-              tma_load_2d(Qs + (gg * Cfg::A + at) * qcols * 128, &qmap, &T->q_full,
-                          at * Cfg::EPA, qrow0 + gg * a.QG * a.H * PARTS);
+              for (int pt = 0; pt < PARTS; ++pt)
+                tma_load_2d(Qs + ((gg * Cfg::A + at) * qcols + pt * part_cols) * 128, &qmap,
+                            &T->q_full, at * Cfg::EPA, qrow0 + gg * a.QG * a.H + pt * lo_rows);
         }
       }
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -621,7 +626,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA --
     if (lane == 0) {
-      const uint32_t idesc = make_idesc<KIND>(qcols);
+      // split-query rows: the hi and lo parts are two MMAs into one accumulator
+      const int ncols = qcols / PARTS;
+      const uint32_t idesc = make_idesc<KIND>(ncols);
       uint32_t kcount = 0, ucount = 0, it = 0;
       bool ok = true;
       for (int round = 0; ok; ++round) {
@@ -650,8 +657,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t ad = make_sdesc(kbase + at * 16384 + kk * 32);
-              const uint64_t bd = make_sdesc(qbase + at * qcols * 128 + kk * 32);
-              tc_mma<KIND>(d, ad, bd, idesc, (at | kk) != 0);
+#pragma unroll
+              for (int pt = 0; pt < PARTS; ++pt) {
+                const uint64_t bd = make_sdesc(qbase + (at * qcols + pt * ncols) * 128 + kk * 32);
+                tc_mma<KIND>(d, ad, bd, idesc, (at | kk | pt) != 0);
+              }
             }
           }
           tc_commit(&T->t_full[s]);
@@ -983,61 +993,18 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                          key - (int)(quad * 32 + lane) + 127 - g.kbeg < T->item_min_nleg;
           fc.hist = hist;
           fc.T = T;
-          if constexpr (SPLIT) {
-            for (int qi = 0; qi < qhalf; ++qi) {
-              const int r = rbase + qi;
-              const float* wr = &T->wsm[r * HT];
-              const uint32_t cb = taddr + (qbeg + qi) * HT * PARTS;
-              float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-              // hi / lo parts of 16 heads at a time, the next 16 in flight
-              auto part16 = [&](const uint32_t (&hi)[16], const uint32_t (&lo)[16], int c0) {
-#pragma unroll
-                for (int jj = 0; jj < 16; jj += 4) {
-                  const float4 wv = *reinterpret_cast<const float4*>(wr + c0 + jj);
-                  acc0 = fmaf(wv.x, fmaxf(fmaf(__uint_as_float(lo[jj + 0]), 0.0625f, __uint_as_float(hi[jj + 0])), 0.f), acc0);
-                  acc1 = fmaf(wv.y, fmaxf(fmaf(__uint_as_float(lo[jj + 1]), 0.0625f, __uint_as_float(hi[jj + 1])), 0.f), acc1);
-                  acc2 = fmaf(wv.z, fmaxf(fmaf(__uint_as_float(lo[jj + 2]), 0.0625f, __uint_as_float(hi[jj + 2])), 0.f), acc2);
-                  acc3 = fmaf(wv.w, fmaxf(fmaf(__uint_as_float(lo[jj + 3]), 0.0625f, __uint_as_float(hi[jj + 3])), 0.f), acc3);
-                }
-              };
-              constexpr int NCH = HT / 16;
-              uint32_t ha[16], la[16], hb[16], lb[16];
-              tmem_ld16(cb, ha);
-              tmem_ld16(cb + HT, la);
-              tmem_ld_wait(ha, la);
-#pragma unroll
-              for (int c = 0; c < NCH; c += 2) {
-                if (c + 1 < NCH) {
-                  tmem_ld16(cb + (c + 1) * 16, hb);
-                  tmem_ld16(cb + HT + (c + 1) * 16, lb);
-                }
-                part16(ha, la, c * 16);
-                if (c + 1 < NCH) {
-                  tmem_ld_wait(hb, lb);
-                  if (c + 2 < NCH) {
-                    tmem_ld16(cb + (c + 2) * 16, ha);
-                    tmem_ld16(cb + HT + (c + 2) * 16, la);
-                  }
-                  part16(hb, lb, (c + 1) * 16);
-                  if (c + 2 < NCH) tmem_ld_wait(ha, la);
-                }
-              }
-              filter_append(fc, r, (acc0 + acc1) + (acc2 + acc3));
-            }
+          if constexpr (HT >= 32) {
+            if (qhalf == 2)
+              unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+            else if (qhalf == 1)
+              unit_heads_n<HT, 1>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+            else
+              unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
           } else {
-            if constexpr (HT >= 32) {
-              if (qhalf == 2)
-                unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
-              else if (qhalf == 1)
-                unit_heads_n<HT, 1>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
-              else
-                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
-            } else {
-              if (qhalf == 8)
-                unit_heads_small<HT, 8>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
-              else
-                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
-            }
+            if (qhalf == 8)
+              unit_heads_small<HT, 8>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+            else
+              unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
           }
           tc_fence_before();
           __syncwarp();
