@@ -32,7 +32,7 @@ bool pow2_in(int v, int lo, int hi) { return v >= lo && v <= hi && (v & (v - 1))
 struct ScanPlan {
   MmaKind kind;
   bool split;
-  int parts, esz, atoms, kstages, tstages;
+  int parts, esz, atoms, kstages, tstages, kt;
   int QG, G, qcols, stage_cols, n_qt, C, chunk, n_items, keep, nsub, capw;
   int rows;
   size_t smem;
@@ -41,13 +41,15 @@ struct ScanPlan {
 
 constexpr size_t kSmemBudget = 227 * 1024;
 
-// Dynamic shared memory of the scan: alignment slack, Q tiles, K stages, then
-// the per-row histograms (streaming rows) or the candidate array (gathered rows).
-size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols, int kstages, bool gather) {
+// Dynamic shared memory of the scan: alignment slack, Q tiles, K stages of kt
+// key tiles, then the per-row histograms (streaming rows) or the candidate
+// array (gathered rows).
+size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols, int kstages, bool gather,
+                       int kt = 1) {
   const int esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   const int atoms = esz;  // d = 128
   size_t q = align_up((size_t)G * atoms * qcols * 128, 1024);
-  size_t k = (size_t)kstages * atoms * 128 * 128;
+  size_t k = (size_t)kstages * kt * atoms * 128 * 128;
   size_t h = gather ? (size_t)kMaxGatherKeys * sizeof(uint64_t) +
                           (size_t)kGatherBins * sizeof(uint32_t) +
                           (size_t)kGatherBoundary * sizeof(uint64_t)
@@ -59,15 +61,16 @@ size_t scan_smem_bytes(MmaKind kind, int G, int QG, int qcols, int kstages, bool
 // memory and TMEM; a CTA alone on its SM deepens its K pipeline into the
 // spare shared memory, and the TMEM accumulator stages fill 512 columns.
 void finish_plan(ScanPlan& pl, bool gather) {
-  pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather);
+  pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather, pl.kt);
   // 320 threads at up to 168 registers take more than half the register file:
   // one CTA per SM, whatever shared memory and TMEM would allow
   pl.ctas_per_sm = 1;
   {
     while (pl.kstages < 6 &&
-           scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages + 1, gather) <= kSmemBudget)
+           scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages + 1, gather, pl.kt) <=
+               kSmemBudget)
       ++pl.kstages;
-    pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather);
+    pl.smem = scan_smem_bytes(pl.kind, pl.G, pl.QG, pl.qcols, pl.kstages, gather, pl.kt);
   }
   pl.tstages = 512 / (pl.ctas_per_sm * pl.stage_cols);
   if (pl.tstages > kMaxTStages) pl.tstages = kMaxTStages;
@@ -102,8 +105,12 @@ ScanPlan plan_scan(MmaKind kind, bool split, int batch, int n_q, int n_k, int H,
   pl.QG = QG;
   pl.G = G;
   pl.qcols = QG * hp;
+  // one e4m3 query row per item (decode): two 128-key tiles per K stage and per
+  // accumulator hand-off, which halves the per-key count of pipeline hand-offs
+  pl.kt = (kind == MmaKind::E4M3 && G == 1 && QG == 1 && H <= 64) ? 2 : 1;
   {
-    const int n = QG * H;  // MMA N: the split-query parts share one accumulator
+    const int n = QG * H * pl.kt;  // MMA N (the split-query parts share one
+                                   // accumulator) times the key tiles of a unit
     pl.stage_cols = n > 128 ? 256 : (n > 64 ? 128 : 64);
   }
   pl.n_qt = (n_q + QG * G - 1) / (QG * G);
@@ -144,6 +151,7 @@ ScanPlan plan_gather(MmaKind kind, int batch, int n_q, int H, int keep) {
   pl.esz = kind == MmaKind::TF32 ? 4 : (kind == MmaKind::BF16 ? 2 : 1);
   pl.atoms = pl.esz;
   pl.kstages = 2;
+  pl.kt = 1;
   pl.QG = 1;
   pl.G = 1;
   pl.qcols = H < 16 ? 16 : H;
@@ -648,6 +656,7 @@ int run_stage(const dsa_problem* p, const ScanPlan& pl, const StageIO& io, int q
   a.QG = pl.QG;
   a.qcols = pl.qcols;
   a.kstages = pl.kstages;
+  a.kt = pl.kt;
   a.tstages = pl.tstages;
   a.G = pl.G;
   a.stage_cols = pl.stage_cols;
@@ -881,6 +890,7 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.QG = pl.QG;
   a.qcols = pl.qcols;
   a.kstages = pl.kstages;
+  a.kt = pl.kt;
   a.tstages = pl.tstages;
   a.G = pl.G;
   a.stage_cols = pl.stage_cols;

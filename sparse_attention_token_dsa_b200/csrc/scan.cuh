@@ -64,7 +64,9 @@ struct ScanArgs {
   int32_t G;             // groups per work item (1 or 2)
   int32_t stage_cols;    // TMEM columns per accumulator stage (64, 128 or 256)
   int32_t tstages;       // accumulator stages in TMEM (2 .. 8; tstages * stage_cols <= 512)
-  int32_t kstages;       // K-tile pipeline depth (2 .. 8)
+  int32_t kstages;       // K-stage pipeline depth (2 .. 6)
+  int32_t kt;            // 128-key tiles per K stage and accumulator unit (1 or 2; 2 only
+                         // with one query row per item, G = QG = 1)
   int32_t n_qt;          // query tiles per sequence (ceil(n_q / (QG*G)))
   int32_t C;             // key chunks per row (split-K); 1 = whole prefix
   int32_t chunk;         // keys per chunk (multiple of 128) when C > 1
@@ -488,10 +490,14 @@ __global__ void __launch_bounds__(kScanThreads, 1)
   uint8_t* Qs = smem;                                       // [G][A][qcols x 128B]
   const int q_bytes = a.G * Cfg::A * qcols * 128;
   const int KS = a.kstages, NS = a.tstages;
-  uint8_t* Ks = smem + ((q_bytes + 1023) & ~1023);          // [KS][A][128 x 128B]
+  // key tiles per K stage / accumulator unit: 2 only for e4m3 keys (decode), so
+  // every other kind compiles with a constant 1
+  constexpr bool kPairs = KIND == MmaKind::E4M3 && GATHER == 0;
+  const int KT = kPairs && a.kt > 1 ? 2 : 1;
+  uint8_t* Ks = smem + ((q_bytes + 1023) & ~1023);          // [KS][KT][A][128 x 128B]
   // streaming rows: per-row histograms [QT][768]; gathered rows: the row's
   // candidate composites [kMaxGatherKeys]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + KS * Cfg::KTILE_BYTES);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(Ks + KS * KT * Cfg::KTILE_BYTES);
   uint64_t* cand = reinterpret_cast<uint64_t*>(hist);                 // [kMaxGatherKeys]
   uint32_t* ghist = reinterpret_cast<uint32_t*>(cand + kMaxGatherKeys);  // [kGatherBins]
   uint64_t* gbnd = reinterpret_cast<uint64_t*>(ghist + kGatherBins);   // [kGatherBoundary]
@@ -564,7 +570,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const int krow0 = g.b * a.n_k;
       const int32_t* lst = GATHER != 0
           ? a.klist + ((int64_t)g.b * a.n_q + g.row0) * a.klist_len : nullptr;
-      for (int t = 0; t < g.ntiles; ++t) {
+      const int nk = (g.ntiles + KT - 1) / KT;                // K stages of this item
+      for (int t = 0; t < nk; ++t) {
         const int slot = kcount % KS;
         const uint32_t ph = (kcount / KS) & 1;
         // list entries of this tile (loaded before the wait so their latency overlaps it)
@@ -587,18 +594,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             ybox = krow0 + (blk >= 0 ? blk * bs + (e & (bs - 1)) : 0);
           }
         }
+        // tiles of this stage inside the item (a ragged last stage loads one)
+        const int nvalid = kPairs ? min(KT, g.ntiles - t * KT) : 1;
         if (lane == 0) {
           ok = mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2);
-          if (ok) mbar_arrive_expect_tx(&T->k_full[slot], Cfg::KTILE_BYTES);
+          if (ok) mbar_arrive_expect_tx(&T->k_full[slot], nvalid * Cfg::KTILE_BYTES);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if constexpr (GATHER == 0) {
           if (lane == 0) {
-            const int tstart = (g.t_hi - t) << 7;
-            for (int at = 0; at < Cfg::A; ++at)
-              tma_load_2d(Ks + (slot * Cfg::A + at) * 16384, &kmap, &T->k_full[slot],
-                          at * Cfg::EPA, krow0 + tstart);
+            for (int j = 0; j < nvalid; ++j) {
+              const int tstart = (g.t_hi - (t * KT + j)) << 7;
+              for (int at = 0; at < Cfg::A; ++at)
+                tma_load_2d(Ks + ((slot * KT + j) * Cfg::A + at) * 16384, &kmap, &T->k_full[slot],
+                            at * Cfg::EPA, krow0 + tstart);
+            }
           }
         } else if constexpr (GATHER == 1) {
           // four arbitrary key rows per copy (one-row-high boxes), 32 copies per atom
@@ -639,7 +650,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if (!mbar_wait(&T->q_full, it & 1, abort, a.status, 3)) break;
         ++it;
         tc_fence_after();
-        const int nunits = g.ntiles * a.G;
+        const int nunits = (g.ntiles + KT - 1) / KT * a.G;
         for (int u = 0; u < nunits; ++u) {
           const int gg = u & (a.G - 1);
           const int slot = kcount % KS;
@@ -649,18 +660,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const int s = ucount % NS;
           if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d = tmem_base + s * a.stage_cols;
-          const uint32_t kbase = smem_u32(Ks + slot * Cfg::A * 16384);
           const uint32_t qbase = smem_u32(Qs + gg * Cfg::A * qcols * 128);
+          // one accumulator block of ncols columns per key tile of the stage
+          const int nvalid = kPairs ? min(KT, g.ntiles - (u / a.G) * KT) : 1;
+          for (int j = 0; j < nvalid; ++j) {
+            const uint32_t d = tmem_base + s * a.stage_cols + j * ncols;
+            const uint32_t kbase = smem_u32(Ks + (slot * KT + j) * Cfg::A * 16384);
 #pragma unroll
-          for (int at = 0; at < Cfg::A; ++at) {
+            for (int at = 0; at < Cfg::A; ++at) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = make_sdesc(kbase + at * 16384 + kk * 32);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t ad = make_sdesc(kbase + at * 16384 + kk * 32);
 #pragma unroll
-              for (int pt = 0; pt < PARTS; ++pt) {
-                const uint64_t bd = make_sdesc(qbase + (at * qcols + pt * ncols) * 128 + kk * 32);
-                tc_mma<KIND>(d, ad, bd, idesc, (at | kk | pt) != 0);
+                for (int pt = 0; pt < PARTS; ++pt) {
+                  const uint64_t bd = make_sdesc(qbase + (at * qcols + pt * ncols) * 128 + kk * 32);
+                  tc_mma<KIND>(d, ad, bd, idesc, (at | kk | pt) != 0);
+                }
               }
             }
           }
@@ -946,15 +961,24 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       }
       if (etid == 0) T->raise_any = 0;
       named_bar_sync(kBarEpi, kEpiThreads);
-      const int nunits = g.ntiles * a.G;
+      const int nunits = (g.ntiles + KT - 1) / KT * a.G;
       auto ks_at = [&](int uu) -> float {
         if (!a.k_scale) return 1.f;
-        const int key = ((g.t_hi - (uu >> (a.G - 1))) << 7) + quad * 32 + lane;
+        const int key = ((g.t_hi - (uu >> (a.G - 1)) * KT) << 7) + quad * 32 + lane;
         return key < a.n_k ? a.k_scale[(int64_t)g.b * a.n_k + key] : 1.f;
+      };
+      // scale of the second key tile of a unit (below the first; may precede the
+      // item's first tile in a ragged last unit)
+      auto ks_at1 = [&](int uu) -> float {
+        if (!a.k_scale) return 1.f;
+        const int key = ((g.t_hi - (uu >> (a.G - 1)) * KT - 1) << 7) + quad * 32 + lane;
+        return key >= 0 && key < a.n_k ? a.k_scale[(int64_t)g.b * a.n_k + key] : 1.f;
       };
       const int ustep = modeB ? 2 : 1;                  // this warp's units: every / every other
       const int ufirst = modeB ? (int)((ucount + half) & 1) : 0;
       float ks_next = ufirst < nunits ? ks_at(ufirst) : 1.f;
+      float ks_next1 = 1.f;
+      if constexpr (kPairs) ks_next1 = ufirst < nunits && KT > 1 ? ks_at1(ufirst) : 1.f;
       int u = 0;
       int steps = 0;
       while (u < nunits) {
@@ -968,10 +992,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           if (!mine) continue;
           const int gg = uu & (a.G - 1);
           const int t = uu >> (a.G - 1);
-          const int key = ((g.t_hi - t) << 7) + quad * 32 + lane;
+          const int key = ((g.t_hi - t * KT) << 7) + quad * 32 + lane;
           // key dequant scale: loaded one unit of this warp ahead
           const float ks = ks_next;
           if (uu + ustep < nunits) ks_next = ks_at(uu + ustep);
+          float ks1 = 1.f;
+          if constexpr (kPairs) {
+            ks1 = ks_next1;
+            if (KT > 1 && uu + ustep < nunits) ks_next1 = ks_at1(uu + ustep);
+          }
           const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
@@ -1005,6 +1034,22 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               unit_heads_small<HT, 8>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
             else
               unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+          }
+          if constexpr (kPairs) {
+            // the unit's second key tile (one query row per item: mode B, qhalf 1),
+            // in the next ncols accumulator columns; absent in a ragged last unit
+            if (KT > 1 && t * KT + 1 < g.ntiles) {
+              const int key1 = key - 128;
+              fc.key = key1;
+              fc.ks = ks1;
+              fc.all_legal = key1 - (int)(quad * 32 + lane) >= g.kbeg &&
+                             key1 - (int)(quad * 32 + lane) + 127 - g.kbeg < T->item_min_nleg;
+              const uint32_t tcol = taddr + qcols / PARTS;
+              if constexpr (HT >= 32)
+                unit_heads_n<HT, 1>(fc, tcol, &T->wsm[rbase * HT], rbase);
+              else
+                unit_heads<HT>(fc, tcol, &T->wsm[rbase * HT], 1, rbase);
+            }
           }
           tc_fence_before();
           __syncwarp();

@@ -203,6 +203,27 @@ def test_fp8_decode_split_query(B, batch, n_k):
     assert iou > 0.9
 
 
+@pytest.mark.parametrize("batch,n_k", [(5, 9000), (3, 3001), (2, 200)])
+def test_integer_e4m3_decode_bit_exact(B, batch, n_k):
+    """Decode with e4m3 q and k holding small integers (exact codes, unit scales):
+    the split-K scan and merge are bit-exact.  Ragged prefixes give key chunks
+    with odd tile counts, so a pipeline unit of two key tiles ends half full."""
+    k_len = [n_k - 131 * b for b in range(batch)]
+    p = gen.integer_problem(40 + batch, batch, 1, n_k, 64, 128, 2048,
+                            q_pos0=[n - 1 for n in k_len], k_len=k_len)
+    qc = oracle.e4m3_encode(p.q)
+    kc = oracle.e4m3_encode(p.k)
+    assert np.array_equal(oracle.e4m3_decode(qc), p.q) and np.array_equal(oracle.e4m3_decode(kc), p.k)
+    qs = np.ones((batch, 1), np.float32)
+    ks = np.ones((batch, n_k), np.float32)
+    gi, gs = run_dsa(B, p, q=dev(qc), k=dev(kc), q_scale=dev(qs), k_scale=dev(ks),
+                     flags=B.DSA_FLAG_CHECK)
+    inq = oracle.Inputs(p, q=qc, k=kc, q_dtype=gen.E4M3, k_dtype=gen.E4M3, q_scale=qs,
+                        k_scale=ks)
+    ri, rs, _, _ = oracle.dsa(inq, p.topk)
+    parity.exact(gi, gs, ri, rs)
+
+
 def test_fp8_decode_full_size(B):
     """32 sequences x 131072 cached keys, H = 64, k = 2048 (every row checked)."""
     p, _ = gen.decode_problem(3, 32, 131072, 64, 128, 2048)
