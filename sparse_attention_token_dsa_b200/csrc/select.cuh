@@ -177,29 +177,6 @@ __device__ int compact_ge(const uint64_t* const* seg, const int* seg_n, int nseg
   return n;
 }
 
-// In-place descending bitonic sort of n <= cap keys in shared memory (cap a
-// power of two; slots [n, cap) are filled with 0, the smallest key).
-template <int NTHR>
-__device__ void bitonic_sort_desc(uint64_t* a, int n, int cap, int tid, int bar_id) {
-  for (int i = n + tid; i < cap; i += NTHR) a[i] = 0ull;
-  named_bar_sync(bar_id, NTHR);
-  for (int size = 2; size <= cap; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < cap / 2; i += NTHR) {
-        int lo = 2 * i - (i & (stride - 1));
-        int hi = lo + stride;
-        bool desc = ((lo & size) == 0);
-        uint64_t x = a[lo], y = a[hi];
-        if ((x < y) == desc) {
-          a[lo] = y;
-          a[hi] = x;
-        }
-      }
-      named_bar_sync(bar_id, NTHR);
-    }
-  }
-}
-
 // Descending bitonic sort of N = NT * E keys held E per thread in registers
 // (thread t holds positions t*E .. t*E+E-1).  Strides below E compare inside a
 // thread, strides below 32*E across lanes with shuffles, and only strides of
