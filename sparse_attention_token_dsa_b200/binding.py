@@ -97,6 +97,37 @@ def _ptr(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+_OPERAND = (torch.float32, torch.bfloat16, torch.uint8, torch.float8_e4m3fn)
+_F32 = (torch.float32,)
+_I32 = (torch.int32,)
+_U8 = (torch.uint8,)
+
+
+def _args(**named):
+    """Check tensor arguments before any library call: dtype, C-contiguous
+    layout and a CUDA device (the kernels take raw device pointers, so a host or
+    strided tensor would be misread).  Each value is (tensor or None, dtypes)."""
+    given = [(name, t, dtypes) for name, (t, dtypes) in named.items() if t is not None]
+    for name, t, dtypes in given:
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+        if t.dtype not in dtypes:
+            raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+    for name, t, _ in given:
+        if t.device.type != "cuda":
+            raise ValueError(f"{name}: must be on a CUDA device, not {t.device}")
+
+
+def _common_args(q, k, w, q_scale=None, k_scale=None, q_pos0=None, k_len=None, out=None,
+                 workspace=None, **extra):
+    idx, sc = (None, None) if out is None else out
+    _args(q=(q, _OPERAND), k=(k, _OPERAND), w=(w, _F32), q_scale=(q_scale, _F32),
+          k_scale=(k_scale, _F32), q_pos0=(q_pos0, _I32), k_len=(k_len, _I32),
+          out_idx=(idx, _I32), out_score=(sc, _F32), workspace=(workspace, _U8), **extra)
+
+
 def _stream(stream):
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -147,6 +178,7 @@ def _outputs(B, nq, topk, device, out):
 def dsa_index(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_len=None, flags=0,
               out=None, workspace=None, stream=None):
     """DSA indexer top-k.  Returns (idx int32 [B,n_q,k], score fp32 [B,n_q,k])."""
+    _common_args(q, k, w, q_scale, k_scale, q_pos0, k_len, out, workspace)
     p = problem(q, k, topk, q_pos0, k_len, flags)
     ws = _workspace(dsa_workspace_size(p), q.device, workspace)
     idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
@@ -162,6 +194,7 @@ def dsa_index_noalloc(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_
     For callers that cannot allocate device memory at call time; problems that
     need more than the library's 64 MiB scratch raise DsaError(DSA_ERR_WORKSPACE),
     and calls that overlap on the GPU race on the shared scratch."""
+    _common_args(q, k, w, q_scale, k_scale, q_pos0, k_len, out)
     p = problem(q, k, topk, q_pos0, k_len, flags)
     idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
     _check(lib.dsa_index_noalloc(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale),
@@ -172,18 +205,22 @@ def dsa_index_noalloc(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_
 
 def dsa_index_scan(p: DsaProblem, q, k, w, workspace, q_scale=None, k_scale=None, stream=None):
     """First stage of dsa_index (scores + candidate logs in `workspace`)."""
+    _common_args(q, k, w, q_scale, k_scale, workspace=workspace)
     _check(lib.dsa_index_scan(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale), _ptr(w),
                               _ptr(workspace), workspace.numel(), _stream(stream)), "dsa_index_scan")
 
 
 def dsa_index_select(p: DsaProblem, idx, score, workspace, stream=None):
     """Second stage of dsa_index (exact top-k per row from the logs)."""
+    _args(idx=(idx, _I32), score=(score, _F32), workspace=(workspace, _U8))
     _check(lib.dsa_index_select(C.byref(p), _ptr(idx), _ptr(score), _ptr(workspace),
                                 workspace.numel(), _stream(stream)), "dsa_index_select")
 
 
 def misa_index(q, k, w, topk, block, h, q_pos0=None, k_len=None, flags=0, out=None,
                out_heads=None, out_E=None, workspace=None, stream=None):
+    _common_args(q, k, w, None, None, q_pos0, k_len, out, workspace,
+                 out_heads=(out_heads, _I32), out_E=(out_E, _F32))
     p = problem(q, k, topk, q_pos0, k_len, flags)
     rp = route_params(misa_block=block, misa_h=h)
     ws = _workspace(dsa_workspace_size(p, DSA_ALGO_MISA, rp), q.device, workspace)
@@ -196,6 +233,8 @@ def misa_index(q, k, w, topk, block, h, q_pos0=None, k_len=None, flags=0, out=No
 
 def misa_dagger_index(q, k, w, topk, block, h, k_prime, q_pos0=None, k_len=None, flags=0,
                       out=None, out_heads=None, out_pool=None, workspace=None, stream=None):
+    _common_args(q, k, w, None, None, q_pos0, k_len, out, workspace,
+                 out_heads=(out_heads, _I32), out_pool=(out_pool, _I32))
     p = problem(q, k, topk, q_pos0, k_len, flags)
     rp = route_params(misa_block=block, misa_h=h, k_prime=k_prime)
     ws = _workspace(dsa_workspace_size(p, DSA_ALGO_MISA_DAGGER, rp), q.device, workspace)
@@ -208,6 +247,8 @@ def misa_dagger_index(q, k, w, topk, block, h, k_prime, q_pos0=None, k_len=None,
 
 def hisa_index(q, k, w, topk, block, r, route_h=0, route_block=1024, q_pos0=None, k_len=None,
                flags=0, out=None, out_blocks=None, out_heads=None, workspace=None, stream=None):
+    _common_args(q, k, w, None, None, q_pos0, k_len, out, workspace,
+                 out_blocks=(out_blocks, _I32), out_heads=(out_heads, _I32))
     p = problem(q, k, topk, q_pos0, k_len, flags)
     rp = route_params(misa_block=route_block if route_h else 0, misa_h=route_h, hisa_block=block,
                       hisa_r=r)
@@ -221,6 +262,7 @@ def hisa_index(q, k, w, topk, block, r, route_h=0, route_block=1024, q_pos0=None
 
 def dsa_quantize_e4m3(x: torch.Tensor, stream=None):
     """Per-row e4m3 codes (uint8, same shape) and fp32 scales (shape[:-1])."""
+    _args(x=(x, (torch.float32, torch.bfloat16)))
     cols = x.shape[-1]
     rows = x.numel() // cols
     out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
@@ -231,4 +273,5 @@ def dsa_quantize_e4m3(x: torch.Tensor, stream=None):
 
 
 def dsa_read_status(workspace: torch.Tensor, stream=None) -> int:
+    _args(workspace=(workspace, _U8))
     return lib.dsa_read_status(_ptr(workspace), _stream(stream))

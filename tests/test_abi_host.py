@@ -160,3 +160,35 @@ def test_route_entry_points_reject_before_launch(bind):
                                fake, 1 << 40, None) == -1
     assert L.hisa_index(C.byref(p), C.byref(rp), fake, fake, fake, fake, fake, None, None, None,
                         0, None) == -3
+
+
+def test_binding_checks_tensors_before_any_call(bind):
+    """The Python binding refuses host, strided or mistyped tensors itself: the
+    library takes raw device pointers and could not tell."""
+    import torch
+    q = torch.zeros((1, 4, 8, 128), dtype=torch.bfloat16)
+    k = torch.zeros((1, 16, 128), dtype=torch.bfloat16)
+    w = torch.zeros((1, 4, 8), dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA device"):
+        bind.dsa_index(q, k, w, 4)
+    with pytest.raises(TypeError, match="w: dtype"):
+        bind.dsa_index(q, k, w.double(), 4)
+    with pytest.raises(ValueError, match="q: must be contiguous"):
+        bind.dsa_index(q.transpose(2, 3), k, w, 4)
+    with pytest.raises(TypeError, match="k_len: dtype"):
+        bind.dsa_index(q, k, w, 4, k_len=torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(TypeError, match="q: dtype"):
+        bind.dsa_index(q.half(), k, w, 4)
+    with pytest.raises(TypeError, match="out_score: dtype"):
+        bind.dsa_index(q, k, w, 4, out=(torch.zeros((1, 4, 4), dtype=torch.int32),
+                                        torch.zeros((1, 4, 4), dtype=torch.float64)))
+    with pytest.raises(ValueError, match="CUDA device"):
+        bind.misa_index(q, k, w, 4, 16, 8)
+    with pytest.raises(TypeError, match="out_pool: dtype"):
+        bind.misa_dagger_index(q, k, w, 4, 16, 8, 8, out_pool=torch.zeros(1, dtype=torch.int64))
+    with pytest.raises(ValueError, match="CUDA device"):
+        bind.hisa_index(q, k, w, 4, 16, 2)
+    with pytest.raises(ValueError, match="CUDA device"):
+        bind.dsa_quantize_e4m3(k)
+    with pytest.raises(TypeError, match="workspace: dtype"):
+        bind.dsa_read_status(torch.zeros(4, dtype=torch.int32))
