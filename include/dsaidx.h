@@ -55,6 +55,10 @@
  *     DSA_FLAG_CHECK is set.  Calls are asynchronous on `stream` (a
  *     cudaStream_t passed as void*; NULL = the legacy default stream).  Two
  *     calls in flight at once need two distinct workspaces.
+ *   - Alignment.  q, k and the workspace start on 16-byte boundaries (the scan
+ *     reads q, k and buffers inside the workspace with TMA copies); every other
+ *     array is aligned to its element size.  A misaligned q, k or workspace
+ *     returns DSA_ERR_INVALID before any launch.
  *   - Errors.  Every call returns DSA_OK (0) or a negative status; nothing is
  *     thrown across the ABI.  Argument errors are detected on the host before
  *     any launch.  A bounded device wait that expires (DSA_ERR_TIMEOUT) or a

@@ -768,6 +768,7 @@ int route_begin(const dsa_problem* p, int algo, const dsa_route_params* rp, cons
   if (!aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID;
   *L = route_layout(p, c);
   if (!ws || ws_bytes < L->total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(ws)) return DSA_ERR_INVALID;
   uint8_t* w8 = reinterpret_cast<uint8_t*>(ws);
   if (cudaMemsetAsync(w8, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
   if (p->flags & DSA_FLAG_CHECK)
@@ -843,6 +844,7 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   if (p->k_dtype == DSA_E4M3 && !k_scale) return DSA_ERR_INVALID;
   const DsaLayout L = dsa_layout(p);
   if (!workspace || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_INVALID;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   int32_t* status = reinterpret_cast<int32_t*>(ws);
@@ -921,6 +923,7 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
   if (!out_idx || !out_score) return DSA_ERR_INVALID;
   const DsaLayout L = dsa_layout(p);
   if (!workspace || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_INVALID;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   const ScanPlan& pl = L.pl;

@@ -81,6 +81,8 @@ def test_dsa_index_rejects_before_launch(bind):
              None) == -1                                           # misaligned q
     assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, None, 0, None) == -3
     assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, fake, 16, None) == -3
+    assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, C.c_void_p(0x1008), 1 << 30,
+             None) == -1                                           # misaligned workspace
     e4 = _prob(bind, q_dtype=2, k_dtype=2)
     assert f(C.byref(e4), fake, None, fake, None, fake, fake, fake, fake, 1 << 30, None) == -1
 
@@ -160,6 +162,8 @@ def test_route_entry_points_reject_before_launch(bind):
                                fake, 1 << 40, None) == -1
     assert L.hisa_index(C.byref(p), C.byref(rp), fake, fake, fake, fake, fake, None, None, None,
                         0, None) == -3
+    assert L.hisa_index(C.byref(p), C.byref(rp), fake, fake, fake, fake, fake, None, None,
+                        C.c_void_p(0x1008), 1 << 40, None) == -1   # misaligned workspace
 
 
 def test_binding_checks_tensors_before_any_call(bind):
