@@ -179,6 +179,14 @@ def algorithmic_work(p, w=None):
     return int(n.sum()), dots, 2.0 * dots * p.dim
 
 
+def decode_bytes(p):
+    """Algorithmic HBM bytes of one decode scan: every cached key's e4m3 code row
+    (d bytes) and fp32 scale, plus the bf16 query and fp32 weights of each row."""
+    kbytes = p.batch * p.n_k * (p.dim + 4)
+    qbytes = p.batch * p.n_q * p.heads * (p.dim * 2 + 4)
+    return kbytes + qbytes
+
+
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
 
@@ -560,12 +568,11 @@ def main():
         bf16_peak = pk["bf16_sustained"] if long_region else pk["bf16"]
         burst = "sustained" if long_region else "burst"
         if kind == "decode":
-            kbytes = p.batch * p.n_k * (128 + 4)
-            qbytes = p.batch * p.heads * 128 * 2 + p.batch * p.heads * 4
-            gbs = (kbytes + qbytes) / (stage_ms * 1e-3) / 1e9
+            nbytes = decode_bytes(p)
+            gbs = nbytes / (stage_ms * 1e-3) / 1e9
             roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
                     "frac": gbs / pk["hbm"], "peak_source": f"{pk['src']} copy bandwidth",
-                    "work": f"{(kbytes + qbytes) / 1e6:.1f} MB per launch (e4m3 K + scales + q + w)",
+                    "work": f"{nbytes / 1e6:.1f} MB per launch (e4m3 K + scales + q + w)",
                     "kernel": "scan_kernel", "kernel_ms": stage_ms}
         elif kind == "prefill":
             tf = flops / (stage_ms * 1e-3) / 1e12
