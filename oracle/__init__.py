@@ -14,7 +14,11 @@ import numpy as np
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "dsa_oracle.c")
-LIB = os.path.join(HERE, "libdsa_oracle.so")
+# DSA_ORACLE_MUTANT=n builds and loads the oracle with planted mistake n (see
+# the ORC_MUTANT switches in dsa_oracle.c); only tests/test_oracle_mutants.py
+# sets it, to check that the pins reject every such mistake.
+MUTANT = int(os.environ.get("DSA_ORACLE_MUTANT", "0"))
+LIB = os.path.join(HERE, "libdsa_oracle.so" if MUTANT == 0 else f"libdsa_oracle_m{MUTANT}.so")
 
 F32, BF16, E4M3 = 0, 1, 2
 
@@ -24,7 +28,8 @@ def build(force: bool = False) -> str:
     if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
         tmp = LIB + f".tmp{os.getpid()}"
         subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off",
-                               "-fno-fast-math", "-shared", "-fPIC", SRC, "-o", tmp, "-lm"])
+                               "-fno-fast-math", f"-DORC_MUTANT={MUTANT}", "-shared", "-fPIC",
+                               SRC, "-o", tmp, "-lm"])
         os.replace(tmp, LIB)
     return LIB
 

@@ -54,6 +54,15 @@
 #include <stdlib.h>
 #include <string.h>
 
+/* Planted mistakes for the pin tests (tests/test_oracle_mutants.py): a build
+ * with -DORC_MUTANT=n changes one step below; the default build (0) has none.
+ * Each mutant is a plausible slip in writing the definitions down, and the pin
+ * suite must reject every one of them. */
+#ifndef ORC_MUTANT
+#define ORC_MUTANT 0
+#endif
+#define MUT(n) (ORC_MUTANT == (n))
+
 enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2 };
 enum { ORC_OK = 0, ORC_ERR = -1 };
 
@@ -78,7 +87,7 @@ double orc_e4m3_decode(uint8_t c) {
   double v;
   if (e == 15 && m == 7) return NAN;
   if (e == 0)
-    v = ldexp((double)m, -9);
+    v = ldexp((double)m, MUT(13) ? -10 : -9);
   else
     v = ldexp((double)(8 + m), e - 10);
   return sign ? -v : v;
@@ -105,7 +114,7 @@ uint8_t orc_e4m3_encode(float x) {
   double fl = floor(n);
   double r = n - fl;
   double m_int = fl;
-  if (r > 0.5 || (r == 0.5 && fmod(fl, 2.0) != 0.0)) m_int = fl + 1.0;
+  if (r > 0.5 || (r == 0.5 && (MUT(10) || fmod(fl, 2.0) != 0.0))) m_int = fl + 1.0;
   double q = m_int * ulp; /* rounded magnitude */
   if (q >= 448.0) return sign | 0x7E;
   if (q == 0.0) return sign;
@@ -139,7 +148,7 @@ int orc_quantize_rows(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
       float av = fabsf(v);
       if (av > amax) amax = av;
     }
-    volatile float a = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+    volatile float a = (amax > 0.0f) ? amax / (MUT(14) ? 240.0f : 448.0f) : 1.0f;
     out_scale[r] = a;
     for (int32_t c = 0; c < cols; ++c) {
       float v;
@@ -181,7 +190,8 @@ static double bf16_value(uint16_t b) {
 }
 
 static double q_val(const orc_inputs* in, int64_t row, int32_t j, int32_t c) {
-  int64_t off = (row * in->heads + j) * (int64_t)in->dim + c;
+  int64_t off = MUT(11) ? (row * in->dim + c) * (int64_t)in->heads + j
+                        : (row * in->heads + j) * (int64_t)in->dim + c;
   switch (in->q_dtype) {
     case ORC_F32: return (double)((const float*)in->q)[off];
     case ORC_BF16: return bf16_value(((const uint16_t*)in->q)[off]);
@@ -208,8 +218,8 @@ static int32_t row_pos(const orc_inputs* in, int64_t row) {
 /* Number of legal keys of a row: s <= pos and s < k_len. */
 static int64_t row_legal(const orc_inputs* in, int64_t row) {
   int32_t b = (int32_t)(row / in->n_q);
-  int64_t kl = in->k_len ? in->k_len[b] : in->n_k;
-  int64_t n = (int64_t)row_pos(in, row) + 1;
+  int64_t kl = (in->k_len && !MUT(5)) ? in->k_len[b] : in->n_k;
+  int64_t n = (int64_t)row_pos(in, row) + (MUT(3) ? 0 : 1);
   if (n > kl) n = kl;
   return n < 0 ? 0 : n;
 }
@@ -233,8 +243,8 @@ static double score_heads(const orc_inputs* in, int64_t row, int64_t s, const in
   for (int32_t a = 0; a < nh; ++a) {
     int32_t j = heads[a];
     double z = 0.0;
-    for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * kd[c];
-    total += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+    for (int32_t c = 0; c < in->dim - (MUT(12) ? 1 : 0); ++c) z += q_val(in, row, j, c) * kd[c];
+    total += (MUT(4) ? 1.0 : (double)in->w[row * in->heads + j]) * (MUT(1) ? z : (z > 0.0 ? z : 0.0));
   }
   free(kd);
   return total;
@@ -270,8 +280,8 @@ static double score_cached(const orc_inputs* in, row_cache* rc, int64_t row, int
     int32_t j = heads[a];
     const double* qj = rc->q + (size_t)j * in->dim;
     double z = 0.0;
-    for (int32_t c = 0; c < in->dim; ++c) z += qj[c] * rc->kd[c];
-    total += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+    for (int32_t c = 0; c < in->dim - (MUT(12) ? 1 : 0); ++c) z += qj[c] * rc->kd[c];
+    total += (MUT(4) ? 1.0 : (double)in->w[row * in->heads + j]) * (MUT(1) ? z : (z > 0.0 ? z : 0.0));
   }
   return total;
 }
@@ -289,6 +299,7 @@ static int by_value_then_index(const void* a, const void* b) {
   const ranked* y = (const ranked*)b;
   if (x->v > y->v) return -1;
   if (x->v < y->v) return 1;
+  if (MUT(2)) return (x->i < y->i) - (x->i > y->i);
   return (x->i > y->i) - (x->i < y->i);
 }
 
@@ -306,7 +317,7 @@ static void emit_topk(const ranked* r, int64_t n, int32_t topk, int32_t* idx, fl
       sc[a] = to_output_score(r[a].v);
       if (sc64) sc64[a] = r[a].v;
     } else {
-      idx[a] = -1;
+      idx[a] = MUT(15) ? 0 : -1;
       sc[a] = -INFINITY;
       if (sc64) sc64[a] = -INFINITY;
     }
@@ -389,12 +400,13 @@ int orc_abs_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t
 
 /* Mean of key rows [lo, hi) of sequence b, rounded once to the key storage
  * type (bf16 or fp32).  [MISA] step 1 / [HISA] block representatives. */
-static void pooled_key(const orc_inputs* in, int32_t b, int64_t lo, int64_t hi, double* out) {
+static void pooled_key(const orc_inputs* in, int32_t b, int64_t lo, int64_t hi, int32_t blk,
+                       double* out) {
   for (int32_t c = 0; c < in->dim; ++c) {
     double sum = 0.0;
     for (int64_t s = lo; s < hi; ++s) sum += k_val(in, b, s, c);
-    double mean = sum / (double)(hi - lo);
-    out[c] = (in->k_dtype == ORC_BF16) ? round_to_bf16(mean) : (double)(float)mean;
+    double mean = sum / (double)(MUT(6) ? blk : hi - lo);
+    out[c] = MUT(16) ? mean : (in->k_dtype == ORC_BF16) ? round_to_bf16(mean) : (double)(float)mean;
   }
 }
 
@@ -405,7 +417,8 @@ static double* block_representatives(const orc_inputs* in, int32_t b, int64_t n,
   double* reps = (double*)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1) * in->dim);
   for (int64_t a = 0; a < m; ++a) {
     int64_t lo = a * blk, hi = lo + blk < n ? lo + blk : n;
-    pooled_key(in, b, lo, hi, reps + a * in->dim);
+    if (MUT(17)) hi = lo + blk < in->n_k ? lo + blk : in->n_k;
+    pooled_key(in, b, lo, hi, blk, reps + a * in->dim);
   }
   *n_blocks = m;
   return reps;
@@ -431,16 +444,18 @@ static void misa_route(const orc_inputs* in, int64_t row, int32_t blk, int32_t h
   ranked* order = (ranked*)malloc(sizeof(ranked) * in->heads);
   for (int32_t j = 0; j < in->heads; ++j) {
     double s = 0.0;
-    double aw = fabs((double)in->w[row * in->heads + j]);
+    double aw = MUT(7) ? (double)in->w[row * in->heads + j] : fabs((double)in->w[row * in->heads + j]);
     for (int64_t a = 0; a < m; ++a) {
       double z = dot_q_vec(in, row, j, reps + a * in->dim);
       s += aw * (z > 0.0 ? z : 0.0);
     }
     S[j] = s;
     order[j].v = s;
-    order[j].i = j;
+    order[j].i = MUT(8) ? in->heads - 1 - j : j;
   }
   qsort(order, (size_t)in->heads, sizeof(ranked), by_value_then_index);
+  if (MUT(8))
+    for (int32_t j = 0; j < in->heads; ++j) order[j].i = in->heads - 1 - order[j].i;
   /* ascending head order of the selected set */
   char* chosen = (char*)calloc((size_t)in->heads, 1);
   for (int32_t a = 0; a < h; ++a) chosen[order[a].i] = 1;
@@ -501,7 +516,7 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
                 out_score64 ? out_score64 + r * topk : NULL);
     } else {
       /* MISA-dagger: keep k' by the routed score, rerank with all heads */
-      int64_t np = n < k_prime ? n : k_prime;
+      int64_t np = n < k_prime ? n : k_prime - (MUT(18) ? 1 : 0);
       ranked* pool = (ranked*)malloc(sizeof(ranked) * (np > 0 ? np : 1));
       int64_t cnt = 0;
       if (forced_pool) {
@@ -579,14 +594,14 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
       for (int32_t x = 0; x < nh; ++x) {
         int32_t j = heads[x];
         double z = dot_q_vec(in, row, j, reps + a * in->dim);
-        J += (double)in->w[row * in->heads + j] * (z > 0.0 ? z : 0.0);
+        J += (MUT(9) ? 1.0 : (double)in->w[row * in->heads + j]) * (z > 0.0 ? z : 0.0);
       }
       bl[a].v = J;
       bl[a].i = a;
     }
     dots += (int64_t)nh * mb;
     qsort(bl, (size_t)mb, sizeof(ranked), by_value_then_index);
-    int64_t kept = mb < r_keep ? mb : r_keep;
+    int64_t kept = mb < r_keep ? mb : r_keep - (MUT(19) ? 1 : 0);
     char* keep = (char*)calloc((size_t)(mb > 0 ? mb : 1), 1);
     if (forced_blocks) {
       kept = 0;
@@ -608,9 +623,15 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
     ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
     int64_t nc = 0;
     row_cache rc = row_cache_new(in, row);
+    int32_t* allh = NULL;
+    if (MUT(20)) {
+      allh = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+      for (int32_t j = 0; j < in->heads; ++j) allh[j] = j;
+    }
     for (int64_t s = 0; s < n; ++s) {
       if (!keep[s / blk]) continue;
-      cand[nc].v = score_cached(in, &rc, row, s, heads, nh);
+      cand[nc].v = MUT(20) ? score_cached(in, &rc, row, s, allh, in->heads)
+                           : score_cached(in, &rc, row, s, heads, nh);
       cand[nc].i = s;
       ++nc;
     }
@@ -620,6 +641,7 @@ int orc_hisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_kee
               out_score64 ? out_score64 + r * topk : NULL);
     if (out_dots) out_dots[r] = dots;
     row_cache_free(&rc);
+    free(allh);
     free(cand);
     free(keep);
     free(bl);

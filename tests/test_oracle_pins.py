@@ -237,6 +237,43 @@ def test_pool_ramp_mean_closed_form(oracle_mod):
         assert np.all(reps[b, 1:] == 0.0)
 
 
+def test_pool_rounds_the_mean_once_to_the_key_type(oracle_mod):
+    """A representative is the exact block mean, rounded once (to nearest even)
+    to the key storage type: bf16 keys 1 and 1 + 2^-7 average to 1 + 2^-8, a
+    tie between bf16 neighbours that rounds to 1; 1 and 1 + 3 * 2^-7 average to
+    1 + 1.5 * 2^-7, a tie that rounds up to the even 1 + 2^-6.  fp32 keys 1 and
+    1 + 2^-23 average to a tie that rounds to 1."""
+    d = 2
+    k = np.array([[[1.0, 1.0], [1.0 + 2**-7, 1.0 + 3 * 2**-7]]], np.float32)
+    p = make(np.zeros((1, 1, 8, d)), k, np.ones((1, 1, 8)), 1, dtype=BF16)
+    reps = oracle_mod.pool(oracle_mod.Inputs(p), 0, 2, 2)
+    assert reps[0, 0] == 1.0 and reps[0, 1] == 1.0 + 2**-6
+    k = np.array([[[1.0, 3.0], [1.0 + 2**-23, 3.0]]], np.float32)
+    p = make(np.zeros((1, 1, 8, d)), k, np.ones((1, 1, 8)), 1)
+    reps = oracle_mod.pool(oracle_mod.Inputs(p), 0, 2, 2)
+    assert reps[0, 0] == 1.0 and reps[0, 1] == 3.0
+
+
+def test_stacked_hisa_reranks_with_the_routed_heads(oracle_mod):
+    """Stacked MISA + HISA, closed form (d = 2, two heads, h = 1): the router
+    keeps head 0, so the rerank scores only w_0 ReLU(q_0 . k_s).
+
+    q_0 = (10, 0), q_1 = (0, 1), w = (1, 1); keys (1, 0), (0, 5), (1, 0),
+    (0.1, 0); the query sits at position 3.  Router blocks of 2: means
+    (0.5, 2.5) and (0.55, 0) give S_0 = 10.5 > S_1 = 2.5.  HISA with blocks of
+    one token keeping all four: routed scores 10, 0, 10, 1, so the top 3 are
+    tokens 0, 2, 3 with 10, 10, 1 (all heads would give 10, 5, 10, 1 and pick
+    token 1 instead of 3)."""
+    q = np.array([[[[10.0, 0.0], [0.0, 1.0]]]], np.float32)
+    k = np.array([[[1.0, 0.0], [0.0, 5.0], [1.0, 0.0], [0.1, 0.0]]], np.float32)
+    w = np.ones((1, 1, 2), np.float32)
+    p = make(q, k, w, 3, q_pos0=[3])
+    out = oracle_mod.hisa(oracle_mod.Inputs(p), 3, block=1, r=4, route_h=1, route_block=2)
+    assert out["heads"].tolist() == [[0]]
+    assert out["idx"].tolist() == [[0, 2, 3]]
+    assert out["score64"][0].tolist() == [10.0, 10.0, float(np.float32(0.1)) * 10.0]
+
+
 def test_router_closed_form_constant_keys(oracle_mod):
     """All keys = v => every representative = v, S_j = M |w_j| max(q_j.v, 0)."""
     d, H, nk, blk = 4, 8, 50, 16
