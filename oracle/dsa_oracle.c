@@ -114,7 +114,7 @@ uint8_t orc_e4m3_encode(float x) {
   double fl = floor(n);
   double r = n - fl;
   double m_int = fl;
-  if (r > 0.5 || (r == 0.5 && (MUT(10) || fmod(fl, 2.0) != 0.0))) m_int = fl + 1.0;
+  if (!MUT(26) && (r > 0.5 || (r == 0.5 && (MUT(10) || fmod(fl, 2.0) != 0.0)))) m_int = fl + 1.0;
   double q = m_int * ulp; /* rounded magnitude */
   if (q >= 448.0) return sign | 0x7E;
   if (q == 0.0) return sign;
@@ -183,7 +183,7 @@ static double round_to_bf16(double x) {
 /* ------------------------------------------------------------- operands -- */
 
 static double bf16_value(uint16_t b) {
-  uint32_t u = (uint32_t)b << 16;
+  uint32_t u = (uint32_t)b << (MUT(25) ? 15 : 16);
   float f;
   memcpy(&f, &u, 4);
   return (double)f;
@@ -211,7 +211,7 @@ static double k_val(const orc_inputs* in, int32_t b, int64_t s, int32_t c) {
 
 static int32_t row_pos(const orc_inputs* in, int64_t row) {
   int32_t b = (int32_t)(row / in->n_q), i = (int32_t)(row % in->n_q);
-  int32_t p0 = in->q_pos0 ? in->q_pos0[b] : in->n_k - in->n_q;
+  int32_t p0 = in->q_pos0 ? in->q_pos0[b] : (MUT(21) ? 0 : in->n_k - in->n_q);
   return p0 + i;
 }
 
@@ -501,12 +501,14 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
     }
     if (out_heads) memcpy(out_heads + r * h, heads, sizeof(int32_t) * h);
     if (out_E)
-      for (int32_t j = 0; j < in->heads; ++j) out_E[r * in->heads + j] = m > 0 ? S[j] / (double)m : 0.0;
+      for (int32_t j = 0; j < in->heads; ++j)
+        out_E[r * in->heads + j] = m > 0 ? S[j] / (double)(MUT(22) ? 1 : m) : 0.0;
     /* step 4: routed-head score over every legal token */
     ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
     row_cache rc = row_cache_new(in, row);
     for (int64_t s = 0; s < n; ++s) {
-      cand[s].v = score_cached(in, &rc, row, s, heads, h);
+      cand[s].v = MUT(23) ? score_cached(in, &rc, row, s, all, in->heads)
+                          : score_cached(in, &rc, row, s, heads, h);
       cand[s].i = s;
     }
     qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
@@ -531,7 +533,8 @@ int orc_misa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t h, in
         for (int32_t a = 0; a < k_prime; ++a)
           out_pool[r * k_prime + a] = a < cnt ? (int32_t)pool[a].i : -1;
       for (int64_t a = 0; a < cnt; ++a)
-        pool[a].v = score_cached(in, &rc, row, pool[a].i, all, in->heads);
+        pool[a].v = MUT(24) ? score_cached(in, &rc, row, pool[a].i, heads, h)
+                            : score_cached(in, &rc, row, pool[a].i, all, in->heads);
       qsort(pool, (size_t)cnt, sizeof(ranked), by_value_then_index);
       emit_topk(pool, cnt, topk, out_idx + r * topk, out_score + r * topk,
                 out_score64 ? out_score64 + r * topk : NULL);

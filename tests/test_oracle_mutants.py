@@ -36,6 +36,12 @@ MUTANTS = {
     18: "MISA-dagger pool one candidate short",
     19: "HISA keeps one block fewer than r",
     20: "stacked HISA reranks with every head instead of the routed ones",
+    21: "default query position 0 instead of n_k - n_q",
+    22: "router reports E = S instead of S / M_t",
+    23: "MISA scores tokens with every head instead of the routed ones",
+    24: "MISA-dagger reranks with the routed heads instead of all heads",
+    25: "bf16 words decoded with a 15-bit shift",
+    26: "e4m3 encode truncates instead of rounding",
 }
 
 

@@ -254,6 +254,24 @@ def test_pool_rounds_the_mean_once_to_the_key_type(oracle_mod):
     assert reps[0, 0] == 1.0 and reps[0, 1] == 3.0
 
 
+def test_misa_scores_tokens_with_the_routed_heads(oracle_mod):
+    """MISA, closed form (d = 2, two heads, h = 1): the router keeps head 0
+    (S_0 = 10.5 > S_1 = 2.5 over the two blocks of 2 keys), and the token
+    scores use head 0 only: 10, 0, 10, 1 for keys (1, 0), (0, 5), (1, 0),
+    (0.1, 0), so the top 3 are tokens 0, 2, 3 (all heads would give 10, 5, 10,
+    1 and pick token 1 instead of 3).  E = S / M_t with M_t = 2."""
+    q = np.array([[[[10.0, 0.0], [0.0, 1.0]]]], np.float32)
+    k = np.array([[[1.0, 0.0], [0.0, 5.0], [1.0, 0.0], [0.1, 0.0]]], np.float32)
+    w = np.ones((1, 1, 2), np.float32)
+    p = make(q, k, w, 3, q_pos0=[3])
+    out = oracle_mod.misa(oracle_mod.Inputs(p), 3, block=2, h=1)
+    assert out["heads"].tolist() == [[0]]
+    assert out["idx"].tolist() == [[0, 2, 3]]
+    assert out["score64"][0].tolist() == [10.0, 10.0, float(np.float32(0.1)) * 10.0]
+    rep1 = float(np.float32((np.float64(np.float32(0.1)) + 1.0) / 2.0))   # fp32 mean of 1 and 0.1f
+    assert out["E"][0].tolist() == [(10.0 * 0.5 + 10.0 * rep1) / 2.0, 2.5 / 2.0]
+
+
 def test_stacked_hisa_reranks_with_the_routed_heads(oracle_mod):
     """Stacked MISA + HISA, closed form (d = 2, two heads, h = 1): the router
     keeps head 0, so the rerank scores only w_0 ReLU(q_0 . k_s).
