@@ -413,7 +413,7 @@ static void pooled_key(const orc_inputs* in, int32_t b, int64_t lo, int64_t hi, 
 /* Representatives of the ceil(n/blk) blocks of the legal prefix [0, n). */
 static double* block_representatives(const orc_inputs* in, int32_t b, int64_t n, int32_t blk,
                                      int64_t* n_blocks) {
-  int64_t m = (n + blk - 1) / blk;
+  int64_t m = MUT(28) ? n / blk : (n + blk - 1) / blk;
   double* reps = (double*)malloc(sizeof(double) * (size_t)(m > 0 ? m : 1) * in->dim);
   for (int64_t a = 0; a < m; ++a) {
     int64_t lo = a * blk, hi = lo + blk < n ? lo + blk : n;
@@ -447,7 +447,7 @@ static void misa_route(const orc_inputs* in, int64_t row, int32_t blk, int32_t h
     double aw = MUT(7) ? (double)in->w[row * in->heads + j] : fabs((double)in->w[row * in->heads + j]);
     for (int64_t a = 0; a < m; ++a) {
       double z = dot_q_vec(in, row, j, reps + a * in->dim);
-      s += aw * (z > 0.0 ? z : 0.0);
+      s += aw * (MUT(29) ? fabs(z) : (z > 0.0 ? z : 0.0));
     }
     S[j] = s;
     order[j].v = s;

@@ -42,6 +42,8 @@ MUTANTS = {
     24: "MISA-dagger reranks with the routed heads instead of all heads",
     25: "bf16 words decoded with a 15-bit shift",
     26: "e4m3 encode truncates instead of rounding",
+    28: "blocks cover full blocks only (the boundary block dropped)",
+    29: "router takes |q . k~| instead of ReLU(q . k~)",
 }
 
 
