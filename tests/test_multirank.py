@@ -42,7 +42,8 @@ def _worker(rank, world, port, out):
 
 def test_max_over_ranks_gloo_world2():
     port = _free_port()
-    with mp.Manager() as m:
+    # spawn, not fork: the test process already runs torch and OpenMP threads
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         assert dict(out) == {0: 5.5, 1: 5.5}
