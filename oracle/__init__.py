@@ -21,6 +21,7 @@ MUTANT = int(os.environ.get("DSA_ORACLE_MUTANT", "0"))
 LIB = os.path.join(HERE, "libdsa_oracle.so" if MUTANT == 0 else f"libdsa_oracle_m{MUTANT}.so")
 
 F32, BF16, E4M3 = 0, 1, 2
+F64 = 3   # oracle-only operand type: values already decoded to fp64 (split_query)
 
 
 def build(force: bool = False) -> str:
@@ -55,9 +56,10 @@ def lib():
         _lib.orc_e4m3_encode.restype = C.c_uint8
         _lib.orc_e4m3_encode.argtypes = [C.c_float]
         _lib.orc_quantize_rows.argtypes = [vp, i32, i64, i32, vp, vp]
+        _lib.orc_split_query.argtypes = [vp, i32, i64, i32, vp]
         _lib.orc_dsa_rows.argtypes = [vp, i32, vp, i64, vp, vp, vp, vp]
         _lib.orc_score_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
-        _lib.orc_abs_score_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
+        _lib.orc_nu_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
         _lib.orc_pool.argtypes = [vp, i32, i64, i32, vp]
         _lib.orc_misa_rows.argtypes = [vp, i32, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp,
                                        vp, vp, vp]
@@ -174,8 +176,9 @@ def score_pairs(inp: Inputs, rows, s, heads=None):
     return out
 
 
-def abs_score_pairs(inp: Inputs, rows, s, heads=None):
-    """A(t, s) = sum_j |w| sum_c |q_jc k_c|: the error scale of each score."""
+def nu_pairs(inp: Inputs, rows, s, heads=None):
+    """nu(t, s) = sum_j |w_tj| ||q_tj|| ||k_s|| / sqrt(d) (fp64): the magnitude
+    scale of each score, the denominator of the relative score tolerance."""
     rows = np.ascontiguousarray(rows, np.int64)
     s = np.ascontiguousarray(s, np.int64)
     out = np.empty(len(rows), np.float64)
@@ -184,7 +187,7 @@ def abs_score_pairs(inp: Inputs, rows, s, heads=None):
         nh = heads.shape[1]
     else:
         nh = 0
-    lib().orc_abs_score_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(heads), nh, _p(out))
+    lib().orc_nu_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(heads), nh, _p(out))
     return out
 
 
@@ -235,3 +238,13 @@ def quantize_rows(x: np.ndarray, x_dtype: int):
     rc = lib().orc_quantize_rows(_p(x), x_dtype, rows, cols, _p(out), _p(sc))
     assert rc == 0
     return out, sc
+
+
+def split_query(x: np.ndarray, x_dtype: int) -> np.ndarray:
+    """Two-part e4m3 value of each query head vector (last axis): s * (hi + lo), fp64."""
+    x = np.ascontiguousarray(x)
+    dim = x.shape[-1]
+    out = np.empty(x.shape, np.float64)
+    rc = lib().orc_split_query(_p(x), x_dtype, x.size // dim, dim, _p(out))
+    assert rc == 0
+    return out

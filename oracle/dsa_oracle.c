@@ -63,7 +63,9 @@
 #endif
 #define MUT(n) (ORC_MUTANT == (n))
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2 };
+/* ORC_F64: operands already decoded to fp64 values (the tests pass the split
+ * query of orc_split_query this way); the CUDA library has no such type. */
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_E4M3 = 2, ORC_F64 = 3 };
 enum { ORC_OK = 0, ORC_ERR = -1 };
 
 typedef struct {
@@ -165,6 +167,48 @@ int orc_quantize_rows(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
   return ORC_OK;
 }
 
+/* Query operand of the FP8-key path when the query arrives as bf16 / fp32:
+ * the query is converted to the e4m3 compute type in two parts ([FP8]: the
+ * query is converted to the compute type in registers, the dot products
+ * accumulate in higher precision).  Reading: per (row, head) vector x of dim
+ * values, s = amax|x| / 448 in fp32 (amax == 0 gives s = 1), v = x / s in fp32,
+ * hi = e4m3(v), lo = e4m3(v - hi) with the subtraction in fp32; the operand
+ * value is s * (hi + lo), written here exactly in fp64.
+ *   x [vecs, dim] (F32 or BF16), out [vecs, dim] fp64. */
+int orc_split_query(const void* x, int32_t x_dtype, int64_t vecs, int32_t dim, double* out) {
+  if (x_dtype != ORC_F32 && x_dtype != ORC_BF16) return ORC_ERR;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < vecs; ++r) {
+    float amax = 0.0f;
+    for (int32_t c = 0; c < dim; ++c) {
+      float v;
+      if (x_dtype == ORC_F32) {
+        v = ((const float*)x)[r * dim + c];
+      } else {
+        uint32_t b = (uint32_t)((const uint16_t*)x)[r * dim + c] << 16;
+        memcpy(&v, &b, 4);
+      }
+      if (fabsf(v) > amax) amax = fabsf(v);
+    }
+    volatile float sc = (amax > 0.0f) ? amax / 448.0f : 1.0f;
+    for (int32_t c = 0; c < dim; ++c) {
+      float v;
+      if (x_dtype == ORC_F32) {
+        v = ((const float*)x)[r * dim + c];
+      } else {
+        uint32_t b = (uint32_t)((const uint16_t*)x)[r * dim + c] << 16;
+        memcpy(&v, &b, 4);
+      }
+      volatile float t = v / sc;
+      double hi = orc_e4m3_decode(orc_e4m3_encode(t));
+      volatile float res = t - (float)hi;
+      double lo = MUT(33) ? 0.0 : orc_e4m3_decode(orc_e4m3_encode(res));
+      out[r * dim + c] = (double)sc * (hi + lo);
+    }
+  }
+  return ORC_OK;
+}
+
 /* Nearest-even rounding of an exact fp64 value to bf16 (returned as double). */
 static double round_to_bf16(double x) {
   if (x == 0.0 || !isfinite(x)) return x;
@@ -194,6 +238,7 @@ static double q_val(const orc_inputs* in, int64_t row, int32_t j, int32_t c) {
                         : (row * in->heads + j) * (int64_t)in->dim + c;
   switch (in->q_dtype) {
     case ORC_F32: return (double)((const float*)in->q)[off];
+    case ORC_F64: return ((const double*)in->q)[off];
     case ORC_BF16: return bf16_value(((const uint16_t*)in->q)[off]);
     default: return (double)in->q_scale[row] * orc_e4m3_decode(((const uint8_t*)in->q)[off]);
   }
@@ -204,6 +249,7 @@ static double k_val(const orc_inputs* in, int32_t b, int64_t s, int32_t c) {
   int64_t off = kr * in->dim + c;
   switch (in->k_dtype) {
     case ORC_F32: return (double)((const float*)in->k)[off];
+    case ORC_F64: return ((const double*)in->k)[off];
     case ORC_BF16: return bf16_value(((const uint16_t*)in->k)[off]);
     default: return (double)in->k_scale[kr] * orc_e4m3_decode(((const uint8_t*)in->k)[off]);
   }
@@ -372,26 +418,39 @@ int orc_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s,
   return ORC_OK;
 }
 
-/* Error scale of a score at (row, s): A = sum_j |w_{t,j}| sum_c |q_{t,j,c} k_{s,c}|,
- * the sum of the absolute values of the products the score adds up (the
- * standard scale of rounding and quantisation error in a sum of products).
- * heads == NULL means all heads, otherwise heads is [n, nh].  Used by the
- * tests as the denominator of the relative score tolerance. */
-int orc_abs_score_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
-                        const int32_t* heads, int32_t nh, double* out) {
+/* Magnitude scale of a score at (row, s), the denominator of the relative
+ * score tolerance: nu = sum_j |w_{t,j}| ||q_{t,j}|| ||k_s|| / sqrt(d), the
+ * Cauchy-Schwarz bound on |q . k| (||q|| ||k||) scaled by 1/sqrt(d) to the size
+ * a dot product of unaligned d-vectors typically has, weighted by |w| and
+ * summed over the heads.  Norms are of the decoded operand values, in fp64.
+ * heads == NULL means all heads, otherwise heads is [n, nh].  Test
+ * infrastructure: the tolerance rule divides score differences by
+ * max(|I|, nu). */
+int orc_nu_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                 const int32_t* heads, int32_t nh, double* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t a = 0; a < n; ++a) {
     int64_t row = rows[a];
     int32_t b = (int32_t)(row / in->n_q);
     int32_t cnt = heads ? nh : in->heads;
+    double kk = 0.0;
+    for (int32_t c = 0; c < in->dim; ++c) {
+      double v = k_val(in, b, s[a], c);
+      kk += v * v;
+    }
+    double knorm = MUT(32) ? kk : sqrt(kk);
     double acc = 0.0;
     for (int32_t x = 0; x < cnt; ++x) {
       int32_t j = heads ? heads[a * nh + x] : x;
-      double t = 0.0;
-      for (int32_t c = 0; c < in->dim; ++c) t += fabs(q_val(in, row, j, c) * k_val(in, b, s[a], c));
-      acc += fabs((double)in->w[row * in->heads + j]) * t;
+      double qq = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) {
+        double v = q_val(in, row, j, c);
+        qq += v * v;
+      }
+      double wj = (double)in->w[row * in->heads + j];
+      acc += (MUT(30) ? wj : fabs(wj)) * sqrt(qq);
     }
-    out[a] = acc;
+    out[a] = acc * knorm / (MUT(31) ? 1.0 : sqrt((double)in->dim));
   }
   return ORC_OK;
 }

@@ -1,8 +1,11 @@
 """GPU parity of dsa_index (and the FP8 quantiser) against the CPU oracle.
 
 Exact on integer-valued inputs; within the tolerance rule of tests/parity.py on
-real-valued inputs (1e-3 for bf16 operands, 2e-2 for fp8 against the
-unquantised values).  Sizes span several 128-key tiles and query tiles with
+real-valued inputs: 1e-3 of max(|I|, nu) against the oracle on the operands the
+GPU computes with (bf16, or the same e4m3 codes and scales, or the two-part
+e4m3 value of a bf16 query against e4m3 keys).  Against the unquantised values
+an fp8 run differs by its quantisation error, which is measured and reported
+(IoU floor, largest relative difference) rather than asserted.  Sizes span several 128-key tiles and query tiles with
 ragged tails; full-size workloads are checked on sampled rows.
 """
 import numpy as np
@@ -124,8 +127,8 @@ def test_bf16_real_small(B):
     inp = oracle.Inputs(p)
     rows = np.arange(p.batch * p.n_q)[::7]
     ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
-    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
-    assert iou > 0.99
+    r = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
+    assert r.iou > 0.99
 
 
 def test_bf16_needles_32k_sampled(B):
@@ -135,8 +138,8 @@ def test_bf16_needles_32k_sampled(B):
     inp = oracle.Inputs(p)
     rows = gen.stratified_rows(p, 24)
     ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
-    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
-    assert iou > 0.99
+    r = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
+    assert r.iou > 0.99
     for b, t, s in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
         assert s in set(gi[b * p.n_q + t].tolist()), "needle not selected"
 
@@ -179,12 +182,32 @@ def test_fp8_prefill(B):
     inq = oracle.Inputs(p, q=rqc, k=rkc, q_dtype=gen.E4M3, k_dtype=gen.E4M3, q_scale=rqs,
                         k_scale=rks)
     ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
-    parity.within_tolerance(inq, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16)
-    # against the unquantised bf16 values
+    r = parity.within_tolerance(inq, rows, gi[rows], gs[rows], ri, rs64, TOL_BF16,
+                                label="same e4m3 operands")
+    assert r.iou > 0.99
+    # against the unquantised bf16 values: the quantisation's own effect
     inp = oracle.Inputs(p)
     ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
-    iou = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_FP8)
-    assert iou > 0.7
+    r = parity.within_tolerance(inp, rows, gi[rows], gs[rows], ri, rs64, TOL_FP8,
+                                label="vs unquantised", check_scores=False)
+    assert r.iou > 0.9 and r.max_rel < 0.05
+
+
+def _check_split_decode(p, gi, gs, rkc, rks):
+    """bf16 query against e4m3 keys: 1e-3 against the oracle on the operands the
+    MMA sees (the query's two-part e4m3 value, oracle.split_query, and the same
+    key codes and scales); the bf16 query itself differs by the split's own
+    rounding (at most 2^-8 per value), reported against the 2e-2 fp8 figure."""
+    rows = np.arange(p.batch * p.n_q)
+    qsplit = oracle.split_query(p.q.reshape(-1, p.dim), gen.BF16).reshape(p.q.shape)
+    ins = oracle.Inputs(p, q=qsplit, q_dtype=oracle.F64, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
+    ri, _, rs64, _ = oracle.dsa(ins, p.topk, rows)
+    r = parity.within_tolerance(ins, rows, gi, gs, ri, rs64, TOL_BF16, label="split query")
+    assert r.iou > 0.99
+    inq = oracle.Inputs(p, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
+    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
+    r = parity.within_tolerance(inq, rows, gi, gs, ri, rs64, TOL_FP8, label="bf16 query")
+    assert r.iou > 0.95
 
 
 @pytest.mark.parametrize("batch,n_k", [(4, 20000), (3, 5000)])
@@ -196,11 +219,7 @@ def test_fp8_decode_split_query(B, batch, n_k):
     gi, gs = run_dsa(B, p, k=kc, k_scale=ks)
     rkc, rks = oracle.quantize_rows(p.k, gen.BF16)
     assert np.array_equal(kc.cpu().numpy(), rkc)
-    inq = oracle.Inputs(p, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
-    rows = np.arange(batch)
-    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
-    iou = parity.within_tolerance(inq, rows, gi, gs, ri, rs64, TOL_FP8)
-    assert iou > 0.9
+    _check_split_decode(p, gi, gs, rkc, rks)
 
 
 @pytest.mark.parametrize("batch,n_k", [(5, 9000), (3, 3001), (2, 200)])
@@ -230,11 +249,7 @@ def test_fp8_decode_full_size(B):
     kc, ks = B.dsa_quantize_e4m3(dev(p.k))
     gi, gs = run_dsa(B, p, k=kc, k_scale=ks)
     rkc, rks = oracle.quantize_rows(p.k, gen.BF16)
-    inq = oracle.Inputs(p, k=rkc, k_dtype=gen.E4M3, k_scale=rks)
-    rows = np.arange(32)
-    ri, _, rs64, _ = oracle.dsa(inq, p.topk, rows)
-    iou = parity.within_tolerance(inq, rows, gi, gs, ri, rs64, TOL_FP8)
-    assert iou > 0.9
+    _check_split_decode(p, gi, gs, rkc, rks)
 
 
 def test_check_flag_reports_bad_scale(B):

@@ -216,8 +216,11 @@ def check_pool(inp, rows, g_pool, g_heads, kp):
         if len(diff):
             rr = np.full(len(diff), row, np.int64)
             hh = np.repeat(np.asarray(heads)[None], len(diff), 0)
-            scale = oracle.abs_score_pairs(inp, rr, diff, hh)
-            assert np.all(np.abs(v[diff] - cut) <= TOL * scale), f"row {row}: pool differs"
+            e = TOL * np.maximum(np.abs(v[diff]), oracle.nu_pairs(inp, rr, diff, hh))
+            kth = np.array([order[nv - 1]], np.int64)
+            e_cut = TOL * max(abs(cut), float(oracle.nu_pairs(
+                inp, np.array([row], np.int64), kth, np.asarray(heads)[None])[0]))
+            assert np.all(np.abs(v[diff] - cut) <= e + e_cut), f"row {row}: pool differs"
 
 
 def check_blocks(inp, rows, g_blocks, block, r, heads=None):
@@ -254,9 +257,9 @@ def test_misa_real_conditional(B, real_small):
     check_heads(inp, rows, g["heads"], g["E"], ref["E"], 8)
     fh = g["heads"][rows]
     ref2 = oracle.misa(inp, p.topk, 256, 8, rows=rows, forced_heads=fh)
-    iou = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref2["idx"],
-                                  ref2["score64"], TOL, heads=fh)
-    assert iou > 0.98
+    r = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref2["idx"],
+                                ref2["score64"], TOL, heads=fh)
+    assert r.iou > 0.98
 
 
 def test_misa_dagger_real_conditional(B, real_small):
@@ -267,9 +270,9 @@ def test_misa_dagger_real_conditional(B, real_small):
     check_pool(inp, rows, g["pool"], g["heads"], 1024)
     ref = oracle.misa(inp, p.topk, 256, 8, k_prime=1024, rows=rows,
                       forced_heads=g["heads"][rows], forced_pool=g["pool"][rows])
-    iou = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
-                                  ref["score64"], TOL)
-    assert iou > 0.98
+    r = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
+                                ref["score64"], TOL)
+    assert r.iou > 0.98
 
 
 @pytest.mark.parametrize("stacked", [False, True])
@@ -284,10 +287,10 @@ def test_hisa_real_conditional(B, real_small, stacked):
     ref = oracle.hisa(inp, p.topk, 64, 16, route_h=h, route_block=256, rows=rows,
                       forced_heads=None if heads is None else heads[rows],
                       forced_blocks=g["blocks"][rows])
-    iou = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
-                                  ref["score64"], TOL,
-                                  heads=None if heads is None else heads[rows])
-    assert iou > 0.98
+    r = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
+                                ref["score64"], TOL,
+                                heads=None if heads is None else heads[rows])
+    assert r.iou > 0.98
 
 
 # ------------------------------------------------- full size, sampled rows ---
@@ -308,15 +311,17 @@ def test_full_size_misa_and_dagger_sampled(B, full128k):
     check_heads(inp, rows, g["heads"], g["E"], ref["E"], 8)
     fh = g["heads"][rows]
     ref2 = oracle.misa(inp, p.topk, 1024, 8, rows=rows, forced_heads=fh)
-    parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref2["idx"],
-                            ref2["score64"], TOL, heads=fh)
+    r = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref2["idx"],
+                                ref2["score64"], TOL, heads=fh, label="MISA 128K")
+    assert r.iou > 0.98
     gd = run_route(B, p, "dagger", block=1024, h=8, k_prime=8192)
     assert np.array_equal(gd["heads"], g["heads"])
     check_pool(inp, rows, gd["pool"], gd["heads"], 8192)
     ref3 = oracle.misa(inp, p.topk, 1024, 8, k_prime=8192, rows=rows, forced_heads=fh,
                        forced_pool=gd["pool"][rows])
-    parity.within_tolerance(inp, rows, gd["idx"][rows], gd["score"][rows], ref3["idx"],
-                            ref3["score64"], TOL)
+    r = parity.within_tolerance(inp, rows, gd["idx"][rows], gd["score"][rows], ref3["idx"],
+                                ref3["score64"], TOL, label="MISA-dagger 128K")
+    assert r.iou > 0.98
 
 
 @pytest.mark.parametrize("stacked", [False, True])
@@ -332,5 +337,7 @@ def test_full_size_hisa_sampled(B, full128k, stacked):
     ref = oracle.hisa(inp, p.topk, 64, 128, route_h=h, route_block=1024, rows=rows,
                       forced_heads=None if heads is None else heads[rows],
                       forced_blocks=g["blocks"][rows])
-    parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
-                            ref["score64"], TOL, heads=None if heads is None else heads[rows])
+    r = parity.within_tolerance(inp, rows, g["idx"][rows], g["score"][rows], ref["idx"],
+                                ref["score64"], TOL, heads=None if heads is None else heads[rows],
+                                label="HISA 128K")
+    assert r.iou > 0.98

@@ -44,6 +44,10 @@ MUTANTS = {
     26: "e4m3 encode truncates instead of rounding",
     28: "blocks cover full blocks only (the boundary block dropped)",
     29: "router takes |q . k~| instead of ReLU(q . k~)",
+    30: "tolerance scale nu sums signed w instead of |w|",
+    31: "tolerance scale nu without the 1/sqrt(d) factor",
+    32: "tolerance scale nu with the squared key norm",
+    33: "split query drops its low e4m3 part",
 }
 
 

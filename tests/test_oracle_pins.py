@@ -470,3 +470,81 @@ def test_cost_counters_match_page_arithmetic(oracle_mod):
     assert 131072 * 32 == by["fp8_key_bytes_128k_d32"]
     assert 131072 * 128 == by["fp8_key_bytes_128k_d128"]
     assert 2048 * 4 == by["indices_bytes_per_request_k2048"]
+
+
+# ------------------------------------------------- tolerance scale nu (closed form) --
+
+def test_nu_closed_form(oracle_mod):
+    """nu(t, s) = sum_j |w_tj| ||q_tj|| ||k_s|| / sqrt(d).  With q_tj = c_j (1, ..., 1)
+    (||q_tj|| = |c_j| sqrt(d)) and k_s = b_s e_0 (||k_s|| = |b_s|) it is
+    |b_s| sum_j |w_j| |c_j|, whatever d is; negative weights count by magnitude."""
+    d, H = 16, 3
+    c = np.array([2.0, -1.0, 0.5], np.float32)
+    w = np.array([1.0, -0.5, 3.0], np.float32)
+    b = np.array([3.0, -2.0, 0.0, 1.5], np.float32)
+    q = np.ones((1, 1, H, d), np.float32) * c[None, None, :, None]
+    k = np.zeros((1, len(b), d), np.float32)
+    k[0, :, 0] = b
+    p = make(q, k, w[None, None], topk=1, q_pos0=[len(b) - 1])
+    inp = oracle_mod.Inputs(p)
+    s = np.arange(len(b), dtype=np.int64)
+    got = oracle_mod.nu_pairs(inp, np.zeros(len(b), np.int64), s)
+    want = np.abs(b) * float(np.sum(np.abs(w) * np.abs(c)))   # = |b| * (2 + 0.5 + 1.5)
+    assert np.array_equal(got, want.astype(np.float64))
+    # restricted to heads (0, 2): |b| (2 + 1.5)
+    got2 = oracle_mod.nu_pairs(inp, np.zeros(len(b), np.int64), s,
+                               np.tile(np.array([[0, 2]], np.int32), (len(b), 1)))
+    assert np.array_equal(got2, np.abs(b) * 3.5)
+
+
+def test_nu_is_the_typical_score_size(oracle_mod):
+    """For independent N(0,1) q and k the dot product of one head has standard
+    deviation sqrt(d) = E[||q|| ||k||] / sqrt(d) up to O(1/d): over many pairs the
+    single-head nu (|w| = 1) matches the root mean square of q . k within 5 %."""
+    rng = np.random.default_rng(8)
+    d, n = 128, 4000
+    q = rng.standard_normal((1, n, 1, d)).astype(np.float32)
+    k = rng.standard_normal((1, n, d)).astype(np.float32)
+    p = make(q, k, np.ones((1, n, 1), np.float32), topk=1)
+    inp = oracle_mod.Inputs(p)
+    rows = np.arange(n, dtype=np.int64)
+    s = np.zeros(n, np.int64)                       # key 0 is legal for every row
+    nu = oracle_mod.nu_pairs(inp, rows, s)
+    dots = np.einsum("nd,d->n", q[0, :, 0].astype(np.float64), k[0, 0].astype(np.float64))
+    rms = math.sqrt(float(np.mean(dots ** 2)))
+    assert abs(float(np.mean(nu)) / rms - 1.0) < 0.05
+
+
+# --------------------------------------------------- split query (FP8-key path) --
+
+def test_split_query_worked_values(oracle_mod):
+    """amax 448 gives s = 1.  300 -> hi 288 (e4m3 spacing 32 on [256, 512)), residual
+    12 (exact) -> 300; 301 -> 288 + 13 = 301; 300.5 -> residual 12.5, an e4m3 tie
+    between 12 and 13 (spacing 1 on [8, 16)), rounded to even: 300."""
+    x = np.zeros((1, 8), np.float32)
+    x[0, :5] = [448.0, 300.0, 301.0, 300.5, -3.0]
+    v = oracle_mod.split_query(x, F32)
+    assert list(v[0, :5]) == [448.0, 300.0, 301.0, 300.0, -3.0]
+    assert np.all(v[0, 5:] == 0.0)
+    z = oracle_mod.split_query(np.zeros((2, 8), np.float32), F32)
+    assert np.all(z == 0.0)
+
+
+def test_split_query_error_bound(oracle_mod):
+    """Per value: |x - s (hi + lo)| <= 2^-8 |x| + 2^-10 s.  hi has e4m3's four
+    significant bits, so the residual is at most half hi's spacing, <= 2^-4 |x|;
+    its own code adds at most half its spacing, <= 2^-8 |x|, or at most half the
+    subnormal step 2^-9 (times s) below 2^-6.  A bf16 input (eight significant
+    bits) is reproduced within the same bound, and exact e4m3 multiples of s are
+    reproduced exactly."""
+    rng = np.random.default_rng(9)
+    x = (rng.standard_normal((64, 128)) * np.exp(rng.uniform(-6, 6, (64, 1)))).astype(np.float32)
+    xb = gen.f32_to_bf16_bits(x)
+    for arr, dt, vals in ((x, F32, x.astype(np.float64)),
+                          (xb, BF16, gen.bf16_bits_to_f32(xb).astype(np.float64))):
+        v = oracle_mod.split_query(arr, dt)
+        s = np.max(np.abs(vals), axis=1, keepdims=True).astype(np.float32) / np.float32(448.0)
+        assert np.all(np.abs(vals - v) <= 2.0 ** -8 * np.abs(vals) + 2.0 ** -10 * s)
+    codes = rng.integers(-7, 8, size=(4, 128)).astype(np.float32) * 32.0
+    codes[:, 0] = 448.0
+    assert np.array_equal(oracle_mod.split_query(codes, F32), codes.astype(np.float64))

@@ -37,7 +37,8 @@ def _row_with_room(case):
 
 def test_reference_rows_pass(case):
     inp, rows, ri, rs, rs64 = case
-    assert parity.within_tolerance(inp, rows, ri, rs, ri, rs64, TOL) == 1.0
+    r = parity.within_tolerance(inp, rows, ri, rs, ri, rs64, TOL)
+    assert r.iou == 1.0 and r.max_rel < 1e-6
     parity.exact(ri, rs, ri, rs)
 
 
@@ -57,15 +58,48 @@ def test_far_token_swapped_in_is_rejected(case):
         parity.within_tolerance(inp, rows, gi, gs, ri, rs64, TOL)
 
 
-def test_score_outside_tolerance_is_rejected(case):
+def _nu_numpy(inp, row, s):
+    """nu(t, s) = sum_j |w_tj| ||q_tj|| ||k_s|| / sqrt(d), from the bf16 operands."""
+    p = inp.prob
+    q = gen.bf16_bits_to_f32(p.q.reshape(p.batch * p.n_q, p.heads, p.dim)[row]).astype(np.float64)
+    k = gen.bf16_bits_to_f32(p.k[row // p.n_q, s]).astype(np.float64)
+    w = p.w.reshape(-1, p.heads)[row].astype(np.float64)
+    return float(np.sum(np.abs(w) * np.linalg.norm(q, axis=1)) * np.linalg.norm(k)
+                 / np.sqrt(p.dim))
+
+
+@pytest.mark.parametrize("factor,rejected", [(2.0, True), (0.5, False)])
+def test_score_error_against_the_tolerance(case, factor, rejected):
+    """A last-place score moved by factor x tol x max(|I|, nu) (nu computed here
+    from the operands, independently of the oracle) is rejected above the
+    tolerance and accepted below it."""
     inp, rows, ri, rs, rs64 = case
     a = 3
     row = int(rows[a])
-    scale = oracle.abs_score_pairs(inp, np.array([row], np.int64), ri[a, -1:])[0]
+    nv = int(np.sum(ri[a] >= 0))
+    scale = max(abs(float(rs64[a, nv - 1])), _nu_numpy(inp, row, int(ri[a, nv - 1])))
     gs = rs.copy()
-    gs[a, -1] = np.float32(gs[a, -1] - 10 * TOL * scale)   # still last in order
-    with pytest.raises(AssertionError, match="score error"):
-        parity.within_tolerance(inp, rows, ri, gs, ri, rs64, TOL)
+    gs[a, nv - 1] = np.float32(rs64[a, nv - 1] - factor * TOL * scale)   # still last in order
+    if rejected:
+        with pytest.raises(AssertionError, match="score error"):
+            parity.within_tolerance(inp, rows, ri, gs, ri, rs64, TOL)
+    else:
+        r = parity.within_tolerance(inp, rows, ri, gs, ri, rs64, TOL)
+        assert 0.4 * TOL < r.max_rel < 0.6 * TOL
+
+
+def test_nu_is_well_below_the_absolute_sum(case):
+    """On N(0,1) operands nu is several times smaller than sum_j |w| sum_c |q_c k_c|
+    (the scale an earlier rule used), so the tolerance rule is that much tighter."""
+    inp, rows, ri, _, _ = case
+    p = inp.prob
+    row = int(rows[5])
+    s = int(ri[5, 0])
+    q = gen.bf16_bits_to_f32(p.q.reshape(-1, p.heads, p.dim)[row]).astype(np.float64)
+    k = gen.bf16_bits_to_f32(p.k[0, s]).astype(np.float64)
+    w = p.w.reshape(-1, p.heads)[row].astype(np.float64)
+    absum = float(np.sum(np.abs(w) * np.sum(np.abs(q * k[None]), axis=1)))
+    assert _nu_numpy(inp, row, s) < absum / 4
 
 
 def test_duplicate_index_is_rejected(case):
