@@ -1,19 +1,22 @@
 #!/usr/bin/env python
 """Benchmark of the B200 DSA lightning indexer (one JSON line on rank 0).
 
-Default workload: DSA indexer prefill, batch 1, L = 32768 causal, H_I = 64,
-d = 128, top-k = 2048, bf16 q / k ~ N(0,1), w ~ N(0, 1/64), 32 planted needles.
-A step is one whole indexer layer (score -> causal mask -> exact token top-k
-set, the library's default unordered output) through the library's C ABI.
-Inputs are larger than L2 (q alone is 512 MiB), so no explicit flush is needed
-between steps.  Other workloads: the 32K fp8 variant, the 128K-key decode
-batch, and at L = 131072 the DSA layer, MISA, MISA-dagger, HISA and stacked
-MISA + HISA (--workload).
+Default workload: the DSA indexer prefill layer the metric is quoted on,
+batch 1, L = 131072 causal, H_I = 64, d = 128, top-k = 2048, bf16 q / k ~ N(0,1),
+w ~ N(0, 1/64).  A step is one whole indexer layer (score -> causal mask ->
+exact token top-k set, the library's default unordered output) through the
+library's C ABI.  Inputs are larger than L2 (q alone is 2 GiB), so no explicit
+flush is needed between steps.  The same run then times, on one GPU, the
+metric's other configurations as secondary lines: the 32 x 131072-key e4m3
+decode batch (us / query) and MISA, MISA-dagger, HISA and stacked MISA + HISA
+at L = 131072 (ms / layer).  Other workloads run alone with --workload.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-N > 1 (torchrun): every rank runs its own independent layer (weak scaling, no
-collective on the data path); the reported time is the max over ranks.
+N > 1 (torchrun): the layer is partitioned across the ranks (prefill: zigzag
+query-row chunks, decode: sequences; sparse_attention_token_dsa_b200.partition)
+with no collective on the data path; the reported time of a layer is the max
+over ranks (strong scaling: the layer is fixed, the ranks share it).
 --impl reference times the CPU oracle (the only reference this method has) on
 a bounded sample of rows of the same workload, extrapolated to a full layer.
 """
@@ -26,6 +29,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -100,17 +104,8 @@ WORKLOADS = {
 }
 ROUTED = ("misa", "dagger", "hisa")
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one scan-kernel launch, from the
-# ncu captures summarised under profiles/, valid only while the kernel sources
-# hash to `src`; otherwise the traffic is reported as null.
-TRAFFIC = {
-    # profiles/scan_kernel_dsa_prefill_32k.md: 601.29 MB read + 1.91 GB written
-    "dsa_prefill_32k": {"bytes": 601_290_000 + 1_910_000_000, "src": "23b61bde9a857492"},
-    # profiles/scan_kernel_dsa_decode_128k.md: 559.32 MB read + 26.36 MB written
-    "dsa_decode_128k": {"bytes": 559_320_000 + 26_360_000, "src": "23b61bde9a857492"},
-}
-
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic_scan_kernel.md")
 
 
 def kernel_hash() -> str:
@@ -119,6 +114,24 @@ def kernel_hash() -> str:
         with open(os.path.join(ROOT, "sparse_attention_token_dsa_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """dram__bytes_read.sum + dram__bytes_write.sum of one scan-kernel launch of
+    `workload`, from the table of one-pass ncu captures in profiles/; None
+    unless that capture was taken on the present kernel sources (their hash is
+    recorded beside each row)."""
+    if not os.path.exists(TRAFFIC_TABLE):
+        return None
+    src = kernel_hash()
+    for line in open(TRAFFIC_TABLE):
+        f = [x.strip().strip("`") for x in line.strip().strip("|").split("|")]
+        if len(f) >= 5 and f[0] == workload and f[4] == src:
+            try:
+                return int(f[1].replace(",", "")) + int(f[2].replace(",", ""))
+            except ValueError:
+                return None
+    return None
 
 
 def peaks():
@@ -193,10 +206,9 @@ class ClockSampler:
     def __init__(self, index: int):
         self.index = index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"dsa_bench_clocks_{os.getpid()}.csv")
 
     def __enter__(self):
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -346,6 +358,12 @@ def run_reference(args, w, p):
 
 # ------------------------------------------------------------------ GPU arm --
 
+# in an order that reuses generated problems: MISA and MISA-dagger share the
+# headline problem, stacked HISA shares HISA's clustered keys
+SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "hisa_prefill_128k",
+             "hisa_misa_prefill_128k", "dsa_decode_128k"]
+
+
 def max_over_ranks(x: float, device=None) -> float:
     """The largest value of x over all ranks (x itself without a process group)."""
     import torch
@@ -357,14 +375,373 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
+def _bf16(a):
+    import torch
+    return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+
+
+class Case:
+    """One workload on this rank: its share of the layer (partition.py) as a list
+    of library calls on device-resident inputs, plus the same calls fed from
+    pinned host buffers for the end-to-end measurement."""
+
+    def __init__(self, w, p, dev, world, rank):
+        import torch
+        from sparse_attention_token_dsa_b200 import binding as B
+        from sparse_attention_token_dsa_b200 import partition as part
+        self.w, self.p, self.dev, self.B = w, p, dev, B
+        self.kind = w["kind"]
+        self.fp8 = w.get("fp8", False)
+        self.stream = torch.cuda.current_stream()
+        # this rank's share: (batch start, batch count, row start, row count) pieces
+        if self.kind == "decode":
+            b0, nb = part.decode_seq_range(p.batch, world, rank)
+            self.pieces = [(b0, nb, 0, p.n_q)] if nb else []
+        else:
+            assert p.batch == 1 or world == 1, "prefill partition is per sequence (batch 1)"
+            self.pieces = [(0, p.batch, r0, nr)
+                           for r0, nr in part.prefill_row_ranges(p.n_q, world, rank)]
+        self.qh, self.kh, self.wh = _bf16(p.q), _bf16(p.k), torch.from_numpy(p.w)
+        self.q = self.qh.to(dev)
+        self.k = self.kh.to(dev)
+        self.wt = self.wh.to(dev)
+        self.q_scale = self.k_scale = None
+        if self.fp8:
+            self.k, self.k_scale = B.dsa_quantize_e4m3(self.k)
+            if self.kind == "prefill":
+                q2, qs = B.dsa_quantize_e4m3(self.q.reshape(p.batch * p.n_q, -1))
+                self.q, self.q_scale = q2.reshape(p.q.shape), qs.reshape(p.batch, p.n_q)
+        self.idx = torch.full((p.batch, p.n_q, p.topk), -1, dtype=torch.int32, device=dev)
+        self.sc = torch.empty((p.batch, p.n_q, p.topk), dtype=torch.float32, device=dev)
+        self.calls = [self._piece(pc) for pc in self.pieces]
+        nbytes = max([c["ws_bytes"] for c in self.calls] + [256])
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.launches = sum(c["launches"] for c in self.calls)
+        torch.cuda.synchronize()
+
+    def _piece(self, pc):
+        """Argument views of one library call over rows [r0, r0 + nr) of sequences
+        [b0, b0 + nb), with its causal position and key length made explicit."""
+        import torch
+        B, p, w = self.B, self.p, self.w
+        b0, nb, r0, nr = pc
+        pos0 = torch.tensor([p.pos0(b) + r0 for b in range(b0, b0 + nb)], dtype=torch.int32,
+                            device=self.dev)
+        klen = torch.tensor([p.klen(b) for b in range(b0, b0 + nb)], dtype=torch.int32,
+                            device=self.dev)
+
+        def view(t, seq_axis_rows=True):
+            if t is None:
+                return None
+            t = t[b0:b0 + nb]
+            return t[:, r0:r0 + nr] if seq_axis_rows else t
+
+        c = dict(q=view(self.q), k=view(self.k, False), w=view(self.wt),
+                 q_scale=view(self.q_scale), k_scale=view(self.k_scale, False),
+                 idx=view(self.idx), sc=view(self.sc), pos0=pos0, klen=klen, rows=(b0, nb, r0, nr))
+        for key in ("q", "w", "q_scale", "idx", "sc"):
+            if c[key] is not None and not c[key].is_contiguous():
+                raise ValueError("partitioned rows must be contiguous (batch 1 prefill)")
+        c["prob"] = B.problem(c["q"], c["k"], p.topk, pos0, klen)
+        if self.kind in ROUTED:
+            algo = {"misa": B.DSA_ALGO_MISA, "dagger": B.DSA_ALGO_MISA_DAGGER,
+                    "hisa": B.DSA_ALGO_HISA}[self.kind]
+            if self.kind == "hisa":
+                rp = B.route_params(misa_block=w["block"] if w["h"] else 0, misa_h=w["h"],
+                                    hisa_block=w["hb"], hisa_r=w["r"])
+            else:
+                rp = B.route_params(misa_block=w["block"], misa_h=w["h"],
+                                    k_prime=w.get("k_prime", 0))
+            c["ws_bytes"] = B.dsa_workspace_size(c["prob"], algo, rp)
+            chunks = -(-nr // B.dsa_route_chunk_rows(c["prob"], algo, rp))
+            c["chunks"] = chunks
+            if self.kind == "misa":
+                c["launches"] = 2 + 2 * chunks
+            elif self.kind == "dagger":
+                c["launches"] = 2 + 4 * chunks
+            else:
+                c["launches"] = (2 if w["h"] else 0) + 1 + 5 * chunks
+        else:
+            c["ws_bytes"] = B.dsa_workspace_size(c["prob"])
+            c["launches"] = 2 + (1 if (self.fp8 and self.kind == "decode") else 0)
+        return c
+
+    def _routed(self, c, q, k, w_, out):
+        B, p, w = self.B, self.p, self.w
+        if self.kind == "misa":
+            B.misa_index(q, k, w_, p.topk, w["block"], w["h"], q_pos0=c["pos0"],
+                         k_len=c["klen"], out=out, workspace=self.ws)
+        elif self.kind == "dagger":
+            B.misa_dagger_index(q, k, w_, p.topk, w["block"], w["h"], w["k_prime"],
+                                q_pos0=c["pos0"], k_len=c["klen"], out=out, workspace=self.ws)
+        else:
+            B.hisa_index(q, k, w_, p.topk, w["hb"], w["r"], route_h=w["h"],
+                         route_block=w["block"], q_pos0=c["pos0"], k_len=c["klen"], out=out,
+                         workspace=self.ws)
+
+    def step(self, ev=None):
+        """One pass over this rank's share.  ev: a list of (start, end) event pairs
+        that bracket the scan stage of each DSA call (the whole call when routed)."""
+        B = self.B
+        for i, c in enumerate(self.calls):
+            if ev is not None:
+                ev[i][0].record(self.stream)
+            if self.kind in ROUTED:
+                self._routed(c, c["q"], c["k"], c["w"], (c["idx"], c["sc"]))
+                if ev is not None:
+                    ev[i][1].record(self.stream)
+            else:
+                B.dsa_index_scan(c["prob"], c["q"], c["k"], c["w"], self.ws, q_scale=c["q_scale"],
+                                 k_scale=c["k_scale"], stream=self.stream)
+                if ev is not None:
+                    ev[i][1].record(self.stream)
+                B.dsa_index_select(c["prob"], c["idx"], c["sc"], self.ws, stream=self.stream)
+
+    def status(self):
+        return self.B.dsa_read_status(self.ws)
+
+    # ---- end to end: this rank's inputs copied from pinned host buffers, its
+    # outputs copied back, inside the timed region
+    def e2e_setup(self):
+        import torch
+        p = self.p
+        self.qp, self.kp, self.wp = (self.qh.pin_memory(), self.kh.pin_memory(),
+                                     self.wh.pin_memory())
+        self.e2e_bufs = []
+        h2d = d2h = 0
+        for c in self.calls:
+            b0, nb, r0, nr = c["rows"]
+            hq = self.qp[b0:b0 + nb, r0:r0 + nr]
+            hw = self.wp[b0:b0 + nb, r0:r0 + nr]
+            hk = self.kp[b0:b0 + nb]
+            bufs = dict(hq=hq, hw=hw, hk=hk,
+                        dq=torch.empty(hq.shape, dtype=hq.dtype, device=self.dev),
+                        dw=torch.empty(hw.shape, dtype=hw.dtype, device=self.dev),
+                        dk=torch.empty(hk.shape, dtype=hk.dtype, device=self.dev),
+                        hi=torch.empty(c["idx"].shape, dtype=torch.int32).pin_memory(),
+                        hs=torch.empty(c["sc"].shape, dtype=torch.float32).pin_memory())
+            h2d += sum(t.numel() * t.element_size() for t in (hq, hw, hk))
+            d2h += c["idx"].numel() * 4 + c["sc"].numel() * 4
+            self.e2e_bufs.append(bufs)
+        return h2d, d2h
+
+    def e2e_step(self):
+        B, p = self.B, self.p
+        for c, b in zip(self.calls, self.e2e_bufs):
+            b["dq"].copy_(b["hq"], non_blocking=True)
+            b["dk"].copy_(b["hk"], non_blocking=True)
+            b["dw"].copy_(b["hw"], non_blocking=True)
+            out = (c["idx"], c["sc"])
+            if self.kind in ROUTED:
+                self._routed(c, b["dq"], b["dk"], b["dw"], out)
+            else:
+                qq, kk, qs_, ks_ = b["dq"], b["dk"], None, None
+                if self.fp8:
+                    kk, ks_ = B.dsa_quantize_e4m3(b["dk"])
+                    if self.kind == "prefill":
+                        n = qq.shape[0] * qq.shape[1]
+                        q2, qs_ = B.dsa_quantize_e4m3(qq.reshape(n, -1))
+                        qq, qs_ = q2.reshape(b["dq"].shape), qs_.reshape(qq.shape[0], qq.shape[1])
+                B.dsa_index(qq, kk, b["dw"], p.topk, q_scale=qs_, k_scale=ks_, q_pos0=c["pos0"],
+                            k_len=c["klen"], out=out, workspace=self.ws, stream=self.stream)
+            b["hi"].copy_(c["idx"], non_blocking=True)
+            b["hs"].copy_(c["sc"], non_blocking=True)
+
+
+def timed(case, steps, warmup, world, dev, sample_clocks=False, local=0):
+    """W untimed steps, then K steps between barriers and device syncs, CUDA
+    events on the launching stream.  Returns (ms per layer max over ranks,
+    kernel ms per layer of this rank, clock summary)."""
+    import torch
+    import torch.distributed as dist
+    for _ in range(max(warmup, 3)):
+        case.step()
+    st = case.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {case.B.status_string(st)}")
+    torch.cuda.synchronize()
+    n = len(case.calls)
+    stage_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(n)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clk = ClockSampler(local) if sample_clocks else None
+    if clk:
+        clk.__enter__()
+    try:
+        t0.record(case.stream)
+        for i in range(steps):
+            case.step(stage_ev[i])
+        t1.record(case.stream)
+        torch.cuda.synchronize()
+    finally:
+        if clk:
+            clk.__exit__(None, None, None)
+    if world > 1:
+        dist.barrier()
+    st = case.status()
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {case.B.status_string(st)}")
+    elapsed = max_over_ranks(t0.elapsed_time(t1), dev)
+    kernel_ms = (sum(a.elapsed_time(b) for evs in stage_ev for a, b in evs) / steps
+                 if n else 0.0)
+    return elapsed / steps, kernel_ms, (clk.summary() if clk else None)
+
+
+def e2e_ms(case, steps, world, dev):
+    import torch
+    import torch.distributed as dist
+    h2d, d2h = case.e2e_setup()
+    case.e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(case.stream)
+    for _ in range(steps):
+        case.e2e_step()
+    e1.record(case.stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / steps, dev), h2d, d2h
+
+
+def roofline(case, name, ms_per_step, kernel_ms, long_region):
+    """Roofline of the dominant kernel: the scan (DSA prefill: tensor; decode: HBM)
+    or, for routed methods, the whole call (all its launches) as a lower bound."""
+    p, w, kind = case.p, case.w, case.kind
+    pk = peaks()
+    pairs, dots, flops = algorithmic_work(p, w)
+    bf16_peak = pk["bf16_sustained"] if long_region else pk["bf16"]
+    burst = "sustained" if long_region else "burst"
+    if kind == "decode":
+        nbytes = decode_bytes(p)
+        gbs = nbytes / (kernel_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": gbs / pk["hbm"], "peak_source": f"{pk['src']} copy bandwidth",
+                "work": f"{nbytes / 1e6:.1f} MB per launch (e4m3 K + scales + q + w)",
+                "kernel": "scan_kernel", "kernel_ms": kernel_ms}
+    elif kind == "prefill":
+        tf = flops / (kernel_ms * 1e-3) / 1e12
+        peak = 2.0 * bf16_peak if case.fp8 else bf16_peak
+        roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
+                "frac": tf / peak,
+                "peak_source": f"{pk['src']} bf16 {burst}"
+                               + (" x2 (fp8 nominal ratio)" if case.fp8 else ""),
+                "work": f"{flops / 1e12:.3f} TFLOP per launch (2*pairs*H*d)",
+                "kernel": "scan_kernel", "kernel_ms": kernel_ms}
+    else:
+        tf = flops / (kernel_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": tf, "peak": bf16_peak, "unit": "TFLOP/s",
+                "frac": tf / bf16_peak, "peak_source": f"{pk['src']} bf16 {burst}",
+                "work": f"{flops / 1e12:.3f} TFLOP per call ({dots} scored "
+                        "query-key-head dots x 2d, router and rerank included)",
+                "kernel": f"whole {kind} call ({case.launches} launches: pooling, router, "
+                          "scans, selects)", "kernel_ms": kernel_ms}
+    roof["traffic"] = measured_traffic(name) if kind in ("prefill", "decode") else None
+    return roof, dots
+
+
+def iou_rows(a_idx, b_idx, rows):
+    """Mean IoU of two top-k index sets over the listed rows (on the GPU)."""
+    import torch
+    topk = a_idx.shape[-1]
+    a_ = a_idx.reshape(-1, topk)[rows].sort(dim=1).values
+    b_ = b_idx.reshape(-1, topk)[rows].sort(dim=1).values
+    inter = torch.zeros(len(rows), device=a_.device)
+    for j in range(0, topk, 256):          # |A ∩ B| by membership of A's entries
+        blk = a_[:, j:j + 256]
+        pos = torch.searchsorted(b_, blk).clamp(max=topk - 1)
+        inter += ((torch.gather(b_, 1, pos) == blk) & (blk >= 0)).sum(1).float()
+    nv = (a_ >= 0).sum(1).float()
+    return (inter / (2 * nv - inter)).mean().item()
+
+
+def dense_reference(case):
+    """The exact DSA top-k of the same problem (GPU) and its time, for a routed
+    method's overlap and speed-up."""
+    import torch
+    B, p = case.B, case.p
+    prob = B.problem(case.q, case.k, p.topk)
+    dws = torch.empty(B.dsa_workspace_size(prob), dtype=torch.uint8, device=case.dev)
+    didx = torch.empty_like(case.idx)
+    dsc = torch.empty_like(case.sc)
+    B.dsa_index(case.q, case.k, case.wt, p.topk, out=(didx, dsc), workspace=dws)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(case.stream)
+    B.dsa_index(case.q, case.k, case.wt, p.topk, out=(didx, dsc), workspace=dws)
+    d1.record(case.stream)
+    torch.cuda.synchronize()
+    del dws
+    return didx, d0.elapsed_time(d1)
+
+
+def quality(case, name, ms_per_step, dense=None):
+    """Selection quality outside every timed region: needle recall at the probe
+    rows; for routed methods the IoU with the exact DSA top-k of the same rows
+    (both on the GPU) and the speed-up over that dense layer."""
+    import torch
+    p = case.p
+    out = {}
+    gi = case.idx.reshape(p.batch * p.n_q, p.topk)
+    if p.needles:
+        found = 0
+        for b, t, s_ in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
+            found += int((gi[b * p.n_q + t] == s_).any().item())
+        out["needle_recall"] = found / len(p.needles["s"])
+    if case.kind in ROUTED:
+        didx, dense_ms = dense if dense is not None else dense_reference(case)
+        rows = torch.linspace(p.n_q // 16, p.n_q - 1, 512).long().to(case.dev)
+        out.update({"iou_vs_dsa": iou_rows(case.idx, didx, rows), "dsa_ms": dense_ms,
+                    "speedup_vs_dsa": dense_ms / ms_per_step})
+    return out
+
+
+def secondary_line(name, steps, warmup, dev, cache):
+    """A secondary configuration timed in the same run (one GPU)."""
+    import torch
+    w = WORKLOADS[name]
+    key = (w["seed"], w["L"], w["H"], w.get("keys", "iid"), w["kind"] == "decode")
+    if key not in cache:
+        cache.clear()
+        torch.cuda.empty_cache()
+        cache[key] = make_problem(w)
+    p = cache[key]
+    case = Case(w, p, dev, 1, 0)
+    ms, kms, _ = timed(case, steps, warmup, 1, dev)
+    unit, scale = unit_of(w)
+    roof, dots = roofline(case, name, ms, kms, ms * steps > 1000.0)
+    dense = cache.get(("dense",) + key)
+    if case.kind in ROUTED and dense is None:
+        dense = dense_reference(case)
+        cache[("dense",) + key] = dense
+    q = quality(case, name, ms, dense)
+    line = {"workload": w["desc"], "value": ms * scale, "unit": unit, "ms_per_step": ms,
+            "steps": steps, "warmup": max(warmup, 3), "roofline": roof,
+            "scored_dots_per_s": dots / (ms * 1e-3), "gpu_launches": steps * case.launches}
+    if case.kind == "decode":
+        line["select_ms"] = ms - kms
+    else:
+        line["row_chunks"] = sum(c.get("chunks", 1) for c in case.calls)
+    line.update(q)
+    del case
+    torch.cuda.empty_cache()
+    return line
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="dsa_prefill_32k", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="dsa_prefill_128k", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="time only --workload (no secondary configurations)")
     args = ap.parse_args()
     w = WORKLOADS[args.workload]
     kind = w["kind"]
@@ -385,239 +762,66 @@ def main():
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    from sparse_attention_token_dsa_b200 import binding as B
+    dev = torch.device("cuda", local)
 
     p = make_problem(w)
-    dev = torch.device("cuda", local)
-    fp8 = w.get("fp8", False)
-
-    qh = torch.from_numpy(p.q.view(np.int16)).view(torch.bfloat16)
-    kh = torch.from_numpy(p.k.view(np.int16)).view(torch.bfloat16)
-    wh = torch.from_numpy(p.w)
-    q, k, wt = qh.to(dev), kh.to(dev), wh.to(dev)
-    q_scale = k_scale = None
-    if fp8:
-        k, k_scale = B.dsa_quantize_e4m3(k)
-        if kind == "prefill":
-            q2, q_scale = B.dsa_quantize_e4m3(q.reshape(p.batch * p.n_q, -1))
-            q = q2.reshape(p.q.shape)
-            q_scale = q_scale.reshape(p.batch, p.n_q)
-    torch.cuda.synchronize()
-    prob = B.problem(q, k, p.topk)
-    idx = torch.empty((p.batch, p.n_q, p.topk), dtype=torch.int32, device=dev)
-    sc = torch.empty((p.batch, p.n_q, p.topk), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
-
-    if kind in ROUTED:
-        algo = {"misa": B.DSA_ALGO_MISA, "dagger": B.DSA_ALGO_MISA_DAGGER,
-                "hisa": B.DSA_ALGO_HISA}[kind]
-        if kind == "hisa":
-            rp = B.route_params(misa_block=w["block"] if w["h"] else 0, misa_h=w["h"],
-                                hisa_block=w["hb"], hisa_r=w["r"])
-        else:
-            rp = B.route_params(misa_block=w["block"], misa_h=w["h"],
-                                k_prime=w.get("k_prime", 0))
-        ws = torch.empty(B.dsa_workspace_size(prob, algo, rp), dtype=torch.uint8, device=dev)
-        chunks = -(-p.n_q // B.dsa_route_chunk_rows(prob, algo, rp))
-        if kind == "misa":
-            per_call = 2 + 2 * chunks
-        elif kind == "dagger":
-            per_call = 2 + 4 * chunks
-        else:
-            per_call = (2 if w["h"] else 0) + 1 + 5 * chunks
-
-        def call(qq, kk, ww):
-            if kind == "misa":
-                B.misa_index(qq, kk, ww, p.topk, w["block"], w["h"], out=(idx, sc), workspace=ws)
-            elif kind == "dagger":
-                B.misa_dagger_index(qq, kk, ww, p.topk, w["block"], w["h"], w["k_prime"],
-                                    out=(idx, sc), workspace=ws)
-            else:
-                B.hisa_index(qq, kk, ww, p.topk, w["hb"], w["r"], route_h=w["h"],
-                             route_block=w["block"], out=(idx, sc), workspace=ws)
-
-        def step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            call(q, k, wt)
-            if ev is not None:
-                ev[1].record(stream)
-    else:
-        ws = torch.empty(B.dsa_workspace_size(prob), dtype=torch.uint8, device=dev)
-        per_call = 2 + (1 if (fp8 and kind == "decode") else 0)
-
-        def step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            B.dsa_index_scan(prob, q, k, wt, ws, q_scale=q_scale, k_scale=k_scale, stream=stream)
-            if ev is not None:
-                ev[1].record(stream)
-            B.dsa_index_select(prob, idx, sc, ws, stream=stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    st = B.dsa_read_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
-    torch.cuda.synchronize()
-
-    stage_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t0.record(stream)
-        for i in range(args.steps):
-            step(stage_ev[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    elapsed = t0.elapsed_time(t1)
-    stage_ms = statistics.mean(a.elapsed_time(b) for a, b in stage_ev)
-    st = B.dsa_read_status(ws)
-    if st != 0:
-        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
-    elapsed = max_over_ranks(elapsed, dev)
-
-    # end to end through the public call with host buffers (pinned), copies inside
-    qp, kp, wp = qh.pin_memory(), kh.pin_memory(), wh.pin_memory()
-    idx_h = torch.empty(idx.shape, dtype=torch.int32).pin_memory()
-    sc_h = torch.empty(sc.shape, dtype=torch.float32).pin_memory()
-    q_d = torch.empty_like(qh, device=dev)
-    k_d = torch.empty_like(kh, device=dev)
-    w_d = torch.empty_like(wh, device=dev)
-
-    def e2e_step():
-        q_d.copy_(qp, non_blocking=True)
-        k_d.copy_(kp, non_blocking=True)
-        w_d.copy_(wp, non_blocking=True)
-        if kind in ROUTED:
-            call(q_d, k_d, w_d)
-        else:
-            qq, kk, qs_, ks_ = q_d, k_d, None, None
-            if fp8:
-                kk, ks_ = B.dsa_quantize_e4m3(k_d)
-                if kind == "prefill":
-                    q2, qs_ = B.dsa_quantize_e4m3(q_d.reshape(p.batch * p.n_q, -1))
-                    qq, qs_ = q2.reshape(p.q.shape), qs_.reshape(p.batch, p.n_q)
-            B.dsa_index(qq, kk, w_d, p.topk, q_scale=qs_, k_scale=ks_, out=(idx, sc), workspace=ws)
-        idx_h.copy_(idx, non_blocking=True)
-        sc_h.copy_(sc, non_blocking=True)
-
+    case = Case(w, p, dev, world, rank)
+    ms_per_step, kernel_ms, clocks = timed(case, args.steps, args.warmup, world, dev,
+                                           sample_clocks=True, local=local)
     e2e_steps = max(3, min(args.steps, 10))
-    e2e_step()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    e2e_ms = max_over_ranks(e2e_ms, dev)
-    h2d = qh.numel() * qh.element_size() + kh.numel() * kh.element_size() + wh.numel() * 4
-    d2h = idx.numel() * 4 + sc.numel() * 4
+    e2e, h2d, d2h = e2e_ms(case, e2e_steps, world, dev)
+    # every rank's own kernel share is timed; the slowest rank sets the roofline
+    kernel_ms = max_over_ranks(kernel_ms, dev)
+    launches = case.launches * args.steps
+    qual = quality(case, args.workload, ms_per_step) if (rank == 0 and world == 1) else {}
 
-    # quality of the selection (outside every timed region): needle recall at the
-    # probe rows; for routed methods the overlap with the exact DSA top-k of the
-    # same rows (both on the GPU) and the dense layer's time for the speed-up
-    quality = {}
-    if rank == 0:
-        gi = idx.reshape(p.batch * p.n_q, p.topk)
-        if p.needles:
-            found = 0
-            for b, t, s_ in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
-                found += int((gi[b * p.n_q + t] == s_).any().item())
-            quality["needle_recall"] = found / len(p.needles["s"])
-        if kind in ROUTED:
-            dprob = B.problem(q, k, p.topk)
-            dws = torch.empty(B.dsa_workspace_size(dprob), dtype=torch.uint8, device=dev)
-            didx = torch.empty_like(idx)
-            dsc = torch.empty_like(sc)
-            B.dsa_index(q, k, wt, p.topk, out=(didx, dsc), workspace=dws)
-            d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            d0.record(stream)
-            B.dsa_index(q, k, wt, p.topk, out=(didx, dsc), workspace=dws)
-            d1.record(stream)
-            torch.cuda.synchronize()
-            dense_ms = d0.elapsed_time(d1)
-            rows = torch.linspace(p.n_q // 16, p.n_q - 1, 512).long().to(dev)
-            a_ = gi[rows].sort(dim=1).values
-            b_ = didx.reshape(-1, p.topk)[rows].sort(dim=1).values
-            inter = torch.zeros(len(rows), device=dev)
-            for j in range(0, p.topk, 256):          # |A ∩ B| by membership of A's entries
-                blk = a_[:, j:j + 256]
-                pos = torch.searchsorted(b_, blk).clamp(max=p.topk - 1)
-                inter += ((torch.gather(b_, 1, pos) == blk) & (blk >= 0)).sum(1).float()
-            nv = (a_ >= 0).sum(1).float()
-            iou = (inter / (2 * nv - inter)).mean().item()
-            quality.update({"iou_vs_dsa": iou, "dsa_ms": dense_ms,
-                            "speedup_vs_dsa": dense_ms / (elapsed / args.steps)})
-            del dws
-
+    line = None
     if rank == 0:
         unit, scale = unit_of(w)
-        ms_per_step = elapsed / args.steps
-        value = ms_per_step / world * scale
-        pk = peaks()
-        pairs, dots, flops = algorithmic_work(p, w)
-        long_region = elapsed > 1000.0
-        bf16_peak = pk["bf16_sustained"] if long_region else pk["bf16"]
-        burst = "sustained" if long_region else "burst"
-        if kind == "decode":
-            nbytes = decode_bytes(p)
-            gbs = nbytes / (stage_ms * 1e-3) / 1e9
-            roof = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm"], "unit": "GB/s",
-                    "frac": gbs / pk["hbm"], "peak_source": f"{pk['src']} copy bandwidth",
-                    "work": f"{nbytes / 1e6:.1f} MB per launch (e4m3 K + scales + q + w)",
-                    "kernel": "scan_kernel", "kernel_ms": stage_ms}
-        elif kind == "prefill":
-            tf = flops / (stage_ms * 1e-3) / 1e12
-            peak = 2.0 * bf16_peak if fp8 else bf16_peak
-            roof = {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s",
-                    "frac": tf / peak,
-                    "peak_source": f"{pk['src']} bf16 {burst}"
-                                   + (" x2 (fp8 nominal ratio)" if fp8 else ""),
-                    "work": f"{flops / 1e12:.3f} TFLOP per launch (2*pairs*H*d)",
-                    "kernel": "scan_kernel", "kernel_ms": stage_ms}
-        else:
-            tf = flops / (stage_ms * 1e-3) / 1e12
-            roof = {"bound": "tensor", "achieved": tf, "peak": bf16_peak, "unit": "TFLOP/s",
-                    "frac": tf / bf16_peak, "peak_source": f"{pk['src']} bf16 {burst}",
-                    "work": f"{flops / 1e12:.3f} TFLOP per call ({dots} scored "
-                            "query-key-head dots x 2d, router and rerank included)",
-                    "kernel": f"whole {kind} call ({per_call} launches: pooling, router, "
-                              "scans, selects)", "kernel_ms": stage_ms}
-        tr = TRAFFIC.get(args.workload)
-        roof["traffic"] = tr["bytes"] if tr and tr["src"] == kernel_hash() else None
+        roof, dots = roofline(case, args.workload, ms_per_step, kernel_ms,
+                              ms_per_step * args.steps > 1000.0)
+        par = (f"{world} ranks, one layer partitioned by "
+               + ("sequences" if kind == "decode" else "zigzag query-row chunks")
+               + ", no data-path collective") if world > 1 else "single GPU"
         cfg = {"workload": w["desc"], "l2": "inputs larger than L2 (no flush)",
-               "parallelism": f"replicas x{world}",
-               "scored_dots_per_s": dots / (ms_per_step * 1e-3)}
+               "parallelism": par, "scored_dots_per_s": dots / (ms_per_step * 1e-3)}
         if kind in ("prefill", "decode"):
-            cfg["select_ms"] = ms_per_step - stage_ms
+            cfg["select_ms"] = ms_per_step - kernel_ms
         else:
-            cfg["row_chunks"] = chunks
-        cfg.update(quality)
-        line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world,
+            cfg["row_chunks"] = sum(c.get("chunks", 1) for c in case.calls)
+        cfg.update(qual)
+        line = {"metric": METRIC, "value": ms_per_step * scale, "unit": unit, "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-                "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-                "dtype": "e4m3/f32" if fp8 else "bf16/f32", "data": "synthetic",
-                "config": cfg,
-                "roofline": roof,
-                "e2e": {"value": e2e_ms / world * scale, "unit": unit, "h2d_bytes_per_step": h2d,
+                "higher_is_better": False, "scaling": "strong" if world > 1 else "weak",
+                "vs_baseline": None, "dtype": "e4m3/f32" if case.fp8 else "bf16/f32",
+                "data": "synthetic", "config": cfg, "roofline": roof,
+                "e2e": {"value": e2e * scale, "unit": unit, "h2d_bytes_per_step": h2d,
                         "d2h_bytes_per_step": d2h},
-                "gpu_launches": args.steps * per_call,
-                "clocks": clk.summary()}
-        if world == 1 and not args.no_cpu_baseline:
+                "gpu_launches": launches, "clocks": clocks}
+    dense = None
+    if world == 1 and case.kind == "prefill" and not case.fp8:
+        dense = (case.idx.clone(), ms_per_step)     # exact DSA of this problem
+    del case
+    torch.cuda.empty_cache()
+
+    if world == 1 and rank == 0:
+        if not args.no_secondary and args.workload == "dsa_prefill_128k":
+            cache = {(w["seed"], w["L"], w["H"], w.get("keys", "iid"), False): p}
+            if dense is not None:
+                cache[("dense", w["seed"], w["L"], w["H"], w.get("keys", "iid"), False)] = dense
+            line["secondary"] = [secondary_line(n, min(args.steps, 5), args.warmup, dev, cache)
+                                 for n in SECONDARY]
+            line["gpu_launches"] += sum(s["gpu_launches"] for s in line["secondary"])
+            cache.clear()
+        if not args.no_cpu_baseline:
             cb = cpu_baseline(p, w)
+            unit, scale = unit_of(w)
             line["cpu_baseline"] = {"value": cb["layer_ms"] * scale, "unit": unit,
                                     "cores": cb["omp"], "kind": "oracle",
                                     "sample": f"{cb['rows']} random query rows "
                                               f"({cb['pairs']} causal pairs, {cb['wall_s']:.1f} s"
                                               "), extrapolated by causal pair count"}
+    if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -164,7 +164,14 @@ int dsa_index(const dsa_problem* p, const void* q, const float* q_scale, const v
  * capture).  Every call on a device shares the one scratch array, so calls
  * whose executions overlap on the GPU (different streams, no ordering between
  * them) race and corrupt each other's results; order them on one stream or
- * with events.  Other arguments and results are as for dsa_index. */
+ * with events.  The scratch address is looked up once per device and kept, so
+ * the library must not be used on a device again after cudaDeviceReset there.
+ * A device-side status (a bounded wait that expired, or a bad scale or length
+ * under DSA_FLAG_CHECK) is recorded in that scratch, which the caller cannot
+ * read with dsa_read_status: pass DSA_FLAG_CHECK to have the call synchronise
+ * the stream and return the device status itself (without it an expired wait
+ * shows only as padded output rows).  Other arguments and results are as for
+ * dsa_index. */
 int dsa_index_noalloc(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
                       const float* k_scale, const float* w, int32_t* out_idx, float* out_score,
                       void* stream);

@@ -293,7 +293,7 @@ struct OutMap {
 
 cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint64_t* logs,
                             const int32_t* cnt, const unsigned long long* thr, int32_t* out_idx,
-                            float* out_score, OutMap om, cudaStream_t st) {
+                            float* out_score, OutMap om, const int32_t* status, cudaStream_t st) {
   FinalArgs f{};
   f.rows = pl.rows;
   f.nq_c = om.nq_c;
@@ -312,6 +312,7 @@ cudaError_t launch_finalize(const ScanPlan& pl, int topk, int sorted, const uint
   f.log_thr = thr;
   f.out_idx = out_idx;
   f.out_score = out_score;
+  f.status = status;
   if (pl.C == 1 && sc <= 2048) {
     // one key chunk per row: about k candidates; up to four rows per CTA
     const int stage_cap = sc + sc / 2;
@@ -430,7 +431,9 @@ int finish(const dsa_problem* p, void* ws, cudaStream_t st) {
 // Scratch of dsa_index_noalloc: a fixed 64 MiB array in device memory that
 // every GPU loading this library holds until the process exits.  Host code
 // must not use the name as an address; the device address comes from
-// cudaGetSymbolAddress, taken once per device with that device current.
+// cudaGetSymbolAddress, taken once per device with that device current and
+// kept for the life of the process (a cudaDeviceReset would reload the module
+// and could move it; the header rules that use out).
 constexpr size_t kNoAllocScratchBytes = 64ull << 20;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -931,7 +934,8 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
   if (launch_finalize(pl, p->topk, sorted, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
                       reinterpret_cast<const int32_t*>(ws + L.off_cnt),
                       reinterpret_cast<const unsigned long long*>(ws + L.off_thr), out_idx,
-                      out_score, OutMap{p->n_q, p->n_q, 0}, st) != cudaSuccess)
+                      out_score, OutMap{p->n_q, p->n_q, 0}, reinterpret_cast<const int32_t*>(ws),
+                      st) != cudaSuccess)
     return DSA_ERR_CUDA;
   return finish(p, workspace, st);
 }
@@ -1000,7 +1004,7 @@ int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
     rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
     if (rc != DSA_OK) return rc;
     if (launch_finalize(rs.s1, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
-                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+                        OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return finish(p, workspace, st);
@@ -1040,7 +1044,7 @@ int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const vo
     rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
     if (rc != DSA_OK) return rc;
     if (launch_finalize(rs.s1, L.c.kp, 0, lp.logs, lp.cnt, lp.thr, pool, nullptr,
-                        OutMap{nq, nq, 0}, st) != cudaSuccess)
+                        OutMap{nq, nq, 0}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
     if (out_pool) {
       rc = copy_lists(out_pool, pool, p, q_off, nq, L.c.kp, st);
@@ -1063,7 +1067,7 @@ int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const vo
     rc = run_stage(p, rs.s2, io2, q_off, nq, lp, status, st);
     if (rc != DSA_OK) return rc;
     if (launch_finalize(rs.s2, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
-                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+                        OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return finish(p, workspace, st);
@@ -1136,7 +1140,7 @@ int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
     boundary_candidate_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(ba);
     if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
     if (launch_finalize(rs.s1, c.r, 0, lp.logs, lp.cnt, lp.thr, blocks, nullptr,
-                        OutMap{nq, nq, 0}, st) != cudaSuccess)
+                        OutMap{nq, nq, 0}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
     if (out_blocks) {
       rc = copy_lists(out_blocks, blocks, p, q_off, nq, c.r, st);
@@ -1160,7 +1164,7 @@ int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
     rc = run_stage(p, rs.s2, io2, q_off, nq, lp, status, st);
     if (rc != DSA_OK) return rc;
     if (launch_finalize(rs.s2, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
-                        OutMap{nq, p->n_q, q_off}, st) != cudaSuccess)
+                        OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
   return finish(p, workspace, st);

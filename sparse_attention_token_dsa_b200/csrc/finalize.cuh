@@ -34,6 +34,8 @@ struct FinalArgs {
   int32_t q_off;         // row i of sequence b writes output row b * nq_total + q_off + i
   int32_t* out_idx;      // [batch * nq_total, topk]
   float* out_score;      // [batch * nq_total, topk] or null
+  const int32_t* status; // workspace status word: a failed scan leaves its logs
+                         //   unfinished, and the rows are then written as padding
 };
 
 constexpr int kFinBoundary = 1024;  // boundary-bin capacity per row group
@@ -80,12 +82,16 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
   int* segn = segn_all[grp];
   unsigned long long* segt = segt_all[grp];
   const int nseg = a.C * a.nsub;
+  // after a device error (a scan that gave up on a wait) the logs and their
+  // fills are not this call's: read none of them, write the padding
+  const bool failed = *reinterpret_cast<const volatile int32_t*>(a.status) != DSA_OK;
   for (int g = tid; g < nseg; g += NT) {
     const int c = g / a.nsub, sb = g % a.nsub;
     const int64_t rs = (int64_t)row * a.C + c;
     segp[g] = a.logs + (rs * a.nsub + sb) * a.capw;
-    segn[g] = a.log_cnt[rs * a.nsub + sb];
-    segt[g] = a.log_thr[rs];
+    const int n = failed ? 0 : a.log_cnt[rs * a.nsub + sb];
+    segn[g] = n < 0 ? 0 : (n > a.capw ? a.capw : n);
+    segt[g] = failed ? 0ull : a.log_thr[rs];
   }
   for (int i = tid; i < 256; i += NT) G->sc.hist[i] = 0;
   if (tid == 0) {

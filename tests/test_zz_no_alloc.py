@@ -12,6 +12,8 @@ import ctypes as C
 import numpy as np
 import pytest
 
+import oracle
+import parity
 from sparse_attention_token_dsa_b200 import inputs as gen
 
 pytestmark = pytest.mark.gpu
@@ -68,6 +70,21 @@ def test_noalloc_matches_dsa_index_on_two_calls(B, kind):
         assert rc == B.DSA_OK, B.status_string(rc)
         assert np.array_equal(gi, ref_i)
         assert np.array_equal(gs, ref_s)   # same kernels: identical to the last bit
+    # with DSA_FLAG_CHECK the call reads the device status from its own scratch
+    # (the caller cannot) and returns it: a clean run reports DSA_OK
+    rc, gi, gs = _call_noalloc(B, p, q, k, w, pos0, klen, flags | B.DSA_FLAG_CHECK)
+    assert rc == B.DSA_OK, B.status_string(rc)
+    assert np.array_equal(gi, ref_i) and np.array_equal(gs, ref_s)
+    # and the oracle agrees with both
+    oracle.build()
+    inp = oracle.Inputs(p)
+    ri, rs, rs64, _ = oracle.dsa(inp, p.topk)
+    gi, gs = gi.reshape(-1, p.topk), gs.reshape(-1, p.topk)
+    if kind == "integer":
+        parity.exact(gi, gs, ri, rs)
+    else:
+        r = parity.within_tolerance(inp, np.arange(p.batch * p.n_q), gi, gs, ri, rs64, 1e-3)
+        assert r.iou > 0.99
 
 
 def test_noalloc_refuses_problems_beyond_its_scratch(B):
