@@ -60,6 +60,16 @@ WORKLOADS = {
         desc="DSA indexer prefill, batch 1, L=8192 causal, H_I=64, d=128, top-k=2048, bf16 "
              "(small case of the 32K workload, sized for ncu captures)",
         kind="prefill", batch=1, L=8192, H=64, topk=2048, fp8=False, seed=2, needles=8),
+    "dsa_prefill_16k": dict(
+        desc="DSA indexer prefill, batch 1, L=16384 causal, H_I=64, d=128, top-k=2048, bf16 "
+             "(small case of the 128K workload, sized for ncu captures)",
+        kind="prefill", batch=1, L=16384, H=64, topk=2048, fp8=False, seed=2, needles=0),
+    "misa_dagger_prefill_16k": dict(
+        desc="MISA-dagger prefill, batch 1, L=16384 causal, H_I=64, d=128, B=1024, h=8, "
+             "k'=8192, top-k=2048, bf16 (small case of the 128K workload, sized for ncu "
+             "captures)",
+        kind="dagger", batch=1, L=16384, H=64, topk=2048, seed=4, block=1024, h=8,
+        k_prime=8192),
     "dsa_decode_128k": dict(
         desc="DSA indexer decode, 32 sequences x 131072 cached keys, one query each, H_I=64, "
              "d=128, e4m3 K with per-token fp32 scale, bf16 q, fp32 w, top-k=2048",
