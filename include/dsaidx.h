@@ -87,7 +87,9 @@ enum {
   DSA_ERR_WORKSPACE = -3,    /* workspace NULL or smaller than dsa_workspace_size() */
   DSA_ERR_CUDA = -4,         /* a CUDA runtime call or launch failed */
   DSA_ERR_NONFINITE = -5,    /* a scale is NaN, inf, zero or negative (DSA_FLAG_CHECK) */
-  DSA_ERR_TIMEOUT = -6       /* a bounded device-side wait expired */
+  DSA_ERR_TIMEOUT = -6,      /* a bounded device-side wait expired */
+  DSA_ERR_INTERNAL = -7      /* a device-side capacity or bounds check failed (a library
+                                fault; the outputs of that call are not to be used) */
 };
 
 typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
@@ -98,6 +100,13 @@ enum { DSA_ALGO_DSA = 0, DSA_ALGO_MISA = 1, DSA_ALGO_MISA_DAGGER = 2, DSA_ALGO_H
 /* problem.flags */
 #define DSA_FLAG_CHECK 1u  /* validate scales/lengths on device, synchronise, return device status */
 #define DSA_FLAG_SORTED 2u /* order each row's top-k by (score desc, index asc) */
+/* For tests of the timeout path only, never in production: dsa_index /
+ * dsa_index_scan run with a wait budget of about 1 ms instead of about 4 s, and
+ * the scan's first CTA withholds one stage of keys, so its bounded waits run
+ * out.  The call then records DSA_ERR_TIMEOUT, every role of that CTA drains
+ * its own copies and MMAs and exits, the select writes padding rows, and the
+ * GPU context stays usable for the next call. */
+#define DSA_FLAG_TEST_STALL 0x80000000u
 
 typedef struct {
   int32_t batch;          /* sequences */

@@ -16,11 +16,12 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdsaidx.so")
 
 DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE = 0, -1, -2, -3
-DSA_ERR_CUDA, DSA_ERR_NONFINITE, DSA_ERR_TIMEOUT = -4, -5, -6
+DSA_ERR_CUDA, DSA_ERR_NONFINITE, DSA_ERR_TIMEOUT, DSA_ERR_INTERNAL = -4, -5, -6, -7
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
 DSA_ALGO_DSA, DSA_ALGO_MISA, DSA_ALGO_MISA_DAGGER, DSA_ALGO_HISA = 0, 1, 2, 3
 DSA_FLAG_CHECK = 1
 DSA_FLAG_SORTED = 2
+DSA_FLAG_TEST_STALL = 0x80000000   # tests of the timeout path only (see include/dsaidx.h)
 
 
 class DsaProblem(C.Structure):

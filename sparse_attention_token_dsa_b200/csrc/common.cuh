@@ -28,6 +28,9 @@ __device__ __forceinline__ void set_status(int32_t* st, int32_t code, int32_t wh
 // Bounded waits: every spin gives up after kWaitCycles SM clocks (about four
 // seconds), far beyond any legitimate wait in these kernels.
 constexpr long long kWaitCycles = 8000000000ll;
+// Wait budget under DSA_FLAG_TEST_STALL (tests of the timeout path): about a
+// millisecond, far above any wait of a healthy run of the small test problems.
+constexpr long long kTestWaitCycles = 2000000ll;
 
 // -------------------------------------------------------------- smem utils --
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -74,14 +77,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // spent (records DSA_ERR_TIMEOUT and raises *abort) or as soon as another role
 // raised *abort; returns false in both cases.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int32_t* status, int where) {
+                                          int32_t* status, int where,
+                                          long long budget = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15) == 0) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > budget) {
         *abort = 1;
         set_status(status, DSA_ERR_TIMEOUT, where);
         return false;
@@ -90,10 +94,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 // Same budget, no abort flag: used to drain this CTA's own copies in flight.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity,
+                                                long long budget = kWaitCycles) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > budget) return false;
   return true;
 }
 
@@ -197,6 +202,40 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t smem_addr) {
   d |= (uint64_t)1 << 46;
   d |= (uint64_t)2 << 61;
   return d;
+}
+
+// The same descriptor split into its two 32-bit words: the low word holds the
+// start address (addr >> 4, 14 bits) and the leading offset; the high word is
+// the same constant for every operand of this layout.  Advancing an operand
+// then costs one 32-bit add on the low word (shared addresses stay below
+// 2^18, so the address field never carries into the leading offset).
+constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
+__device__ __forceinline__ uint32_t sdesc_lo(uint32_t smem_addr) {
+  return ((smem_addr >> 4) & 0x3FFFu) | (1u << 16);
+}
+// tcgen05.mma from split descriptors; ACC (compile-time) selects accumulate.
+template <MmaKind K, int ACC>
+__device__ __forceinline__ void tc_mma_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
+                                          uint32_t idesc) {
+  if constexpr (K == MmaKind::BF16) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
+  } else if constexpr (K == MmaKind::TF32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
+  }
 }
 
 // 32 lanes x 32 consecutive fp32 columns per thread.

@@ -676,6 +676,8 @@ int run_stage(const dsa_problem* p, const ScanPlan& pl, const StageIO& io, int q
   a.log_cnt = lp.cnt;
   a.log_thr = lp.thr;
   a.status = status;
+  a.wait_cycles = kWaitCycles;
+  a.test_stall = 0;
   return launch_scan(pl, qm, km, a, st, io.gather) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -794,6 +796,7 @@ const char* dsa_status_string(int32_t s) {
     case DSA_ERR_CUDA: return "CUDA runtime error or launch failure";
     case DSA_ERR_NONFINITE: return "non-finite, zero or negative scale";
     case DSA_ERR_TIMEOUT: return "a bounded device wait expired";
+    case DSA_ERR_INTERNAL: return "a device-side capacity or bounds check failed";
     default: return "unknown status";
   }
 }
@@ -915,6 +918,9 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.log_cnt = reinterpret_cast<int32_t*>(ws + L.off_cnt);
   a.log_thr = reinterpret_cast<unsigned long long*>(ws + L.off_thr);
   a.status = status;
+  const bool stall = (p->flags & DSA_FLAG_TEST_STALL) != 0;
+  a.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
+  a.test_stall = stall ? 1 : 0;
   if (launch_scan(pl, qm, km, a, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }

@@ -83,6 +83,9 @@ struct ScanArgs {
   int32_t* log_cnt;      // [rows * C][nsub]
   unsigned long long* log_thr;  // [rows * C] final threshold of the slot
   int32_t* status;       // workspace status word
+  long long wait_cycles; // budget of every bounded wait (kWaitCycles; shorter in tests)
+  int32_t test_stall;    // DSA_FLAG_TEST_STALL: CTA 0 withholds the second K stage of
+                         //   its first item, so the waits on it run out (tests only)
 };
 
 constexpr int kEpiWarps = 8;
@@ -229,6 +232,8 @@ struct FilterCtx {
   uint32_t row_stride;   // entries between consecutive rows' sub-logs
   uint32_t* hist;
   ScanSmemTail* T;
+  int capw;              // sub-log capacity (a write past it is recorded, not made)
+  int32_t* status;
 };
 
 // Legality, composite key, threshold filter and append for one query row.
@@ -246,6 +251,11 @@ __device__ __forceinline__ void filter_append(const FilterCtx& f, int r, float a
   if (bal) {
     int* cnt = &T->subcnt[r][f.sub];
     const int base = *cnt;
+    if (base + __popc(bal) > f.capw) {
+      // cannot happen while compaction keeps its slack; never write past the log
+      if (f.lane == 0) set_status(f.status, DSA_ERR_INTERNAL, 110);
+      return;
+    }
     if (surv) {
       f.logs[(uint32_t)r * f.row_stride + (uint32_t)(base + __popc(bal & f.lanemask_lt))] = comp;
       uint32_t* h = f.hist + r * kHistWords;
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       ItemGeom g = item_geom<GATHER>(a, item);
       if (g.ntiles == 0) continue;
       if (lane == 0) {
-        ok = mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1);
+        ok = mbar_wait(&T->q_empty, (it & 1) ^ 1, abort, a.status, 1, a.wait_cycles);
         if (ok) {
           mbar_arrive_expect_tx(&T->q_full, q_bytes);
           // split-query rows: the hi parts of all rows come first, then the lo parts
@@ -577,11 +587,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         // list entries of this tile (loaded before the wait so their latency overlaps it)
         int rr[4] = {0, 0, 0, 0};
         int ybox = -1;
+        // list entries outside [-1, n_k) (never written by this library's own
+        // selects) are recorded and read as empty slots
         if constexpr (GATHER == 1) {
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int e = t * 128 + lane * 4 + j;
-            const int kk = e < a.klist_len ? lst[e] : -1;
+            int kk = e < a.klist_len ? lst[e] : -1;
+            if (kk < -1 || kk >= a.n_k) {
+              set_status(a.status, DSA_ERR_INTERNAL, 111);
+              kk = -1;
+            }
             rr[j] = krow0 + (kk >= 0 ? kk : 0);
           }
         } else if constexpr (GATHER == 2) {
@@ -590,18 +606,29 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           if (lane < 128 / box) {
             const int e = t * 128 + lane * box;            // token slot in the row's list
             const int slot_b = e >> a.lb_shift;
-            const int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
+            int blk = slot_b < a.klist_len ? lst[slot_b] : -1;
+            if (blk < -1 || (long long)blk * bs >= a.n_k) {
+              set_status(a.status, DSA_ERR_INTERNAL, 112);
+              blk = -1;
+            }
             ybox = krow0 + (blk >= 0 ? blk * bs + (e & (bs - 1)) : 0);
           }
         }
         // tiles of this stage inside the item (a ragged last stage loads one)
         const int nvalid = kPairs ? min(KT, g.ntiles - t * KT) : 1;
+        // DSA_FLAG_TEST_STALL: this stage is counted but never loaded, so the MMA
+        // warp's bounded wait on it runs out and the abort path runs
+        const bool stall = GATHER == 0 && a.test_stall && blockIdx.x == 0 && it == 1 && t == 1;
         if (lane == 0) {
-          ok = mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2);
-          if (ok) mbar_arrive_expect_tx(&T->k_full[slot], nvalid * Cfg::KTILE_BYTES);
+          ok = mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2, a.wait_cycles);
+          if (ok && !stall) mbar_arrive_expect_tx(&T->k_full[slot], nvalid * Cfg::KTILE_BYTES);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
+        if (stall) {
+          ++kcount;
+          continue;
+        }
         if constexpr (GATHER == 0) {
           if (lane == 0) {
             for (int j = 0; j < nvalid; ++j) {
@@ -630,9 +657,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     }
     if (lane == 0 && *abort) {
       // abort path: let this CTA's own copies in flight land before exit
-      if (it > 0) mbar_wait_drain(&T->q_full, (it - 1) & 1);
+      if (it > 0) mbar_wait_drain(&T->q_full, (it - 1) & 1, a.wait_cycles);
       for (uint32_t i = kcount > (uint32_t)KS ? kcount - KS : 0; i < kcount; ++i)
-        mbar_wait_drain(&T->k_full[i % KS], (i / KS) & 1);
+        mbar_wait_drain(&T->k_full[i % KS], (i / KS) & 1, a.wait_cycles);
     }
   } else if (warp == kMmaWarp) {
     // ----------------------------------------------------------------- MMA --
@@ -647,7 +674,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         if (item >= a.n_items) break;
         ItemGeom g = item_geom<GATHER>(a, item);
         if (g.ntiles == 0) continue;
-        if (!mbar_wait(&T->q_full, it & 1, abort, a.status, 3)) break;
+        if (!mbar_wait(&T->q_full, it & 1, abort, a.status, 3, a.wait_cycles)) break;
         ++it;
         tc_fence_after();
         const int nunits = (g.ntiles + KT - 1) / KT * a.G;
@@ -655,26 +682,31 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const int gg = u & (a.G - 1);
           const int slot = kcount % KS;
           if (gg == 0) {
-            if (!mbar_wait(&T->k_full[slot], (kcount / KS) & 1, abort, a.status, 4)) { ok = false; break; }
+            if (!mbar_wait(&T->k_full[slot], (kcount / KS) & 1, abort, a.status, 4, a.wait_cycles)) { ok = false; break; }
           }
           const int s = ucount % NS;
-          if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5)) { ok = false; break; }
+          if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5, a.wait_cycles)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t qbase = smem_u32(Qs + gg * Cfg::A * qcols * 128);
+          // descriptor low words: one add per MMA (32 bytes of K per k-step = 2)
+          const uint32_t qlo = sdesc_lo(smem_u32(Qs + gg * Cfg::A * qcols * 128));
           // one accumulator block of ncols columns per key tile of the stage
           const int nvalid = kPairs ? min(KT, g.ntiles - (u / a.G) * KT) : 1;
           for (int j = 0; j < nvalid; ++j) {
             const uint32_t d = tmem_base + s * a.stage_cols + j * ncols;
-            const uint32_t kbase = smem_u32(Ks + (slot * KT + j) * Cfg::A * 16384);
+            const uint32_t klo = sdesc_lo(smem_u32(Ks + (slot * KT + j) * Cfg::A * 16384));
 #pragma unroll
             for (int at = 0; at < Cfg::A; ++at) {
+              const uint32_t qat = qlo + (uint32_t)(at * qcols * 8);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t ad = make_sdesc(kbase + at * 16384 + kk * 32);
+                const uint32_t alo = klo + (uint32_t)(at * 1024 + kk * 2);
 #pragma unroll
                 for (int pt = 0; pt < PARTS; ++pt) {
-                  const uint64_t bd = make_sdesc(qbase + (at * qcols + pt * ncols) * 128 + kk * 32);
-                  tc_mma<KIND>(d, ad, bd, idesc, (at | kk | pt) != 0);
+                  const uint32_t blo = qat + (uint32_t)(pt * ncols * 8 + kk * 2);
+                  if (at == 0 && kk == 0 && pt == 0)
+                    tc_mma_lo<KIND, 0>(d, alo, blo, idesc);
+                  else
+                    tc_mma_lo<KIND, 1>(d, alo, blo, idesc);
                 }
               }
             }
@@ -692,7 +724,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       if (!ok) {
         // abort path: wait for the MMAs already issued before TMEM is freed
         tc_commit(&T->drain);
-        mbar_wait_drain(&T->drain, 0);
+        mbar_wait_drain(&T->drain, 0, a.wait_cycles);
       }
     }
   } else if constexpr (GATHER != 0) {
@@ -748,7 +780,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         const int e = u * 128 + quad * 32 + lane;
         const int key = key_next;
         if (u + 2 < g.ntiles) key_next = key_at(u + 2);
-        const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
+        const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6, a.wait_cycles);
         __syncwarp();
         if (!__all_sync(0xffffffffu, got)) continue;
         tc_fence_after();
@@ -1001,7 +1033,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             ks1 = ks_next1;
             if (KT > 1 && uu + ustep < nunits) ks_next1 = ks_at1(uu + ustep);
           }
-          const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6);
+          const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6, a.wait_cycles);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
           tc_fence_after();
@@ -1022,6 +1054,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
                          key - (int)(quad * 32 + lane) + 127 - g.kbeg < T->item_min_nleg;
           fc.hist = hist;
           fc.T = T;
+          fc.capw = a.capw;
+          fc.status = a.status;
           if constexpr (HT >= 32) {
             if (qhalf == 2)
               unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);

@@ -50,7 +50,7 @@ def _prob(bind, **kw):
 
 
 def test_status_strings(bind):
-    for s in (0, -1, -2, -3, -4, -5, -6):
+    for s in (0, -1, -2, -3, -4, -5, -6, -7):
         assert bind.status_string(s) and bind.status_string(s) != "unknown status"
     assert bind.status_string(-99) == "unknown status"
 

@@ -261,3 +261,40 @@ def test_check_flag_reports_bad_scale(B):
         B.dsa_index(qc, kc, dev(p.w), p.topk, q_scale=qs, k_scale=ks, flags=B.DSA_FLAG_CHECK)
     assert e.value.status == B.DSA_ERR_NONFINITE
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ failure path --
+
+def test_expired_wait_returns_timeout_then_next_call_is_exact(B):
+    """DSA_FLAG_TEST_STALL makes the first CTA withhold one stage of keys and
+    shortens every bounded wait to about a millisecond: the wait on that stage
+    runs out, the call returns DSA_ERR_TIMEOUT within a fraction of a second,
+    the select writes padding rows, and the next call on the same stream and
+    workspace is bit-exact.  Nothing traps or hangs: every role drains its own
+    copies and MMAs and exits."""
+    import time
+    import torch
+    p = gen.integer_problem(8, 1, 1024, 1024, 64, 128, 128, dtype=gen.BF16)
+    q, k, w = dev(p.q), dev(p.k), dev(p.w)
+    prob = B.problem(q, k, p.topk)
+    ws = torch.empty(B.dsa_workspace_size(prob), dtype=torch.uint8, device="cuda")
+    idx = torch.full((1, p.n_q, p.topk), 7, dtype=torch.int32, device="cuda")
+    sc = torch.full((1, p.n_q, p.topk), 7.0, dtype=torch.float32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with pytest.raises(B.DsaError) as e:
+        B.dsa_index(q, k, w, p.topk, flags=B.DSA_FLAG_CHECK | B.DSA_FLAG_TEST_STALL,
+                    out=(idx, sc), workspace=ws)
+    took = time.perf_counter() - t0
+    assert e.value.status == B.DSA_ERR_TIMEOUT
+    assert took < 1.0, f"the failed call took {took:.3f} s"
+    assert B.dsa_read_status(ws) == B.DSA_ERR_TIMEOUT
+    assert torch.all(idx == -1).item() and torch.all(torch.isneginf(sc)).item()
+    # the same stream and workspace, a normal call: exact
+    B.dsa_index(q, k, w, p.topk, flags=B.DSA_FLAG_CHECK | B.DSA_FLAG_SORTED, out=(idx, sc),
+                workspace=ws)
+    torch.cuda.synchronize()
+    assert B.dsa_read_status(ws) == B.DSA_OK
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(idx.cpu().numpy().reshape(-1, p.topk), sc.cpu().numpy().reshape(-1, p.topk),
+                 ri, rs)
