@@ -67,6 +67,10 @@ def lib():
                                        vp, vp, vp, vp]
         _lib.orc_block_scores.restype = C.c_int64
         _lib.orc_block_scores.argtypes = [vp, i64, i32, vp, i32, vp]
+        _lib.orc_lisa_rows.argtypes = [vp, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp]
+        _lib.orc_resmisa_rows.argtypes = [vp, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp, vp]
+        _lib.orc_residual_bounds.restype = C.c_int64
+        _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_score_row.restype = C.c_int64
         _lib.orc_score_row.argtypes = [vp, i64, vp, i32, vp]
     return _lib
@@ -160,6 +164,48 @@ def hisa(inp: Inputs, topk: int, block: int, r: int, route_h: int = 0, route_blo
                              _p(out["blocks"]), _p(out["J"]), _p(out["heads"]), _p(out["dots"]))
     assert rc == 0
     return out
+
+
+def lisa(inp: Inputs, topk: int, pool_m: int = 0, rows=None, forced_pool=None):
+    """Indexer LISA (pool_m == 0: tokens ranked by the linear term l = g . k) or
+    LISA-dagger (pool_m > 0: top-pool_m by l reranked by the full I).
+    Returns dict(idx, score, score64, pool, dots)."""
+    rows = _rows(inp.prob, rows)
+    n = len(rows)
+    out = dict(idx=np.empty((n, topk), np.int32), score=np.empty((n, topk), np.float32),
+               score64=np.empty((n, topk), np.float64), dots=np.empty(n, np.int64),
+               pool=np.empty((n, pool_m), np.int32) if pool_m > 0 else None)
+    fp = None if forced_pool is None else np.ascontiguousarray(forced_pool, np.int32)
+    rc = lib().orc_lisa_rows(inp.ref, topk, pool_m, _p(rows), n, _p(fp), _p(out["idx"]),
+                             _p(out["score"]), _p(out["score64"]), _p(out["pool"]),
+                             _p(out["dots"]))
+    assert rc == 0
+    return out
+
+
+def resmisa(inp: Inputs, topk: int, block: int, r: int, rows=None, forced_heads=None):
+    """ResMiSA rows: returns dict(idx, score, score64, heads [n, r], S [n, H], dots)."""
+    rows = _rows(inp.prob, rows)
+    n, H = len(rows), inp.prob.heads
+    out = dict(idx=np.empty((n, topk), np.int32), score=np.empty((n, topk), np.float32),
+               score64=np.empty((n, topk), np.float64), heads=np.empty((n, max(r, 1)), np.int32),
+               S=np.empty((n, H), np.float64), dots=np.empty(n, np.int64))
+    fh = None if forced_heads is None else np.ascontiguousarray(forced_heads, np.int32)
+    rc = lib().orc_resmisa_rows(inp.ref, topk, block, r, _p(rows), n, _p(fh), _p(out["idx"]),
+                                _p(out["score"]), _p(out["score64"]), _p(out["heads"]),
+                                _p(out["S"]), _p(out["dots"]))
+    assert rc == 0
+    out["heads"] = out["heads"][:, :r]
+    return out
+
+
+def residual_bounds(inp: Inputs, row: int, block: int):
+    """U^- [M_t, H] of one row (the ResMiSA router's per-block residual bounds)."""
+    p = inp.prob
+    m = (p.n_k + block - 1) // block + 1
+    out = np.empty((m, p.heads), np.float64)
+    got = lib().orc_residual_bounds(inp.ref, int(row), block, _p(out))
+    return out[:got]
 
 
 def score_pairs(inp: Inputs, rows, s, heads=None):

@@ -28,6 +28,19 @@
  *         tokens with the original formula"; "The new bottleneck of sparse
  *         attention", route one: HISA (mean-pooled block keys scored with the
  *         same indexer query, top blocks kept, DSA indexer run on their tokens).
+ *  [LISA] "PaperTrace 2.2.2", section 3.1 "the shared key merges the linear
+ *         term exactly": ReLU(x) = x + ReLU(-x), so
+ *         I_{t,s} = g_t . k_s + sum_j w_{t,j} ReLU(-q_{t,j} . k_s) with the fused
+ *         query g_t = sum_j w_{t,j} q_{t,j}; indexer LISA ranks tokens by the
+ *         linear term l_{t,s} = g_t . k_s alone; LISA-dagger screens a pool by
+ *         l and reranks it with every head.
+ *  [RES]  "PaperTrace 2.2.2", section 3.2 "MISA-2 keeps the shared linear term
+ *         and routes sparse residuals" (ResMiSA): per block b of the legal
+ *         prefix and dimension c the key range [kmin_{b,c}, kmax_{b,c}];
+ *         U^-_{t,b,j} = sum_c q+_c (-kmin_{b,c}) + q-_c kmax_{b,c} bounds
+ *         -q_{t,j} . k over the block (q+ = max(q, 0), q- = max(-q, 0));
+ *         S_{t,j} = |w_{t,j}| max_b ReLU(U^-_{t,b,j}); the top-r heads A_t;
+ *         I^_{t,s} = l_{t,s} + sum_{j in A_t} w_{t,j} ReLU(-q_{t,j} . k_s).
  *  [FP8]  "PaperTrace 2.2.2", section 2.3 "from formula to FP8 cache":
  *         k^ = round(k/a), FP8 data plus scale, higher-precision accumulation.
  *         The e4m3 code follows the OCP 8-bit floating point specification
@@ -48,6 +61,14 @@
  *  - HISA scores a block with the DSA formula on its representative
  *    (weights keep their sign, no absolute value).
  *  - Stacked MISA + HISA: the routed heads are used in both HISA stages.
+ *  - LISA-dagger's pool is the exact top-min(M, |legal|) by the linear score
+ *    (ties to the lower index): one fixed size inside the page's range
+ *    [min(k, N_t), min(C, N_t)] for the pool; the page's sampling and
+ *    histogram threshold estimate is not given, so the exact screen stands in.
+ *  - ResMiSA's blocks are those of the MISA router (B tokens over the legal
+ *    prefix, the boundary block holding only legal tokens); block extrema are
+ *    of the key operand values; the routed residual heads are used in
+ *    ascending head order; the reported score is I^.
  */
 #include <math.h>
 #include <stdint.h>
@@ -735,6 +756,204 @@ int64_t orc_block_scores(const orc_inputs* in, int64_t row, int32_t blk, const i
   }
   free(reps);
   return m;
+}
+
+/* ------------------------------------------------------ LISA / ResMiSA -- */
+
+/* [LISA] fused query g_t = sum_j w_{t,j} q_{t,j} (fp64, heads ascending). */
+static void fused_query(const orc_inputs* in, int64_t row, double* g) {
+  for (int32_t c = 0; c < in->dim; ++c) g[c] = 0.0;
+  for (int32_t j = 0; j < in->heads; ++j) {
+    double wj = (double)in->w[row * in->heads + j];
+    for (int32_t c = 0; c < in->dim; ++c) g[c] += wj * q_val(in, row, j, c);
+  }
+}
+
+/* [LISA] linear term l_{t,s} = g_t . k_s. */
+static double linear_score(const orc_inputs* in, int64_t row, int64_t s, const double* g) {
+  int32_t b = (int32_t)(row / in->n_q);
+  double acc = 0.0;
+  for (int32_t c = 0; c < in->dim; ++c) acc += g[c] * k_val(in, b, s, c);
+  return acc;
+}
+
+/* [LISA] indexer LISA (pool_m == 0): top-k of l over the legal prefix, scores l.
+ * LISA-dagger (pool_m > 0): pool = top-min(pool_m, |legal|) by l (or
+ * forced_pool [n_rows, pool_m], entries < 0 ignored), reranked by the full I
+ * over every head; top-k, scores I.
+ * out_pool [n_rows, pool_m] (rank order, -1 padded); out_dots = |legal| key dots
+ * (+ H * |pool| for the rerank). */
+int orc_lisa_rows(const orc_inputs* in, int32_t topk, int32_t pool_m, const int64_t* rows,
+                  int64_t n_rows, const int32_t* forced_pool, int32_t* out_idx, float* out_score,
+                  double* out_score64, int32_t* out_pool, int64_t* out_dots) {
+  if (pool_m < 0) return ORC_ERR;
+  int32_t* all = (int32_t*)malloc(sizeof(int32_t) * in->heads);
+  for (int32_t j = 0; j < in->heads; ++j) all[j] = j;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t row = rows[r];
+    int64_t n = row_legal(in, row);
+    double* g = (double*)malloc(sizeof(double) * in->dim);
+    fused_query(in, row, g);
+    ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    row_cache rc = row_cache_new(in, row);
+    for (int64_t s = 0; s < n; ++s) {
+      cand[s].v = MUT(34) ? score_cached(in, &rc, row, s, all, in->heads)
+                          : linear_score(in, row, s, g);
+      cand[s].i = s;
+    }
+    qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
+    int64_t dots = n;
+    if (pool_m == 0) {
+      emit_topk(cand, n, topk, out_idx + r * topk, out_score + r * topk,
+                out_score64 ? out_score64 + r * topk : NULL);
+    } else {
+      int64_t np = n < pool_m ? n : pool_m - (MUT(39) ? 1 : 0);
+      ranked* pool = (ranked*)malloc(sizeof(ranked) * (np > 0 ? np : 1));
+      int64_t cnt = 0;
+      if (forced_pool) {
+        for (int32_t a = 0; a < pool_m; ++a) {
+          int32_t s = forced_pool[r * pool_m + a];
+          if (s >= 0 && cnt < np) pool[cnt++].i = s;
+        }
+      } else {
+        for (int64_t a = 0; a < np; ++a) pool[cnt++].i = cand[a].i;
+      }
+      if (out_pool)
+        for (int32_t a = 0; a < pool_m; ++a)
+          out_pool[r * pool_m + a] = a < cnt ? (int32_t)pool[a].i : -1;
+      for (int64_t a = 0; a < cnt; ++a)
+        pool[a].v = score_cached(in, &rc, row, pool[a].i, all, in->heads);
+      qsort(pool, (size_t)cnt, sizeof(ranked), by_value_then_index);
+      emit_topk(pool, cnt, topk, out_idx + r * topk, out_score + r * topk,
+                out_score64 ? out_score64 + r * topk : NULL);
+      dots += (int64_t)in->heads * cnt;
+      free(pool);
+    }
+    if (out_dots) out_dots[r] = dots;
+    row_cache_free(&rc);
+    free(cand);
+    free(g);
+  }
+  free(all);
+  return ORC_OK;
+}
+
+/* [RES] residual bounds of one row: U^-_{t,a,j} for the M_t blocks a of the
+ * legal prefix (blocks of blk tokens; the last holds only legal tokens) and
+ * every head j, written to out [M_t, H]; returns M_t. */
+static int64_t residual_bounds(const orc_inputs* in, int64_t row, int32_t blk, double* out) {
+  int32_t b = (int32_t)(row / in->n_q);
+  int64_t n = row_legal(in, row);
+  if (MUT(38)) n = in->n_k;
+  int64_t m = (n + blk - 1) / blk;
+  double* kmin = (double*)malloc(sizeof(double) * in->dim);
+  double* kmax = (double*)malloc(sizeof(double) * in->dim);
+  for (int64_t a = 0; a < m; ++a) {
+    int64_t lo = a * blk, hi = lo + blk < n ? lo + blk : n;
+    for (int32_t c = 0; c < in->dim; ++c) {
+      kmin[c] = INFINITY;
+      kmax[c] = -INFINITY;
+    }
+    for (int64_t s = lo; s < hi; ++s)
+      for (int32_t c = 0; c < in->dim; ++c) {
+        double v = k_val(in, b, s, c);
+        if (v < kmin[c]) kmin[c] = v;
+        if (v > kmax[c]) kmax[c] = v;
+      }
+    for (int32_t j = 0; j < in->heads; ++j) {
+      double u = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) {
+        double qc = q_val(in, row, j, c);
+        double qp = qc > 0.0 ? qc : 0.0, qn = qc < 0.0 ? -qc : 0.0;
+        u += MUT(36) ? qp * (-kmax[c]) + qn * kmin[c] : qp * (-kmin[c]) + qn * kmax[c];
+      }
+      out[a * in->heads + j] = u;
+    }
+  }
+  free(kmin);
+  free(kmax);
+  return m;
+}
+
+/* Exported for tests: U^- [M_t, H] of one row; returns M_t. */
+int64_t orc_residual_bounds(const orc_inputs* in, int64_t row, int32_t blk, double* out) {
+  return residual_bounds(in, row, blk, out);
+}
+
+/* [RES] ResMiSA for the listed rows: residual routing S_{t,j} =
+ * |w_{t,j}| max_a ReLU(U^-_{t,a,j}), A_t = top-r by (S desc, j asc) (or
+ * forced_heads [n_rows, r]), then I^ = l + sum_{j in A_t} w_{t,j} ReLU(-q_{t,j}.k_s)
+ * over the legal prefix; top-k, scores I^.
+ * out_heads [n_rows, r] ascending; out_S [n_rows, H]; out_dots = (1 + r) |legal|
+ * key dots (the router's H M_t block bounds are extra). */
+int orc_resmisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_res,
+                     const int64_t* rows, int64_t n_rows, const int32_t* forced_heads,
+                     int32_t* out_idx, float* out_score, double* out_score64, int32_t* out_heads,
+                     double* out_S, int64_t* out_dots) {
+  if (r_res < 0 || r_res > in->heads || blk < 1) return ORC_ERR;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < n_rows; ++r) {
+    int64_t row = rows[r];
+    int64_t n = row_legal(in, row);
+    int64_t mmax = (in->n_k + blk - 1) / blk + 1;
+    double* U = (double*)malloc(sizeof(double) * (size_t)mmax * in->heads);
+    int64_t m = residual_bounds(in, row, blk, U);
+    double* S = (double*)malloc(sizeof(double) * in->heads);
+    ranked* order = (ranked*)malloc(sizeof(ranked) * in->heads);
+    for (int32_t j = 0; j < in->heads; ++j) {
+      double best = 0.0;
+      for (int64_t a = 0; a < m; ++a) {
+        double u = U[a * in->heads + j];
+        if (u > best) best = u;
+      }
+      double wj = (double)in->w[row * in->heads + j];
+      S[j] = (MUT(37) ? wj : fabs(wj)) * best;
+      order[j].v = S[j];
+      order[j].i = j;
+    }
+    qsort(order, (size_t)in->heads, sizeof(ranked), by_value_then_index);
+    int32_t* heads = (int32_t*)malloc(sizeof(int32_t) * (r_res > 0 ? r_res : 1));
+    if (forced_heads) {
+      memcpy(heads, forced_heads + r * r_res, sizeof(int32_t) * r_res);
+    } else {
+      for (int32_t a = 0; a < r_res; ++a) heads[a] = (int32_t)order[a].i;
+    }
+    qsort(heads, (size_t)r_res, sizeof(int32_t), cmp_i32);
+    if (out_heads) memcpy(out_heads + r * r_res, heads, sizeof(int32_t) * r_res);
+    if (out_S) memcpy(out_S + r * in->heads, S, sizeof(double) * in->heads);
+    double* g = (double*)malloc(sizeof(double) * in->dim);
+    fused_query(in, row, g);
+    ranked* cand = (ranked*)malloc(sizeof(ranked) * (n > 0 ? n : 1));
+    row_cache rc = row_cache_new(in, row);
+    int32_t b = (int32_t)(row / in->n_q);
+    for (int64_t s = 0; s < n; ++s) {
+      double v = linear_score(in, row, s, g);
+      for (int32_t c = 0; c < in->dim; ++c) rc.kd[c] = k_val(in, b, s, c);
+      for (int32_t a = 0; a < r_res; ++a) {
+        int32_t j = heads[a];
+        const double* qj = rc.q + (size_t)j * in->dim;
+        double z = 0.0;
+        for (int32_t c = 0; c < in->dim; ++c) z += qj[c] * rc.kd[c];
+        double neg = MUT(35) ? z : -z;
+        v += (double)in->w[row * in->heads + j] * (neg > 0.0 ? neg : 0.0);
+      }
+      cand[s].v = v;
+      cand[s].i = s;
+    }
+    qsort(cand, (size_t)n, sizeof(ranked), by_value_then_index);
+    emit_topk(cand, n, topk, out_idx + r * topk, out_score + r * topk,
+              out_score64 ? out_score64 + r * topk : NULL);
+    if (out_dots) out_dots[r] = (int64_t)(1 + r_res) * n;
+    row_cache_free(&rc);
+    free(cand);
+    free(g);
+    free(heads);
+    free(order);
+    free(S);
+    free(U);
+  }
+  return ORC_OK;
 }
 
 /* Full fp64 score row (all legal s) of one query row for the listed heads

@@ -48,6 +48,12 @@ MUTANTS = {
     31: "tolerance scale nu without the 1/sqrt(d) factor",
     32: "tolerance scale nu with the squared key norm",
     33: "split query drops its low e4m3 part",
+    34: "indexer LISA ranks by the full ReLU score instead of the linear term",
+    35: "ResMiSA residual takes ReLU(q . k) instead of ReLU(-q . k)",
+    36: "residual bound pairs q+ with the block maximum (wrong extreme)",
+    37: "residual router weighs the bound by signed w instead of |w|",
+    38: "residual bound blocks reach past the causal position",
+    39: "LISA-dagger pool one candidate short",
 }
 
 

@@ -548,3 +548,160 @@ def test_split_query_error_bound(oracle_mod):
     codes = rng.integers(-7, 8, size=(4, 128)).astype(np.float32) * 32.0
     codes[:, 0] = 448.0
     assert np.array_equal(oracle_mod.split_query(codes, F32), codes.astype(np.float64))
+
+
+# ------------------------------------------------ LISA / LISA-dagger / ResMiSA --
+
+def _golden(name):
+    return json.load(open(os.path.join(GOLD, name)))
+
+
+def test_lisa_decomposition_worked_example(oracle_mod):
+    """[PT] 3.1: the fused query 1.5 gives the linear term 4.5 (indexer LISA's score),
+    the correction 1.5 restores the score 6; ResMiSA with one residual head picks
+    the second head and recovers 6, with none it is LISA."""
+    g = _golden("lisa_decomposition.json")
+    p = make(np.array(g["q"])[None, None], np.array(g["k"])[None, None],
+             np.array(g["w"])[None, None], topk=1)
+    inp = oracle_mod.Inputs(p)
+    assert oracle_mod.dsa(inp, 1)[2][0, 0] == g["score"]
+    assert oracle_mod.lisa(inp, 1)["score64"][0, 0] == g["linear_term"]
+    assert g["linear_term"] == g["fused_query"] * g["k"][0]
+    assert g["linear_term"] + g["correction"] == g["score"]
+    r0 = oracle_mod.resmisa(inp, 1, 1, 0)
+    assert r0["score64"][0, 0] == g["linear_term"]
+    r1 = oracle_mod.resmisa(inp, 1, 1, 1)
+    assert list(r1["heads"][0]) == [g["residual_head"]]
+    assert r1["score64"][0, 0] == g["score"]
+
+
+def test_residual_bound_worked_example(oracle_mod):
+    """[PT] 3.2: q = (1, -2) over a block with key ranges [-1, 3] x [0, 4] has U- = 9,
+    above both actual negative dot products (1 and 5)."""
+    g = _golden("residual_bound_example.json")
+    q = np.array(g["q"], np.float32)[None, None, None]          # [1, 1, 1, 2]
+    keys = np.array(g["keys"], np.float32)[None]                  # [1, 2, 2]
+    p = make(q, keys, np.ones((1, 1, 1), np.float32), topk=1)    # query at position 1
+    inp = oracle_mod.Inputs(p)
+    U = oracle_mod.residual_bounds(inp, 0, 2)
+    assert U.shape == (1, 1) and U[0, 0] == g["bound"]
+    neg = -(keys[0] @ np.array(g["q"]))
+    assert list(neg) == g["negative_dots"] and np.all(neg <= U[0, 0])
+
+
+def test_residual_bound_covers_every_legal_key_and_no_future_key(oracle_mod):
+    """U-_{b,j} >= -q_j . k_s for every legal key of block b; a future key, however
+    extreme, does not move the bound (blocks cover the legal prefix only)."""
+    rng = np.random.default_rng(12)
+    nq, nk, H, d, blk = 6, 100, 4, 8, 16
+    q = rng.standard_normal((1, nq, H, d)).astype(np.float32)
+    k = rng.standard_normal((1, nk, d)).astype(np.float32)
+    w = rng.standard_normal((1, nq, H)).astype(np.float32)
+    p = make(q, k, w, topk=4, q_pos0=[50])
+    inp = oracle_mod.Inputs(p)
+    k2 = k.copy()
+    k2[0, 60:] = 1e3 * np.sign(k2[0, 60:])       # every row sits at position <= 55
+    inp2 = oracle_mod.Inputs(make(q, k2, w, topk=4, q_pos0=[50]))
+    for row in range(nq):
+        U = oracle_mod.residual_bounds(inp, row, blk)
+        n = 50 + row + 1
+        assert U.shape[0] == (n + blk - 1) // blk
+        for a in range(U.shape[0]):
+            ks = k[0, a * blk:min((a + 1) * blk, n)].astype(np.float64)
+            neg = -(ks @ q[0, row].astype(np.float64).T)           # [keys, H]
+            assert np.all(neg <= U[a][None] + 1e-9)
+        assert np.array_equal(U, oracle_mod.residual_bounds(inp2, row, blk))
+
+
+def test_resmisa_routes_by_weight_magnitude(oracle_mod):
+    """S_j = |w_j| max_b ReLU(U-_{b,j}): a head whose weight is negative but large in
+    magnitude outranks a positive head with the same bound."""
+    d = 4
+    q = np.zeros((1, 1, 3, d), np.float32)
+    q[0, 0, :, 0] = [-1.0, -1.0, 1.0]             # heads 0, 1 see -q.k = k_0 > 0
+    k = np.zeros((1, 8, d), np.float32)
+    k[0, :, 0] = np.arange(8)
+    w = np.array([[[-3.0, 1.0, 2.0]]], np.float32)
+    p = make(q, k, w, topk=3)
+    out = oracle_mod.resmisa(oracle_mod.Inputs(p), 3, 4, 1)
+    # bounds: heads 0, 1: max k_0 = 7; head 2: -min k_0 = 0
+    assert np.allclose(out["S"][0], [21.0, 7.0, 0.0])
+    assert list(out["heads"][0]) == [0]
+
+
+def test_resmisa_with_every_head_is_dsa(oracle_mod):
+    """r = H: l + sum_j w_j ReLU(-z_j) = sum_j w_j ReLU(z_j) (integer operands, exact)."""
+    p = gen.integer_problem(95, 2, 40, 90, 8, 16, 12, q_pos0=[50, 0], k_len=[90, 60])
+    inp = oracle_mod.Inputs(p)
+    ri, rs, rs64, _ = oracle_mod.dsa(inp, p.topk)
+    out = oracle_mod.resmisa(inp, p.topk, 16, p.heads)
+    assert np.array_equal(out["idx"], ri) and np.array_equal(out["score64"], rs64)
+    assert np.all(out["heads"] == np.arange(p.heads))
+
+
+def test_resmisa_without_residual_heads_is_lisa(oracle_mod):
+    p = gen.integer_problem(96, 1, 30, 70, 8, 16, 10)
+    inp = oracle_mod.Inputs(p)
+    a = oracle_mod.resmisa(inp, p.topk, 16, 0)
+    b = oracle_mod.lisa(inp, p.topk)
+    assert np.array_equal(a["idx"], b["idx"]) and np.array_equal(a["score64"], b["score64"])
+
+
+def test_lisa_closed_form_line(oracle_mod):
+    """q_{t,j} = c_j e_0, k_s = s e_0: l_{t,s} = s sum_j w_j c_j (the ReLU plays no
+    part); positive sums rank the latest keys first, negative sums the earliest."""
+    rng = np.random.default_rng(14)
+    nq, nk, H, topk = 10, 30, 5, 6
+    c = rng.integers(-3, 4, size=(nq, H)).astype(np.float32)
+    w = rng.integers(-2, 3, size=(nq, H)).astype(np.float32)
+    p = _line_problem(nq, nk, c, w, +1.0, topk)
+    out = oracle_mod.lisa(oracle_mod.Inputs(p), topk)
+    for i in range(nq):
+        pos = nk - nq + i
+        gsum = float(np.sum(w[i] * c[i]))
+        legal = np.arange(pos + 1)
+        want = legal[::-1][:topk] if gsum > 0 else legal[:topk]
+        assert list(out["idx"][i]) == list(want), (i, gsum)
+        assert np.array_equal(out["score64"][i], want * gsum + 0.0)
+
+
+def test_lisa_dagger_full_pool_is_dsa(oracle_mod):
+    p = gen.integer_problem(97, 1, 40, 80, 8, 16, 10)
+    inp = oracle_mod.Inputs(p)
+    ri, rs, rs64, _ = oracle_mod.dsa(inp, p.topk)
+    out = oracle_mod.lisa(inp, p.topk, pool_m=80)
+    assert np.array_equal(out["idx"], ri) and np.array_equal(out["score64"], rs64)
+
+
+def test_lisa_dagger_pool_of_k_keeps_the_lisa_set(oracle_mod):
+    """A pool of exactly k keeps LISA's set; only the scores (now the full I) and
+    their order change."""
+    p = gen.normal_problem(98, 1, 30, 120, 8, 32, 16)
+    inp = oracle_mod.Inputs(p)
+    a = oracle_mod.lisa(inp, p.topk)
+    b = oracle_mod.lisa(inp, p.topk, pool_m=p.topk)
+    assert np.array_equal(np.sort(a["idx"], 1), np.sort(b["idx"], 1))
+    rows = np.repeat(np.arange(p.n_q), p.topk)
+    full = oracle_mod.score_pairs(inp, rows, b["idx"].ravel()).reshape(b["idx"].shape)
+    assert np.array_equal(full, b["score64"])
+
+
+def test_lisa_and_resmisa_cost_counts_match_page_arithmetic(oracle_mod):
+    """[PT] 3.2 'one set of numbers': per query at N = 131072, H_I = 64, k = 2048,
+    pool M = 8192, r = 7: DSA 8,388,608 key dots, LISA 131,072, ResMiSA 1,048,576
+    (1/8), LISA-dagger 655,360 (7.81 %).  Counted on the last row of an
+    N-key prefix (d = 4: the counts do not depend on d)."""
+    g = _golden("cost_arithmetic.json")["lisa_resmisa_example"]
+    N, H = g["N"], g["heads"]
+    rng = np.random.default_rng(15)
+    q = rng.integers(-2, 3, size=(1, 1, H, 4)).astype(np.float32)
+    k = rng.integers(-2, 3, size=(1, N, 4)).astype(np.float32)
+    w = rng.integers(-2, 3, size=(1, 1, H)).astype(np.float32)
+    inp = oracle_mod.Inputs(make(q, k, w, topk=2048))
+    assert oracle_mod.dsa(inp, 2048)[3][0] == g["dsa_dots_per_query"]
+    assert oracle_mod.lisa(inp, 2048)["dots"][0] == g["lisa_dots_per_query"]
+    assert oracle_mod.resmisa(inp, 2048, 1024, g["residual_heads"])["dots"][0] == \
+        g["resmisa_dots_per_query"] == g["dsa_dots_per_query"] * g["resmisa_fraction"]
+    ld = oracle_mod.lisa(inp, 2048, pool_m=g["pool"])["dots"][0]
+    assert ld == g["lisa_dagger_dots_per_query"]
+    assert round(100.0 * ld / g["dsa_dots_per_query"], 2) == g["lisa_dagger_percent"]
