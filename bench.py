@@ -106,13 +106,25 @@ WORKLOADS = {
              "Gaussian centres in contiguous runs",
         kind="hisa", batch=1, L=_L128, H=64, topk=2048, seed=5, hb=64, r=128, h=0,
         block=1024, keys="clusters"),
+    "lisa_prefill_128k": dict(
+        desc="Indexer LISA prefill, batch 1, L=131072 causal, H_I=64, d=128, top-k=2048 by "
+             "the linear term of the fused query, bf16 q,k ~N(0,1), w ~N(0,1/64)",
+        kind="lisa", batch=1, L=_L128, H=64, topk=2048, seed=4, pool=0),
+    "lisa_dagger_prefill_128k": dict(
+        desc="LISA-dagger prefill, batch 1, L=131072 causal, H_I=64, d=128, pool M=8192 by "
+             "the linear term reranked by all heads, top-k=2048, bf16 q,k ~N(0,1)",
+        kind="lisa", batch=1, L=_L128, H=64, topk=2048, seed=4, pool=8192),
+    "resmisa_prefill_128k": dict(
+        desc="ResMiSA prefill, batch 1, L=131072 causal, H_I=64, d=128, shared linear term + "
+             "r=7 residual heads routed by block bounds (B=1024), top-k=2048, bf16 q,k ~N(0,1)",
+        kind="resmisa", batch=1, L=_L128, H=64, topk=2048, seed=4, block=1024, r=7),
     "hisa_misa_prefill_128k": dict(
         desc="Stacked MISA (B=1024, h=8) + HISA (b=64, r=128) prefill, batch 1, L=131072 "
              "causal, H_I=64, d=128, top-k=2048, bf16, clustered keys",
         kind="hisa", batch=1, L=_L128, H=64, topk=2048, seed=5, hb=64, r=128, h=8,
         block=1024, keys="clusters"),
 }
-ROUTED = ("misa", "dagger", "hisa")
+ROUTED = ("misa", "dagger", "hisa", "lisa", "resmisa")
 
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
 TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic_scan_kernel.md")
@@ -179,7 +191,8 @@ def algorithmic_work(p, w=None):
     """Scored (query, key, head) dot products of the method and their FLOPs (2 d each).
 
     DSA: H |legal|.  MISA: H M_t + h |legal| (router + routed scan).  MISA-dagger:
-    + H min(k', |legal|).  HISA: hh M^b_t + hh min(r b, |legal|) (coarse + rerank;
+    + H min(k', |legal|).  LISA: |legal| (one fused-query dot per key; LISA-dagger
+    + H min(M, |legal|)).  ResMiSA: H M_t block bounds + (1 + r) |legal|.  HISA: hh M^b_t + hh min(r b, |legal|) (coarse + rerank;
     the rerank count is an upper bound, exact unless the kept set holds the
     partial boundary block), hh = h when stacked (+ H M_t for its router)."""
     n = legal_counts(p)
@@ -192,6 +205,10 @@ def algorithmic_work(p, w=None):
         dots = H * m + w["h"] * n
         if kind == "dagger":
             dots = dots + H * np.minimum(w["k_prime"], n)
+    elif kind == "lisa":
+        dots = n + (H * np.minimum(w["pool"], n) if w["pool"] else 0)
+    elif kind == "resmisa":
+        dots = H * ((n + w["block"] - 1) // w["block"]) + (1 + w["r"]) * n
     else:
         hh = w["h"] if w["h"] else H
         mb = (n + w["hb"] - 1) // w["hb"]
@@ -290,6 +307,10 @@ def _oracle_rows(inp, p, w, rows):
         oracle.misa(inp, p.topk, w["block"], w["h"], rows=rows)
     elif kind == "dagger":
         oracle.misa(inp, p.topk, w["block"], w["h"], k_prime=w["k_prime"], rows=rows)
+    elif kind == "lisa":
+        oracle.lisa(inp, p.topk, pool_m=w["pool"], rows=rows)
+    elif kind == "resmisa":
+        oracle.resmisa(inp, p.topk, w["block"], w["r"], rows=rows)
     else:
         oracle.hisa(inp, p.topk, w["hb"], w["r"], route_h=w["h"], route_block=w["block"],
                     rows=rows)
@@ -370,7 +391,8 @@ def run_reference(args, w, p):
 
 # in an order that reuses generated problems: MISA and MISA-dagger share the
 # headline problem, stacked HISA shares HISA's clustered keys
-SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "hisa_prefill_128k",
+SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "lisa_prefill_128k",
+             "lisa_dagger_prefill_128k", "resmisa_prefill_128k", "hisa_prefill_128k",
              "hisa_misa_prefill_128k", "dsa_decode_128k"]
 
 
@@ -455,10 +477,15 @@ class Case:
         c["prob"] = B.problem(c["q"], c["k"], p.topk, pos0, klen)
         if self.kind in ROUTED:
             algo = {"misa": B.DSA_ALGO_MISA, "dagger": B.DSA_ALGO_MISA_DAGGER,
-                    "hisa": B.DSA_ALGO_HISA}[self.kind]
+                    "hisa": B.DSA_ALGO_HISA, "lisa": B.DSA_ALGO_LISA,
+                    "resmisa": B.DSA_ALGO_RESMISA}[self.kind]
             if self.kind == "hisa":
                 rp = B.route_params(misa_block=w["block"] if w["h"] else 0, misa_h=w["h"],
                                     hisa_block=w["hb"], hisa_r=w["r"])
+            elif self.kind == "lisa":
+                rp = B.route_params(lisa_pool=w["pool"])
+            elif self.kind == "resmisa":
+                rp = B.route_params(res_block=w["block"], res_r=w["r"])
             else:
                 rp = B.route_params(misa_block=w["block"], misa_h=w["h"],
                                     k_prime=w.get("k_prime", 0))
@@ -469,6 +496,10 @@ class Case:
                 c["launches"] = 2 + 2 * chunks
             elif self.kind == "dagger":
                 c["launches"] = 2 + 4 * chunks
+            elif self.kind == "lisa":
+                c["launches"] = 1 + (4 if w["pool"] else 2) * chunks
+            elif self.kind == "resmisa":
+                c["launches"] = (3 if w["r"] else 1) + 2 * chunks
             else:
                 c["launches"] = (2 if w["h"] else 0) + 1 + 5 * chunks
         else:
@@ -484,6 +515,12 @@ class Case:
         elif self.kind == "dagger":
             B.misa_dagger_index(q, k, w_, p.topk, w["block"], w["h"], w["k_prime"],
                                 q_pos0=c["pos0"], k_len=c["klen"], out=out, workspace=self.ws)
+        elif self.kind == "lisa":
+            B.lisa_index(q, k, w_, p.topk, pool=w["pool"], q_pos0=c["pos0"], k_len=c["klen"],
+                         out=out, workspace=self.ws)
+        elif self.kind == "resmisa":
+            B.resmisa_index(q, k, w_, p.topk, w["block"], w["r"], q_pos0=c["pos0"],
+                            k_len=c["klen"], out=out, workspace=self.ws)
         else:
             B.hisa_index(q, k, w_, p.topk, w["hb"], w["r"], route_h=w["h"],
                          route_block=w["block"], q_pos0=c["pos0"], k_len=c["klen"], out=out,

@@ -95,7 +95,14 @@ enum {
 typedef enum { DSA_F32 = 0, DSA_BF16 = 1, DSA_E4M3 = 2 } dsa_dtype;
 
 /* Algorithm ids for dsa_workspace_size(). */
-enum { DSA_ALGO_DSA = 0, DSA_ALGO_MISA = 1, DSA_ALGO_MISA_DAGGER = 2, DSA_ALGO_HISA = 3 };
+enum {
+  DSA_ALGO_DSA = 0,
+  DSA_ALGO_MISA = 1,
+  DSA_ALGO_MISA_DAGGER = 2,
+  DSA_ALGO_HISA = 3,
+  DSA_ALGO_LISA = 4,     /* indexer LISA and LISA-dagger (lisa_index) */
+  DSA_ALGO_RESMISA = 5   /* ResMiSA (resmisa_index) */
+};
 
 /* problem.flags */
 #define DSA_FLAG_CHECK 1u  /* validate scales/lengths on device, synchronise, return device status */
@@ -142,6 +149,9 @@ typedef struct {
   int32_t k_prime;
   int32_t hisa_block;
   int32_t hisa_r;
+  int32_t lisa_pool;   /* M: LISA-dagger pool, topk <= M <= 8192 (0: plain indexer LISA) */
+  int32_t res_block;   /* ResMiSA router block B: a power of two in [16, 4096] */
+  int32_t res_r;       /* ResMiSA residual heads r, 0 <= r <= min(heads, 124) */
 } dsa_route_params;
 
 /* Bytes of device workspace that `algo` needs for problem `p` (route params
@@ -228,6 +238,36 @@ int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q,
                const void* k, const float* w, int32_t* out_idx, float* out_score,
                int32_t* out_blocks, int32_t* out_heads, void* workspace,
                size_t workspace_bytes, void* stream);
+
+/* Indexer LISA ("PaperTrace 2.2.2", section 3.1: the shared key lets the linear
+ * part of every head merge exactly, since ReLU(x) = x + ReLU(-x)): the fused
+ * query g_t = sum_j w_{t,j} q_{t,j} scores every legal token by the linear term
+ * l_{t,s} = g_t . k_s alone, and the top-k by l is returned with l as its score.
+ * With rp->lisa_pool = M > 0 (LISA-dagger) the top-M by l form a pool that is
+ * reranked by the full score I over every head: top-k of I, scores I;
+ * out_pool [batch, n_q, M] int32 (optional) receives the pool (unordered,
+ * -1 padded).  The pool is the exact top-min(M, |legal|) by l (ties to the lower
+ * index), one fixed size within the page's range for it.  g is accumulated in
+ * fp32 over the heads in ascending order and enters the tensor core as two bf16
+ * parts (hi + lo, about 16 significant bits).  bf16 q and k only. */
+int lisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+               const float* w, int32_t* out_idx, float* out_score, int32_t* out_pool,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/* ResMiSA ("PaperTrace 2.2.2", section 3.2, MISA-2): the linear term l of every
+ * head plus r routed residual heads,
+ *   I^_{t,s} = l_{t,s} + sum_{j in A_t} w_{t,j} ReLU(-q_{t,j} . k_s).
+ * Router: the legal prefix is cut into blocks of rp->res_block tokens (the last
+ * holds only legal tokens); with the per-dimension key range [kmin, kmax] of
+ * block b, U-_{t,b,j} = sum_c max(q_c,0)(-kmin_c) + max(-q_c,0) kmax_c bounds
+ * -q_{t,j} . k over the block; S_{t,j} = |w_{t,j}| max_b ReLU(U-); A_t = the r
+ * heads of largest S (ties to the lower head), ascending in out_heads
+ * [batch, n_q, r] (optional); out_S [batch, n_q, heads] fp32 (optional).  The
+ * reported score is I^ (r = heads gives the DSA score, r = 0 the LISA score).
+ * bf16 q and k only. */
+int resmisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+                  const float* w, int32_t* out_idx, float* out_score, int32_t* out_heads,
+                  float* out_S, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Operand preparation for the FP8 path: per-row scale a = amax/448 (amax == 0
  * gives a = 1), code = round-to-nearest-even, saturating e4m3 of x/a, both

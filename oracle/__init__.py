@@ -69,6 +69,8 @@ def lib():
         _lib.orc_block_scores.argtypes = [vp, i64, i32, vp, i32, vp]
         _lib.orc_lisa_rows.argtypes = [vp, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp]
         _lib.orc_resmisa_rows.argtypes = [vp, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp, vp]
+        _lib.orc_linear_pairs.argtypes = [vp, vp, vp, i64, vp]
+        _lib.orc_resmisa_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
         _lib.orc_residual_bounds.restype = C.c_int64
         _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_score_row.restype = C.c_int64
@@ -196,6 +198,26 @@ def resmisa(inp: Inputs, topk: int, block: int, r: int, rows=None, forced_heads=
                                 _p(out["S"]), _p(out["dots"]))
     assert rc == 0
     out["heads"] = out["heads"][:, :r]
+    return out
+
+
+def linear_pairs(inp: Inputs, rows, s):
+    """fp64 LISA linear terms l = g . k at (rows[a], s[a])."""
+    rows = np.ascontiguousarray(rows, np.int64)
+    s = np.ascontiguousarray(s, np.int64)
+    out = np.empty(len(rows), np.float64)
+    lib().orc_linear_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(out))
+    return out
+
+
+def resmisa_pairs(inp: Inputs, rows, s, heads):
+    """fp64 ResMiSA scores at (rows[a], s[a]) with residual heads heads[a] ([n, r])."""
+    rows = np.ascontiguousarray(rows, np.int64)
+    s = np.ascontiguousarray(s, np.int64)
+    heads = np.ascontiguousarray(heads, np.int32).reshape(len(rows), -1)
+    out = np.empty(len(rows), np.float64)
+    lib().orc_resmisa_pairs(inp.ref, _p(rows), _p(s), len(rows), _p(heads), heads.shape[1],
+                            _p(out))
     return out
 
 

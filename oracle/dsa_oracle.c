@@ -956,6 +956,42 @@ int orc_resmisa_rows(const orc_inputs* in, int32_t topk, int32_t blk, int32_t r_
   return ORC_OK;
 }
 
+/* fp64 linear terms l_{t,s} = g_t . k_s at explicit (row, s) pairs. [LISA] */
+int orc_linear_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                     double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t a = 0; a < n; ++a) {
+    double* g = (double*)malloc(sizeof(double) * in->dim);
+    fused_query(in, rows[a], g);
+    out[a] = linear_score(in, rows[a], s[a], g);
+    free(g);
+  }
+  return ORC_OK;
+}
+
+/* fp64 ResMiSA scores I^ = l + sum_{j in heads} w_j ReLU(-q_j . k_s) at explicit
+ * (row, s) pairs; heads [n, r] (one residual head list per pair). [RES] */
+int orc_resmisa_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* s, int64_t n,
+                      const int32_t* heads, int32_t r, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t a = 0; a < n; ++a) {
+    int64_t row = rows[a];
+    int32_t b = (int32_t)(row / in->n_q);
+    double* g = (double*)malloc(sizeof(double) * in->dim);
+    fused_query(in, row, g);
+    double v = linear_score(in, row, s[a], g);
+    for (int32_t x = 0; x < r; ++x) {
+      int32_t j = heads[a * r + x];
+      double z = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * k_val(in, b, s[a], c);
+      v += (double)in->w[row * in->heads + j] * (-z > 0.0 ? -z : 0.0);
+    }
+    out[a] = v;
+    free(g);
+  }
+  return ORC_OK;
+}
+
 /* Full fp64 score row (all legal s) of one query row for the listed heads
  * (NULL = all); returns |legal|.  Used by tests for margins and tie checks. */
 int64_t orc_score_row(const orc_inputs* in, int64_t row, const int32_t* heads, int32_t nh,

@@ -19,6 +19,7 @@ DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE = 0, -1, -2, -3
 DSA_ERR_CUDA, DSA_ERR_NONFINITE, DSA_ERR_TIMEOUT, DSA_ERR_INTERNAL = -4, -5, -6, -7
 DSA_F32, DSA_BF16, DSA_E4M3 = 0, 1, 2
 DSA_ALGO_DSA, DSA_ALGO_MISA, DSA_ALGO_MISA_DAGGER, DSA_ALGO_HISA = 0, 1, 2, 3
+DSA_ALGO_LISA, DSA_ALGO_RESMISA = 4, 5
 DSA_FLAG_CHECK = 1
 DSA_FLAG_SORTED = 2
 DSA_FLAG_TEST_STALL = 0x80000000   # tests of the timeout path only (see include/dsaidx.h)
@@ -33,7 +34,8 @@ class DsaProblem(C.Structure):
 
 class DsaRouteParams(C.Structure):
     _fields_ = [("misa_block", C.c_int32), ("misa_h", C.c_int32), ("k_prime", C.c_int32),
-                ("hisa_block", C.c_int32), ("hisa_r", C.c_int32)]
+                ("hisa_block", C.c_int32), ("hisa_r", C.c_int32), ("lisa_pool", C.c_int32),
+                ("res_block", C.c_int32), ("res_r", C.c_int32)]
 
 
 class DsaError(RuntimeError):
@@ -62,12 +64,15 @@ def _load():
     lib.misa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.misa_dagger_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.hisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.lisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.resmisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
     for f in ("dsa_read_status", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
               "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
-              "misa_dagger_index", "hisa_index", "dsa_quantize_e4m3"):
+              "misa_dagger_index", "hisa_index", "lisa_index", "resmisa_index",
+              "dsa_quantize_e4m3"):
         getattr(lib, f).restype = C.c_int
     return lib
 
@@ -144,8 +149,10 @@ def problem(q: torch.Tensor, k: torch.Tensor, topk: int, q_pos0=None, k_len=None
                       _ptr(k_len), flags)
 
 
-def route_params(misa_block=0, misa_h=0, k_prime=0, hisa_block=0, hisa_r=0) -> DsaRouteParams:
-    return DsaRouteParams(misa_block, misa_h, k_prime, hisa_block, hisa_r)
+def route_params(misa_block=0, misa_h=0, k_prime=0, hisa_block=0, hisa_r=0, lisa_pool=0,
+                 res_block=0, res_r=0) -> DsaRouteParams:
+    return DsaRouteParams(misa_block, misa_h, k_prime, hisa_block, hisa_r, lisa_pool, res_block,
+                          res_r)
 
 
 def dsa_workspace_size(p: DsaProblem, algo: int = DSA_ALGO_DSA, rp: DsaRouteParams | None = None) -> int:
@@ -258,6 +265,35 @@ def hisa_index(q, k, w, topk, block, r, route_h=0, route_block=1024, q_pos0=None
     _check(lib.hisa_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(sc),
                           _ptr(out_blocks), _ptr(out_heads), _ptr(ws), ws.numel(), _stream(stream)),
            "hisa_index")
+    return idx, sc
+
+
+def lisa_index(q, k, w, topk, pool=0, q_pos0=None, k_len=None, flags=0, out=None,
+               out_pool=None, workspace=None, stream=None):
+    """Indexer LISA (pool == 0: top-k by the linear term g . k) or LISA-dagger
+    (pool = M: the top-M by g . k reranked by the full score over every head)."""
+    _common_args(q, k, w, None, None, q_pos0, k_len, out, workspace, out_pool=(out_pool, _I32))
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    rp = route_params(lisa_pool=pool)
+    ws = _workspace(dsa_workspace_size(p, DSA_ALGO_LISA, rp), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.lisa_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx), _ptr(sc),
+                          _ptr(out_pool), _ptr(ws), ws.numel(), _stream(stream)), "lisa_index")
+    return idx, sc
+
+
+def resmisa_index(q, k, w, topk, block, r, q_pos0=None, k_len=None, flags=0, out=None,
+                  out_heads=None, out_S=None, workspace=None, stream=None):
+    """ResMiSA: the linear term of every head plus r routed residual heads."""
+    _common_args(q, k, w, None, None, q_pos0, k_len, out, workspace,
+                 out_heads=(out_heads, _I32), out_S=(out_S, _F32))
+    p = problem(q, k, topk, q_pos0, k_len, flags)
+    rp = route_params(res_block=block, res_r=r)
+    ws = _workspace(dsa_workspace_size(p, DSA_ALGO_RESMISA, rp), q.device, workspace)
+    idx, sc = _outputs(q.shape[0], q.shape[1], topk, q.device, out)
+    _check(lib.resmisa_index(C.byref(p), C.byref(rp), _ptr(q), _ptr(k), _ptr(w), _ptr(idx),
+                             _ptr(sc), _ptr(out_heads), _ptr(out_S), _ptr(ws), ws.numel(),
+                             _stream(stream)), "resmisa_index")
     return idx, sc
 
 

@@ -204,40 +204,6 @@ __device__ __forceinline__ uint64_t make_sdesc(uint32_t smem_addr) {
   return d;
 }
 
-// The same descriptor split into its two 32-bit words: the low word holds the
-// start address (addr >> 4, 14 bits) and the leading offset; the high word is
-// the same constant for every operand of this layout.  Advancing an operand
-// then costs one 32-bit add on the low word (shared addresses stay below
-// 2^18, so the address field never carries into the leading offset).
-constexpr uint32_t kSdescHi = (1024u >> 4) | (1u << 14) | (2u << 29);
-__device__ __forceinline__ uint32_t sdesc_lo(uint32_t smem_addr) {
-  return ((smem_addr >> 4) & 0x3FFFu) | (1u << 16);
-}
-// tcgen05.mma from split descriptors; ACC (compile-time) selects accumulate.
-template <MmaKind K, int ACC>
-__device__ __forceinline__ void tc_mma_lo(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo,
-                                          uint32_t idesc) {
-  if constexpr (K == MmaKind::BF16) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
-  } else if constexpr (K == MmaKind::TF32) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "mov.b64 ad, {%1, %5};\n\tmov.b64 bd, {%2, %5};\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], ad, bd, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_lo), "r"(b_lo), "r"(idesc), "n"(ACC), "n"(kSdescHi));
-  }
-}
-
 // 32 lanes x 32 consecutive fp32 columns per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(

@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "finalize.cuh"
 #include "prep.cuh"
+#include "resid.cuh"
 #include "route.cuh"
 #include "scan.cuh"
 
@@ -478,19 +479,48 @@ struct RouteCfg {
   int h, bsR, nblkR, ncolsR;
   bool hisa;
   int bsH, nblkH, r;
-  int kp;            // MISA-dagger pool size
+  int kp;            // MISA-dagger / LISA-dagger pool size
   int hh;            // heads of the token stages
   int list_len;      // per-row list of the second stage (pool or blocks), 0 for MISA
+  bool pseudo;       // LISA / ResMiSA: the token stage runs on pseudo-head rows
+  int hp;            // pseudo-heads per row (power of two >= 4 + res_r)
+  bool res;          // ResMiSA: the residual router runs
+  int bsX, nblkX, res_r;  // ResMiSA router block shift, full blocks, residual heads
 };
 
 int route_cfg(const dsa_problem* p, int algo, const dsa_route_params* rp, RouteCfg* c) {
   if (!rp) return DSA_ERR_INVALID;
-  if (algo != DSA_ALGO_MISA && algo != DSA_ALGO_MISA_DAGGER && algo != DSA_ALGO_HISA)
+  if (algo != DSA_ALGO_MISA && algo != DSA_ALGO_MISA_DAGGER && algo != DSA_ALGO_HISA &&
+      algo != DSA_ALGO_LISA && algo != DSA_ALGO_RESMISA)
     return DSA_ERR_INVALID;
   if (p->q_dtype != DSA_BF16 || p->k_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
   if (p->batch > 65535) return DSA_ERR_UNSUPPORTED;
   *c = RouteCfg{};
   c->algo = algo;
+  if (algo == DSA_ALGO_LISA || algo == DSA_ALGO_RESMISA) {
+    c->pseudo = true;
+    if (algo == DSA_ALGO_LISA) {
+      c->hp = 8;
+      if (rp->lisa_pool != 0) {
+        if (rp->lisa_pool < p->topk) return DSA_ERR_INVALID;
+        if (rp->lisa_pool > 8192) return DSA_ERR_UNSUPPORTED;
+        c->kp = rp->lisa_pool;
+        c->list_len = c->kp;
+      }
+    } else {
+      if (rp->res_r < 0 || rp->res_r > p->heads) return DSA_ERR_INVALID;
+      if (rp->res_r > 124) return DSA_ERR_UNSUPPORTED;
+      if (!pow2_in(rp->res_block, 16, 4096)) return DSA_ERR_UNSUPPORTED;
+      c->res = true;
+      c->res_r = rp->res_r;
+      c->bsX = log2_exact(rp->res_block);
+      c->nblkX = p->n_k >> c->bsX;
+      c->hp = 8;
+      while (c->hp < 4 + c->res_r) c->hp *= 2;
+    }
+    c->hh = c->hp;
+    return DSA_OK;
+  }
   c->route = algo != DSA_ALGO_HISA || rp->misa_h > 0;
   if (c->route) {
     if (rp->misa_h < 1 || rp->misa_h > p->heads) return DSA_ERR_INVALID;
@@ -532,7 +562,14 @@ struct RouteStages {
 
 RouteStages plan_route(const dsa_problem* p, const RouteCfg& c, int nq) {
   RouteStages rs{};
-  if (c.algo == DSA_ALGO_MISA) {
+  if (c.pseudo) {
+    // the pseudo-head scan keeps the LISA-dagger pool or the final top-k
+    rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, p->n_k, c.hp, c.kp > 0 ? c.kp : p->topk);
+    if (c.kp > 0) {
+      rs.s2 = plan_gather(MmaKind::BF16, p->batch, nq, p->heads, p->topk);
+      rs.two = true;
+    }
+  } else if (c.algo == DSA_ALGO_MISA) {
     rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, p->n_k, c.h, p->topk);
   } else if (c.algo == DSA_ALGO_MISA_DAGGER) {
     rs.s1 = plan_scan(MmaKind::BF16, false, p->batch, nq, p->n_k, c.h, c.kp);
@@ -560,6 +597,7 @@ struct RouteLayout {
   int nq_c, n_chunks;
   size_t fullR_rows, fullH_rows;
   size_t off_runR, off_fullR, off_heads, off_qg, off_wg, off_runH, off_fullH, off_list, off_logs;
+  size_t off_extrun, off_extfull;
   size_t total;
 };
 
@@ -577,6 +615,20 @@ RouteLayout route_layout(const dsa_problem* p, const RouteCfg& c) {
   const size_t logs_last = stages_log_bytes(plan_route(p, c, last));
   if (logs_last > logs) logs = logs_last;
   size_t off = kWsHeaderBytes;
+  if (c.pseudo) {
+    L.off_qg = off;
+    off += align_up(rows * c.hp * 128 * 2);
+    L.off_wg = off;
+    off += align_up(rows * c.hp * sizeof(float));
+  }
+  if (c.res) {
+    L.off_extrun = off;
+    off += align_up((size_t)p->batch * p->n_k * 256 * 2);
+    L.off_extfull = off;
+    off += align_up((size_t)p->batch * (c.nblkX > 0 ? c.nblkX : 1) * 256 * 2);
+    L.off_heads = off;
+    off += align_up(rows * (c.res_r > 0 ? c.res_r : 1) * sizeof(int32_t));
+  }
   if (c.route) {
     L.fullR_rows = (size_t)p->batch * (c.nblkR > 0 ? c.nblkR : 1) + 256;
     L.off_runR = off;
@@ -779,6 +831,83 @@ int route_begin(const dsa_problem* p, int algo, const dsa_route_params* rp, cons
   if (p->flags & DSA_FLAG_CHECK)
     check_inputs_kernel<<<64, 256, 0, st>>>(nullptr, 0, nullptr, 0, p->q_pos0, p->k_len, p->batch,
                                             p->n_k, reinterpret_cast<int32_t*>(w8));
+  return DSA_OK;
+}
+
+// Pseudo-head rows of every query (LISA: the linear term; ResMiSA: plus the
+// residual heads), written into the workspace for the token scan.
+int run_pseudo(const dsa_problem* p, const RouteLayout& L, const void* q, const float* w,
+               const int32_t* heads, uint8_t* ws, cudaStream_t st) {
+  PseudoArgs a{};
+  a.rows = (int64_t)p->batch * p->n_q;
+  a.H = p->heads;
+  a.HP = L.c.hp;
+  a.r = L.c.res_r;
+  a.q = reinterpret_cast<const uint16_t*>(q);
+  a.w = w;
+  a.heads = heads;
+  a.qp = reinterpret_cast<uint16_t*>(ws + L.off_qg);
+  a.wp = reinterpret_cast<float*>(ws + L.off_wg);
+  pseudo_heads_kernel<<<(unsigned)((a.rows + 7) / 8), 256, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// The pseudo-head token scan over every legal key, then (LISA-dagger) the
+// all-head rerank of each row's pool; per row chunk.
+int run_pseudo_stages(const dsa_problem* p, const RouteLayout& L, const void* q, const void* k,
+                      const float* w, int32_t* out_idx, float* out_score, int32_t* out_pool,
+                      uint8_t* ws, cudaStream_t st) {
+  int32_t* status = reinterpret_cast<int32_t*>(ws);
+  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  int32_t* pool = reinterpret_cast<int32_t*>(ws + L.off_list);
+  for (int ci = 0; ci < L.n_chunks; ++ci) {
+    const int q_off = ci * L.nq_c;
+    const int nq = p->n_q - q_off < L.nq_c ? p->n_q - q_off : L.nq_c;
+    const RouteStages rs = plan_route(p, L.c, nq);
+    LogPtrs lp = log_ptrs(rs.s1, ws + L.off_logs);
+    StageIO io{};
+    io.q = ws + L.off_qg;
+    io.w = reinterpret_cast<const float*>(ws + L.off_wg);
+    io.q_stride = p->n_q;
+    io.H = L.c.hp;
+    io.k = k;
+    io.k_rows = (uint64_t)p->batch * p->n_k;
+    io.k_box = 128;
+    io.n_kmap = p->n_k;
+    int rc = run_stage(p, rs.s1, io, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (L.c.kp == 0) {
+      if (launch_finalize(rs.s1, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
+                          OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+      continue;
+    }
+    if (launch_finalize(rs.s1, L.c.kp, 0, lp.logs, lp.cnt, lp.thr, pool, nullptr,
+                        OutMap{nq, nq, 0}, status, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    if (out_pool) {
+      rc = copy_lists(out_pool, pool, p, q_off, nq, L.c.kp, st);
+      if (rc != DSA_OK) return rc;
+    }
+    lp = log_ptrs(rs.s2, ws + L.off_logs);
+    StageIO io2{};
+    io2.q = q;
+    io2.w = w;
+    io2.q_stride = p->n_q;
+    io2.H = p->heads;
+    io2.k = k;
+    io2.k_rows = (uint64_t)p->batch * p->n_k;
+    io2.k_box = 1;
+    io2.n_kmap = p->n_k;
+    io2.klist = pool;
+    io2.klist_len = L.c.kp;
+    io2.gather = 1;
+    rc = run_stage(p, rs.s2, io2, q_off, nq, lp, status, st);
+    if (rc != DSA_OK) return rc;
+    if (launch_finalize(rs.s2, p->topk, sorted, lp.logs, lp.cnt, lp.thr, out_idx, out_score,
+                        OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
+      return DSA_ERR_CUDA;
+  }
   return DSA_OK;
 }
 
@@ -1173,6 +1302,68 @@ int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
                         OutMap{nq, p->n_q, q_off}, status, st) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
+  return finish(p, workspace, st);
+}
+
+int lisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+               const float* w, int32_t* out_idx, float* out_score, int32_t* out_pool,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RouteLayout L;
+  int rc = route_begin(p, DSA_ALGO_LISA, rp, q, k, w, out_idx, out_score, workspace,
+                       workspace_bytes, st, &L);
+  if (rc != DSA_OK) return rc;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  rc = run_pseudo(p, L, q, w, nullptr, ws, st);
+  if (rc != DSA_OK) return rc;
+  rc = run_pseudo_stages(p, L, q, k, w, out_idx, out_score, out_pool, ws, st);
+  if (rc != DSA_OK) return rc;
+  return finish(p, workspace, st);
+}
+
+int resmisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, const void* k,
+                  const float* w, int32_t* out_idx, float* out_score, int32_t* out_heads,
+                  float* out_S, void* workspace, size_t workspace_bytes, void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  RouteLayout L;
+  int rc = route_begin(p, DSA_ALGO_RESMISA, rp, q, k, w, out_idx, out_score, workspace,
+                       workspace_bytes, st, &L);
+  if (rc != DSA_OK) return rc;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  const RouteCfg& c = L.c;
+  int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
+  uint16_t* ext_run = reinterpret_cast<uint16_t*>(ws + L.off_extrun);
+  uint16_t* ext_full = reinterpret_cast<uint16_t*>(ws + L.off_extfull);
+  if (c.res_r > 0) {
+    const int nb = (p->n_k + (1 << c.bsX) - 1) >> c.bsX;
+    block_extrema_kernel<<<dim3((unsigned)nb, (unsigned)p->batch), 128, 0, st>>>(
+        reinterpret_cast<const uint16_t*>(k), p->n_k, c.bsX, ext_run, ext_full, c.nblkX);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+    ResRouterArgs ra{};
+    ra.batch = p->batch;
+    ra.n_q = p->n_q;
+    ra.n_tok = p->n_k;
+    ra.H = p->heads;
+    ra.r = c.res_r;
+    ra.bs_shift = c.bsX;
+    ra.nblk_full = c.nblkX;
+    ra.q_pos0 = p->q_pos0;
+    ra.k_len = p->k_len;
+    ra.q = reinterpret_cast<const uint16_t*>(q);
+    ra.w = w;
+    ra.ext_full = ext_full;
+    ra.ext_run = ext_run;
+    ra.heads = heads;
+    ra.S = out_S;
+    const int rpc = kResThreads / p->heads;
+    const long long ctas = (long long)p->batch * ((p->n_q + rpc - 1) / rpc);
+    residual_router_kernel<<<(unsigned)ctas, kResThreads, 0, st>>>(ra);
+    if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  }
+  rc = run_pseudo(p, L, q, w, heads, ws, st);
+  if (rc != DSA_OK) return rc;
+  rc = run_pseudo_stages(p, L, q, k, w, out_idx, out_score, nullptr, ws, st);
+  if (rc != DSA_OK) return rc;
   return finish(p, workspace, st);
 }
 

@@ -687,26 +687,21 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const int s = ucount % NS;
           if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5, a.wait_cycles)) { ok = false; break; }
           tc_fence_after();
-          // descriptor low words: one add per MMA (32 bytes of K per k-step = 2)
-          const uint32_t qlo = sdesc_lo(smem_u32(Qs + gg * Cfg::A * qcols * 128));
+          const uint32_t qbase = smem_u32(Qs + gg * Cfg::A * qcols * 128);
           // one accumulator block of ncols columns per key tile of the stage
           const int nvalid = kPairs ? min(KT, g.ntiles - (u / a.G) * KT) : 1;
           for (int j = 0; j < nvalid; ++j) {
             const uint32_t d = tmem_base + s * a.stage_cols + j * ncols;
-            const uint32_t klo = sdesc_lo(smem_u32(Ks + (slot * KT + j) * Cfg::A * 16384));
+            const uint32_t kbase = smem_u32(Ks + (slot * KT + j) * Cfg::A * 16384);
 #pragma unroll
             for (int at = 0; at < Cfg::A; ++at) {
-              const uint32_t qat = qlo + (uint32_t)(at * qcols * 8);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint32_t alo = klo + (uint32_t)(at * 1024 + kk * 2);
+                const uint64_t ad = make_sdesc(kbase + at * 16384 + kk * 32);
 #pragma unroll
                 for (int pt = 0; pt < PARTS; ++pt) {
-                  const uint32_t blo = qat + (uint32_t)(pt * ncols * 8 + kk * 2);
-                  if (at == 0 && kk == 0 && pt == 0)
-                    tc_mma_lo<KIND, 0>(d, alo, blo, idesc);
-                  else
-                    tc_mma_lo<KIND, 1>(d, alo, blo, idesc);
+                  const uint64_t bd = make_sdesc(qbase + (at * qcols + pt * ncols) * 128 + kk * 32);
+                  tc_mma<KIND>(d, ad, bd, idesc, (at | kk | pt) != 0);
                 }
               }
             }

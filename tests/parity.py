@@ -68,7 +68,7 @@ class Agreement(NamedTuple):
 
 
 def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_score64, tol,
-                     heads=None, legal=None, label="", check_scores=True):
+                     heads=None, legal=None, label="", check_scores=True, score_fn=None):
     """Check the tolerance rule row by row; returns Agreement(iou, max_rel).
 
     heads: per-row head lists [n_rows, h] for routed scores (None: all heads).
@@ -76,7 +76,10 @@ def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_
     check_scores=False measures without asserting the score and near-cut-off
     rules (a comparison against operands the GPU did not see, e.g. the
     unquantised values of an fp8 run, whose differences are the quantisation's);
-    count, uniqueness, legality and order are still asserted."""
+    count, uniqueness, legality and order are still asserted.
+    score_fn(a, rows_v, idx) -> fp64 reference scores of row a at the listed keys,
+    for methods whose score is not the DSA score over `heads` (LISA's linear term,
+    ResMiSA's I^); nu then stays the one of `heads` (None: every head)."""
     p = inp.prob
     ious = []
     max_rel = 0.0
@@ -97,7 +100,8 @@ def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_
         assert np.all((g_set >= 0) & (g_set < n_legal)), f"row {row}: illegal index"
         hrow = None if heads is None else np.repeat(np.asarray(heads[a])[None], nv, 0)
         rows_v = np.full(nv, row, np.int64)
-        ref_at_g = oracle.score_pairs(inp, rows_v, g_set, hrow)
+        ref_at_g = (oracle.score_pairs(inp, rows_v, g_set, hrow) if score_fn is None
+                    else score_fn(a, rows_v, g_set))
         scale_g = np.maximum(np.abs(ref_at_g), oracle.nu_pairs(inp, rows_v, g_set, hrow))
         err = np.abs(gs[:nv].astype(np.float64) - ref_at_g)
         rel = err / scale_g
@@ -122,7 +126,8 @@ def within_tolerance(inp: oracle.Inputs, rows, gpu_idx, gpu_score, ref_idx, ref_
                 continue
             rr = np.full(len(group), row, np.int64)
             hh = None if heads is None else np.repeat(np.asarray(heads[a])[None], len(group), 0)
-            v = oracle.score_pairs(inp, rr, group, hh)
+            v = (oracle.score_pairs(inp, rr, group, hh) if score_fn is None
+                 else score_fn(a, rr, group))
             e_s = tol * np.maximum(np.abs(v), oracle.nu_pairs(inp, rr, group, hh))
             far = np.abs(v - cutoff) > e_s + e_kth
             assert not np.any(far), (f"row {row}: token {group[far][0]} differs from the "

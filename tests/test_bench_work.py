@@ -76,3 +76,17 @@ def test_hisa_work():
     assert dots == sum(parts)
     assert [round(2 * 128 * x / 1e12, 2) for x in parts] == [0.14, 0.28, 2.13]
     assert abs(flops / 1e12 - 2.55) < 0.01
+
+
+def test_lisa_and_resmisa_work():
+    """LISA: one fused-query dot per legal key; LISA-dagger adds H min(M, t + 1);
+    ResMiSA: H M_t block bounds + (1 + r) dots per legal key."""
+    L = 131072
+    p = _shape(1, L, L, 64)
+    pairs = L * (L + 1) // 2
+    _, dots, _ = bench.algorithmic_work(p, bench.WORKLOADS["lisa_prefill_128k"])
+    assert dots == pairs
+    _, dots, _ = bench.algorithmic_work(p, bench.WORKLOADS["lisa_dagger_prefill_128k"])
+    assert dots == pairs + 64 * _min_sum(L, 8192)
+    _, dots, _ = bench.algorithmic_work(p, bench.WORKLOADS["resmisa_prefill_128k"])
+    assert dots == 64 * _ceil_sum(L, 1024) + 8 * pairs

@@ -705,3 +705,18 @@ def test_lisa_and_resmisa_cost_counts_match_page_arithmetic(oracle_mod):
     ld = oracle_mod.lisa(inp, 2048, pool_m=g["pool"])["dots"][0]
     assert ld == g["lisa_dagger_dots_per_query"]
     assert round(100.0 * ld / g["dsa_dots_per_query"], 2) == g["lisa_dagger_percent"]
+
+
+def test_pairwise_lisa_and_resmisa_scores_match_the_rankings(oracle_mod):
+    """The pairwise scores the tolerance checks use are the ones the row
+    functions rank by (same definitions, evaluated at the selected tokens)."""
+    p = gen.normal_problem(99, 1, 24, 90, 8, 32, 10, q_pos0=[50])
+    inp = oracle_mod.Inputs(p)
+    rows = np.repeat(np.arange(p.n_q), p.topk)
+    a = oracle_mod.lisa(inp, p.topk)
+    assert np.array_equal(oracle_mod.linear_pairs(inp, rows, a["idx"].ravel()),
+                          a["score64"].ravel())
+    b = oracle_mod.resmisa(inp, p.topk, 16, 3)
+    hh = np.repeat(b["heads"], p.topk, 0)
+    assert np.array_equal(oracle_mod.resmisa_pairs(inp, rows, b["idx"].ravel(), hh),
+                          b["score64"].ravel())
