@@ -43,7 +43,7 @@
  *     ascending) — the lower index wins a tie — followed by padding (index -1,
  *     score -inf).  The entries come in an unspecified order unless
  *     DSA_FLAG_SORTED is set, which orders them by (score descending, index
- *     ascending).  Sparse attention consumes the set, so order is optional
+ *     ascending), or DSA_FLAG_BY_POSITION, which orders them by index.  Sparse attention consumes the set, so order is optional
  *     ("PaperTrace 2.2.2", section 2.2: indices returned by the top-k are
  *     unordered or score-ordered).  -0.0 is written as +0.0.  The reported
  *     score is the one the final selection used: the full I for dsa_index,
@@ -107,6 +107,11 @@ enum {
 /* problem.flags */
 #define DSA_FLAG_CHECK 1u  /* validate scales/lengths on device, synchronise, return device status */
 #define DSA_FLAG_SORTED 2u /* order each row's top-k by (score desc, index asc) */
+/* Order each row's top-k by token position (index ascending), the order in which
+ * a sparse attention kernel gathers the selected keys most contiguously
+ * ("PaperTrace 2.2.2", section 2.2: re-sorting score-ordered indices by
+ * position makes the gather more contiguous).  Not with DSA_FLAG_SORTED. */
+#define DSA_FLAG_BY_POSITION 4u
 /* For tests of the timeout path only, never in production: dsa_index /
  * dsa_index_scan run with a wait budget of about 1 ms instead of about 4 s, and
  * the scan's first CTA withholds one stage of keys, so its bounded waits run

@@ -71,6 +71,8 @@ def lib():
         _lib.orc_resmisa_rows.argtypes = [vp, i32, i32, i32, vp, i64, vp, vp, vp, vp, vp, vp, vp]
         _lib.orc_linear_pairs.argtypes = [vp, vp, vp, i64, vp]
         _lib.orc_resmisa_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
+        _lib.orc_sparse_mla.argtypes = [vp, vp, vp, i64, i32, i32, i32, i32, i32, i32,
+                                        C.c_double, vp, vp, vp, vp]
         _lib.orc_residual_bounds.restype = C.c_int64
         _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_score_row.restype = C.c_int64
@@ -314,5 +316,25 @@ def split_query(x: np.ndarray, x_dtype: int) -> np.ndarray:
     dim = x.shape[-1]
     out = np.empty(x.shape, np.float64)
     rc = lib().orc_split_query(_p(x), x_dtype, x.size // dim, dim, _p(out))
+    assert rc == 0
+    return out
+
+
+def sparse_mla(q, kv, idx, scale, dv, tps):
+    """Naive gather attention over fixed candidate sets (fp64).
+
+    q [T, heads, dqk] and kv [batch, n_k, dqk] as uint16 bf16 words; idx [T, k]
+    int32 (-1 empty); token t belongs to sequence t // tps.  Returns dict(o
+    [T, heads, dv], lse, max, den [T, heads])."""
+    q = np.ascontiguousarray(q, np.uint16)
+    kv = np.ascontiguousarray(kv, np.uint16)
+    idx = np.ascontiguousarray(idx, np.int32)
+    T, H, dqk = q.shape
+    n_k = kv.shape[1]
+    topk = idx.shape[1]
+    out = dict(o=np.empty((T, H, dv), np.float64), lse=np.empty((T, H), np.float64),
+               max=np.empty((T, H), np.float64), den=np.empty((T, H), np.float64))
+    rc = lib().orc_sparse_mla(_p(q), _p(kv), _p(idx), T, tps, n_k, H, dqk, dv, topk, float(scale),
+                              _p(out["o"]), _p(out["lse"]), _p(out["max"]), _p(out["den"]))
     assert rc == 0
     return out

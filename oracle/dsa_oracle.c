@@ -41,6 +41,11 @@
  *         -q_{t,j} . k over the block (q+ = max(q, 0), q- = max(-q, 0));
  *         S_{t,j} = |w_{t,j}| max_b ReLU(U^-_{t,b,j}); the top-r heads A_t;
  *         I^_{t,s} = l_{t,s} + sum_{j in A_t} w_{t,j} ReLU(-q_{t,j} . k_s).
+ *  [SMLA] "PaperTrace 2.2.2", section 2.3 "end-to-end acceptance", second step:
+ *         Sparse MLA on a fixed candidate set S_t, checked by logits, row
+ *         maximum, softmax denominator and output against a naive gather
+ *         attention; section 2.2: the selected positions feed Sparse MLA,
+ *         which reads the latent KV at those positions.
  *  [FP8]  "PaperTrace 2.2.2", section 2.3 "from formula to FP8 cache":
  *         k^ = round(k/a), FP8 data plus scale, higher-precision accumulation.
  *         The e4m3 code follows the OCP 8-bit floating point specification
@@ -988,6 +993,71 @@ int orc_resmisa_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* 
     }
     out[a] = v;
     free(g);
+  }
+  return ORC_OK;
+}
+
+/* --------------------------------------------------------- Sparse MLA -- */
+
+/* [SMLA] Naive gather attention over a fixed candidate set.  Token t (of
+ * sequence b = t / tps) with query heads q[t, h, 0:dqk] attends to the cached
+ * latent rows kv[b, s, 0:dqk] of its selected positions s = idx[t, i] >= 0
+ * (entries < 0 are empty):
+ *   x_s = scale * q_h . kv_s                     (logits)
+ *   m   = max_s x_s,  den = sum_s exp(x_s - m)   (row maximum, denominator)
+ *   o_h = sum_s exp(x_s - m) kv_s[0:dv] / den    (the value is the latent's
+ *                                                 first dv dimensions)
+ *   lse = m + log(den)
+ * q and kv are bf16 words; everything else fp64.  A token with no selected
+ * position gets o = 0, m = lse = -inf, den = 0.
+ * Reading: the value of MLA's absorbed form is the latent part of the cached
+ * row (the first dv of its dqk dimensions), the rope part joins the logits only. */
+int orc_sparse_mla(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int64_t T,
+                   int32_t tps, int32_t n_k, int32_t heads, int32_t dqk, int32_t dv, int32_t topk,
+                   double scale, double* out_o, double* out_lse, double* out_max,
+                   double* out_den) {
+  if (dv > dqk || tps < 1) return ORC_ERR;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t t = 0; t < T; ++t) {
+    int64_t b = t / tps;
+    double* x = (double*)malloc(sizeof(double) * (topk > 0 ? topk : 1));
+    int32_t* pos = (int32_t*)malloc(sizeof(int32_t) * (topk > 0 ? topk : 1));
+    for (int32_t i = 0; i < topk; ++i) {
+      int32_t s = idx[t * topk + i];
+      pos[i] = (s < 0 && MUT(43)) ? 0 : s;   /* planted mistake 43: empty read as position 0 */
+    }
+    for (int32_t h = 0; h < heads; ++h) {
+      const uint16_t* qh = q + (t * heads + h) * (int64_t)dqk;
+      double m = -INFINITY;
+      for (int32_t i = 0; i < topk; ++i) {
+        int32_t s = pos[i];
+        if (s < 0) { x[i] = -INFINITY; continue; }
+        const uint16_t* ks = kv + (b * n_k + s) * (int64_t)dqk;
+        double acc = 0.0;
+        for (int32_t c = 0; c < dqk; ++c) acc += bf16_value(qh[c]) * bf16_value(ks[c]);
+        x[i] = (MUT(40) ? 1.0 : scale) * acc;
+        if (x[i] > m) m = x[i];
+      }
+      double den = 0.0;
+      double* o = out_o + (t * heads + h) * (int64_t)dv;
+      for (int32_t c = 0; c < dv; ++c) o[c] = 0.0;
+      if (m > -INFINITY) {
+        for (int32_t i = 0; i < topk; ++i) {
+          if (x[i] == -INFINITY) continue;
+          double p = exp(x[i] - m);
+          den += p;
+          const uint16_t* ks = kv + (b * n_k + pos[i]) * (int64_t)dqk;
+          int32_t off = MUT(41) ? dqk - dv : 0;
+          for (int32_t c = 0; c < dv; ++c) o[c] += p * bf16_value(ks[off + c]);
+        }
+        for (int32_t c = 0; c < dv; ++c) o[c] /= den;
+      }
+      if (out_lse) out_lse[t * heads + h] = m > -INFINITY ? m + log(den) : -INFINITY;
+      if (out_max) out_max[t * heads + h] = m;
+      if (out_den) out_den[t * heads + h] = den;
+    }
+    free(pos);
+    free(x);
   }
   return ORC_OK;
 }

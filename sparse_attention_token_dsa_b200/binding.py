@@ -22,6 +22,7 @@ DSA_ALGO_DSA, DSA_ALGO_MISA, DSA_ALGO_MISA_DAGGER, DSA_ALGO_HISA = 0, 1, 2, 3
 DSA_ALGO_LISA, DSA_ALGO_RESMISA = 4, 5
 DSA_FLAG_CHECK = 1
 DSA_FLAG_SORTED = 2
+DSA_FLAG_BY_POSITION = 4
 DSA_FLAG_TEST_STALL = 0x80000000   # tests of the timeout path only (see include/dsaidx.h)
 
 

@@ -376,10 +376,17 @@ int validate_problem(const dsa_problem* p) {
   const bool split = (qd == DSA_BF16 || qd == DSA_F32) && kd == DSA_E4M3;
   if (!same && !split) return DSA_ERR_UNSUPPORTED;
   if (split && p->heads < 32) return DSA_ERR_UNSUPPORTED;
+  if ((p->flags & DSA_FLAG_SORTED) && (p->flags & DSA_FLAG_BY_POSITION)) return DSA_ERR_INVALID;
   return DSA_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Output order of a problem: 0 any, 1 (score desc, index asc), 2 index asc.
+int out_order(const dsa_problem* p) {
+  if (p->flags & DSA_FLAG_BY_POSITION) return 2;
+  return (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+}
 
 // Kind / split decision of a validated problem.
 void kind_of(const dsa_problem* p, MmaKind* kind, bool* split) {
@@ -858,7 +865,7 @@ int run_pseudo_stages(const dsa_problem* p, const RouteLayout& L, const void* q,
                       const float* w, int32_t* out_idx, float* out_score, int32_t* out_pool,
                       uint8_t* ws, cudaStream_t st) {
   int32_t* status = reinterpret_cast<int32_t*>(ws);
-  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  const int sorted = out_order(p);
   int32_t* pool = reinterpret_cast<int32_t*>(ws + L.off_list);
   for (int ci = 0; ci < L.n_chunks; ++ci) {
     const int q_off = ci * L.nq_c;
@@ -1065,7 +1072,7 @@ int dsa_index_select(const dsa_problem* p, int32_t* out_idx, float* out_score, v
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   const ScanPlan& pl = L.pl;
-  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  const int sorted = out_order(p);
   if (launch_finalize(pl, p->topk, sorted, reinterpret_cast<const uint64_t*>(ws + L.off_logs),
                       reinterpret_cast<const int32_t*>(ws + L.off_cnt),
                       reinterpret_cast<const unsigned long long*>(ws + L.off_thr), out_idx,
@@ -1121,7 +1128,7 @@ int misa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
   int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
   rc = run_router(p, L, q, k, w, heads, out_E, ws, st);
   if (rc != DSA_OK) return rc;
-  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  const int sorted = out_order(p);
   for (int ci = 0; ci < L.n_chunks; ++ci) {
     const int q_off = ci * L.nq_c;
     const int nq = p->n_q - q_off < L.nq_c ? p->n_q - q_off : L.nq_c;
@@ -1159,7 +1166,7 @@ int misa_dagger_index(const dsa_problem* p, const dsa_route_params* rp, const vo
   int32_t* heads = out_heads ? out_heads : reinterpret_cast<int32_t*>(ws + L.off_heads);
   rc = run_router(p, L, q, k, w, heads, nullptr, ws, st);
   if (rc != DSA_OK) return rc;
-  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  const int sorted = out_order(p);
   int32_t* pool = reinterpret_cast<int32_t*>(ws + L.off_list);
   for (int ci = 0; ci < L.n_chunks; ++ci) {
     const int q_off = ci * L.nq_c;
@@ -1232,7 +1239,7 @@ int hisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* q, 
   uint8_t* fullH = ws + L.off_fullH;
   rc = launch_pool(k, p, c.bsH, runH, fullH, c.nblkH, st);
   if (rc != DSA_OK) return rc;
-  const int sorted = (p->flags & DSA_FLAG_SORTED) ? 1 : 0;
+  const int sorted = out_order(p);
   int32_t* blocks = reinterpret_cast<int32_t*>(ws + L.off_list);
   for (int ci = 0; ci < L.n_chunks; ++ci) {
     const int q_off = ci * L.nq_c;

@@ -25,7 +25,7 @@ struct FinalArgs {
   int32_t topk;
   int32_t capw;          // entries per sub-log
   int32_t sort_cap;      // power of two >= topk
-  int32_t sorted;        // 1: order by (score desc, index asc); 0: any order
+  int32_t sorted;        // 1: order by (score desc, index asc); 2: by index asc; 0: any order
   const uint64_t* logs;  // [rows * C][nsub][capw]
   const int32_t* log_cnt;               // [rows * C][nsub]
   const unsigned long long* log_thr;    // [rows * C]
@@ -256,7 +256,17 @@ __global__ void __launch_bounds__(E <= 8 ? 1024 : NT)
       n = compact_ge<NT>(sp, sn, ns, t, out, &G->sc, tid, bar, nullptr);
     }
   }
-  if (a.sorted) sort_desc_regs<NT, E>(out, n, tid, bar);   // sort_cap == NT * E
+  if (a.sorted == 2) {
+    // position order: sort on (~index, score) — the composite with its halves
+    // swapped — descending, which is index ascending (indices are unique)
+    named_bar_sync(bar, NT);
+    for (int i = tid; i < n; i += NT) out[i] = (out[i] << 32) | (out[i] >> 32);
+    sort_desc_regs<NT, E>(out, n, tid, bar);
+    for (int i = tid; i < n; i += NT) out[i] = (out[i] << 32) | (out[i] >> 32);
+    named_bar_sync(bar, NT);
+  } else if (a.sorted) {
+    sort_desc_regs<NT, E>(out, n, tid, bar);   // sort_cap == NT * E
+  }
   const int64_t orow = (int64_t)(row / a.nq_c) * a.nq_total + a.q_off + row % a.nq_c;
   int32_t* oi = a.out_idx + orow * a.topk;
   float* os = a.out_score ? a.out_score + orow * a.topk : nullptr;

@@ -298,3 +298,24 @@ def test_expired_wait_returns_timeout_then_next_call_is_exact(B):
     ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
     parity.exact(idx.cpu().numpy().reshape(-1, p.topk), sc.cpu().numpy().reshape(-1, p.topk),
                  ri, rs)
+
+
+@pytest.mark.parametrize("topk", [128, 2048])
+def test_position_order_bit_exact(B, topk):
+    """DSA_FLAG_BY_POSITION: each row is the oracle's top-k set in ascending token
+    order, scores carried with their tokens, padding last."""
+    p = gen.integer_problem(9, 2, 200, 3000, 64, 128, topk, q_pos0=[2800, 100],
+                            k_len=[3000, 2500], dtype=gen.BF16)
+    idx, sc = B.dsa_index(dev(p.q), dev(p.k), dev(p.w), p.topk, q_pos0=dev(p.q_pos0),
+                          k_len=dev(p.k_len), flags=B.DSA_FLAG_BY_POSITION | B.DSA_FLAG_CHECK)
+    import torch
+    torch.cuda.synchronize()
+    gi = idx.cpu().numpy().reshape(-1, p.topk)
+    gs = sc.cpu().numpy().reshape(-1, p.topk)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    for r in range(len(ri)):
+        nv = int(np.sum(ri[r] >= 0))
+        order = np.argsort(ri[r][:nv], kind="stable")
+        assert np.array_equal(gi[r][:nv], ri[r][:nv][order])
+        assert np.array_equal(gs[r][:nv], rs[r][:nv][order])
+        assert np.all(gi[r][nv:] == -1) and np.all(np.isneginf(gs[r][nv:]))

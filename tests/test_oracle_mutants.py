@@ -54,6 +54,9 @@ MUTANTS = {
     37: "residual router weighs the bound by signed w instead of |w|",
     38: "residual bound blocks reach past the causal position",
     39: "LISA-dagger pool one candidate short",
+    40: "sparse attention logits without the softmax scale",
+    41: "sparse attention value taken from the wrong end of the latent row",
+    43: "sparse attention reads an empty (-1) entry as position 0",
 }
 
 

@@ -720,3 +720,80 @@ def test_pairwise_lisa_and_resmisa_scores_match_the_rankings(oracle_mod):
     hh = np.repeat(b["heads"], p.topk, 0)
     assert np.array_equal(oracle_mod.resmisa_pairs(inp, rows, b["idx"].ravel(), hh),
                           b["score64"].ravel())
+
+
+# --------------------------------------------------- Sparse MLA (fixed set) --
+
+def _bf(x):
+    return gen.f32_to_bf16_bits(np.asarray(x, np.float32))
+
+
+def test_sparse_mla_single_key_is_its_value(oracle_mod):
+    """One selected position: the softmax weight is 1, the output is that key's
+    latent value and lse is its logit."""
+    rng = np.random.default_rng(20)
+    q = _bf(rng.integers(-2, 3, size=(3, 2, 16)))
+    kv = _bf(rng.integers(-2, 3, size=(1, 10, 16)))
+    idx = np.full((3, 4), -1, np.int32)
+    idx[:, 1] = [7, 0, 9]
+    out = oracle_mod.sparse_mla(q, kv, idx, 0.5, 12, 3)
+    kvf = gen.bf16_bits_to_f32(kv).astype(np.float64)
+    qf = gen.bf16_bits_to_f32(q).astype(np.float64)
+    for t, s in enumerate([7, 0, 9]):
+        assert np.array_equal(out["o"][t], np.repeat(kvf[0, s, :12][None], 2, 0))
+        assert np.array_equal(out["lse"][t], 0.5 * qf[t] @ kvf[0, s])
+        assert np.array_equal(out["den"][t], [1.0, 1.0])
+
+
+def test_sparse_mla_zero_query_is_the_mean_value(oracle_mod):
+    """q = 0: every logit is 0, the weights are uniform, o is the mean of the
+    selected values and lse = log(n)."""
+    rng = np.random.default_rng(21)
+    kv = _bf(rng.standard_normal((2, 50, 32)))
+    q = np.zeros((4, 3, 32), np.uint16)
+    idx = np.array([[3, 9, 12, -1], [0, -1, -1, -1], [5, 6, 7, 8], [49, 1, -1, 2]], np.int32)
+    out = oracle_mod.sparse_mla(q, kv, idx, 0.1, 24, 2)     # tokens 0-1: seq 0, 2-3: seq 1
+    kvf = gen.bf16_bits_to_f32(kv).astype(np.float64)
+    for t in range(4):
+        sel = idx[t][idx[t] >= 0]
+        want = kvf[t // 2, sel, :24].mean(0)
+        np.testing.assert_allclose(out["o"][t], np.repeat(want[None], 3, 0), rtol=1e-14, atol=1e-15)
+        np.testing.assert_allclose(out["lse"][t], np.log(len(sel)), rtol=1e-14)
+
+
+def test_sparse_mla_two_keys_closed_form(oracle_mod):
+    """Two positions whose logits differ by log 3 (q . k = 0 and q . k = ln 3 / scale
+    chosen exactly): weights 1/4 and 3/4, row max ln 3, denominator 4/3."""
+    d = 4
+    scale = 0.25
+    q = np.zeros((1, 1, d), np.float32)
+    q[0, 0, 0] = 1.0
+    kv = np.zeros((1, 2, d), np.float32)
+    kv[0, 0] = [0.0, 1.0, 0.0, 0.0]
+    kv[0, 1] = [4.0, 0.0, 1.0, 0.0]                          # logit 1.0 vs 0.0
+    out = oracle_mod.sparse_mla(_bf(q), _bf(kv), np.array([[0, 1]], np.int32), scale, 3, 1)
+    e = np.exp(1.0)
+    w0, w1 = 1.0 / (1.0 + e), e / (1.0 + e)
+    np.testing.assert_allclose(out["o"][0, 0], w0 * kv[0, 0, :3] + w1 * kv[0, 1, :3], rtol=1e-15)
+    assert out["max"][0, 0] == 1.0
+    np.testing.assert_allclose(out["den"][0, 0], 1.0 + 1.0 / e, rtol=1e-15)
+    np.testing.assert_allclose(out["lse"][0, 0], 1.0 + np.log(1.0 + 1.0 / e), rtol=1e-15)
+
+
+def test_sparse_mla_ignores_order_and_empty_entries(oracle_mod):
+    """The candidate set is a set: permuting it, or interleaving empty (-1)
+    entries, leaves every output unchanged up to summation order."""
+    rng = np.random.default_rng(22)
+    q = _bf(rng.standard_normal((5, 4, 64)))
+    kv = _bf(rng.standard_normal((1, 300, 64)))
+    idx = np.stack([rng.permutation(300)[:40] for _ in range(5)]).astype(np.int32)
+    a = oracle_mod.sparse_mla(q, kv, idx, 0.125, 48, 5)
+    idx2 = np.full((5, 64), -1, np.int32)
+    for t in range(5):
+        slots = np.sort(rng.permutation(64)[:40])
+        idx2[t, slots] = rng.permutation(idx[t])
+    b = oracle_mod.sparse_mla(q, kv, idx2, 0.125, 48, 5)
+    for key in ("o", "lse", "max", "den"):
+        np.testing.assert_allclose(a[key], b[key], rtol=1e-12, atol=1e-13)
+    z = oracle_mod.sparse_mla(q, kv, np.full((5, 3), -1, np.int32), 0.125, 48, 5)
+    assert np.all(z["o"] == 0.0) and np.all(np.isneginf(z["lse"])) and np.all(z["den"] == 0.0)
