@@ -389,6 +389,65 @@ def run_reference(args, w, p):
 
 # ------------------------------------------------------------------ GPU arm --
 
+MLA_WORKLOAD = dict(
+    desc="Sparse MLA prefill chunk: 4096 query tokens x 128 heads, 2048 selected positions "
+         "each (causal, position order) from a 131072-row latent cache, d_qk 576 (512 latent "
+         "+ 64 rope), d_v 512, bf16, softmax scale 1/sqrt(192)",
+    n_q=4096, n_k=131072, heads=128, topk=2048, seed=5)
+
+
+def mla_line(steps, warmup, dev):
+    """Sparse MLA over fixed selected positions (the indexer's consumer), timed
+    with CUDA events; tensor roofline by its algorithmic FLOPs (2 per
+    multiply-add over the 576 logit and 512 value dimensions of every selected
+    (token, head, position)), and the gathered bytes (each selected row once
+    per token)."""
+    import torch
+    from sparse_attention_token_dsa_b200 import binding as B
+    from sparse_attention_token_dsa_b200 import workloads
+    w = MLA_WORKLOAD
+    pr = workloads.mla_problem(w["n_q"], w["n_k"], w["heads"], w["topk"], seed=w["seed"])
+    q = torch.from_numpy(pr["q"].view(np.int16)).to(dev).view(torch.bfloat16)
+    kv = torch.from_numpy(pr["kv"].view(np.int16)).to(dev).view(torch.bfloat16)
+    idx = torch.from_numpy(pr["idx"]).to(dev)
+    out = torch.empty((w["n_q"], w["heads"], 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w["n_q"], w["heads"]), dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        B.sparse_mla(q, kv, idx, pr["scale"], tokens_per_seq=pr["tps"], out=out, out_lse=lse,
+                     workspace=ws, stream=stream)
+
+    for _ in range(max(warmup, 3)):
+        call()
+    st = B.dsa_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    nsel = int((pr["idx"] >= 0).sum())
+    flops = 2.0 * w["heads"] * nsel * (576 + 512)
+    nbytes = nsel * 576 * 2
+    pk = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w["desc"], "value": ms, "unit": "ms/chunk", "ms_per_step": ms,
+            "steps": steps, "warmup": max(warmup, 3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16"],
+                         "peak_source": f"{pk['src']} bf16 burst",
+                         "work": f"{flops / 1e12:.3f} TFLOP per call",
+                         "gathered_gb_per_s": nbytes / (ms * 1e-3) / 1e9,
+                         "kernel": "sparse_mla_kernel", "kernel_ms": ms, "traffic": None},
+            "gpu_launches": steps}
+
+
 # in an order that reuses generated problems: MISA and MISA-dagger share the
 # headline problem, stacked HISA shares HISA's clustered keys
 SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "lisa_prefill_128k",
@@ -858,6 +917,9 @@ def main():
                 cache[("dense", w["seed"], w["L"], w["H"], w.get("keys", "iid"), False)] = dense
             line["secondary"] = [secondary_line(n, min(args.steps, 5), args.warmup, dev, cache)
                                  for n in SECONDARY]
+            cache.clear()
+            torch.cuda.empty_cache()
+            line["secondary"].append(mla_line(min(args.steps, 5), args.warmup, dev))
             line["gpu_launches"] += sum(s["gpu_launches"] for s in line["secondary"])
             cache.clear()
         if not args.no_cpu_baseline:

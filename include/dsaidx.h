@@ -274,6 +274,42 @@ int resmisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* 
                   const float* w, int32_t* out_idx, float* out_score, int32_t* out_heads,
                   float* out_S, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Sparse MLA on a fixed set of selected positions ("PaperTrace 2.2.2", section
+ * 2.2: the indexer's top-k positions feed Sparse MLA, which reads the latent
+ * KV at those positions; section 2.3, acceptance step two: with the set fixed,
+ * check logits, row maximum, softmax denominator and output against a naive
+ * gather attention).  Token t (sequence t / tokens_per_seq) with absorbed
+ * query heads q_{t,h} attends to the cached rows kv_s of its selected
+ * positions s = idx[t, i] (entries < 0 or >= n_k are empty):
+ *     x_s = scale * q_{t,h} . kv_s,   o_{t,h} = sum_s softmax(x)_s kv_s[0:dim_v],
+ *     lse_{t,h} = log sum_s exp(x_s)      (natural log; -inf for an empty set)
+ * The value is the latent part of the row (its first dim_v dimensions); the
+ * trailing dim_qk - dim_v (rope) dimensions join the logits only.
+ *   q   [batch * tokens_per_seq, heads, dim_qk] bf16
+ *   kv  [batch, n_k, dim_qk] bf16
+ *   idx [batch * tokens_per_seq, topk] int32 (any order; DSA_FLAG_BY_POSITION
+ *       output gathers most contiguously)
+ *   out [batch * tokens_per_seq, heads, dim_v] bf16; out_lse [.., heads] fp32 or NULL
+ * Supported: dim_qk == 576, dim_v == 512 (MLA latent 512 + rope 64), heads <= 128.
+ * The softmax weights enter the value product in bf16 (fp32 accumulation).
+ * workspace: >= 256 bytes (status word; DSA_FLAG_CHECK synchronises and
+ * returns it). */
+typedef struct {
+  int32_t batch;
+  int32_t tokens_per_seq;
+  int32_t n_k;
+  int32_t heads;
+  int32_t dim_qk;
+  int32_t dim_v;
+  int32_t topk;
+  float scale;
+  uint32_t flags;
+} dsa_mla_problem;
+
+int dsa_sparse_mla(const dsa_mla_problem* p, const void* q, const void* kv, const int32_t* idx,
+                   void* out, float* out_lse, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
 /* Operand preparation for the FP8 path: per-row scale a = amax/448 (amax == 0
  * gives a = 1), code = round-to-nearest-even, saturating e4m3 of x/a, both
  * divisions in IEEE fp32 ("PaperTrace 2.2.2", section 2.3 "from formula to

@@ -39,6 +39,12 @@ class DsaRouteParams(C.Structure):
                 ("res_block", C.c_int32), ("res_r", C.c_int32)]
 
 
+class DsaMlaProblem(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("tokens_per_seq", C.c_int32), ("n_k", C.c_int32),
+                ("heads", C.c_int32), ("dim_qk", C.c_int32), ("dim_v", C.c_int32),
+                ("topk", C.c_int32), ("scale", C.c_float), ("flags", C.c_uint32)]
+
+
 class DsaError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {status_string(status)} ({status})")
@@ -68,12 +74,13 @@ def _load():
     lib.lisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.resmisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
+    lib.dsa_sparse_mla.argtypes = [C.POINTER(DsaMlaProblem), vp, vp, vp, vp, vp, vp, sz, vp]
     for f in ("dsa_read_status", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
               "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
               "misa_dagger_index", "hisa_index", "lisa_index", "resmisa_index",
-              "dsa_quantize_e4m3"):
+              "dsa_quantize_e4m3", "dsa_sparse_mla"):
         getattr(lib, f).restype = C.c_int
     return lib
 
@@ -296,6 +303,27 @@ def resmisa_index(q, k, w, topk, block, r, q_pos0=None, k_len=None, flags=0, out
                              _ptr(sc), _ptr(out_heads), _ptr(out_S), _ptr(ws), ws.numel(),
                              _stream(stream)), "resmisa_index")
     return idx, sc
+
+
+def sparse_mla(q, kv, idx, scale, tokens_per_seq=None, flags=0, out=None, out_lse=None,
+               workspace=None, stream=None):
+    """Sparse MLA over fixed selected positions.  q [T, heads, 576] bf16,
+    kv [batch, n_k, 576] bf16, idx [T, k] int32 (-1 empty).  Returns (out
+    [T, heads, 512] bf16, lse [T, heads] fp32)."""
+    _args(q=(q, (torch.bfloat16,)), kv=(kv, (torch.bfloat16,)), idx=(idx, _I32),
+          out=(out, (torch.bfloat16,)), out_lse=(out_lse, _F32), workspace=(workspace, _U8))
+    T, H, dqk = q.shape
+    B, n_k, _ = kv.shape
+    tps = T // B if tokens_per_seq is None else tokens_per_seq
+    p = DsaMlaProblem(B, tps, n_k, H, dqk, 512, idx.shape[1], float(scale), flags)
+    if out is None:
+        out = torch.empty((T, H, 512), dtype=torch.bfloat16, device=q.device)
+    if out_lse is None:
+        out_lse = torch.empty((T, H), dtype=torch.float32, device=q.device)
+    ws = _workspace(256, q.device, workspace)
+    _check(lib.dsa_sparse_mla(C.byref(p), _ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(out_lse),
+                              _ptr(ws), ws.numel(), _stream(stream)), "dsa_sparse_mla")
+    return out, out_lse
 
 
 def dsa_quantize_e4m3(x: torch.Tensor, stream=None):

@@ -13,6 +13,7 @@
 #include "../../include/dsaidx.h"
 #include "common.cuh"
 #include "finalize.cuh"
+#include "mla.cuh"
 #include "prep.cuh"
 #include "resid.cuh"
 #include "route.cuh"
@@ -213,6 +214,35 @@ bool make_map(CUtensorMap* m, const void* base, int esz, uint64_t rows, uint32_t
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D map over the query of sparse attention, [T][heads][576] bf16: box of 64
+// dimensions x 128 head rows x one token, 128-byte swizzle; head rows past
+// `heads` read as zeros.
+bool make_map_q3d(CUtensorMap* m, const void* base, uint64_t tokens, uint64_t heads) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kMlaDqk, (cuuint64_t)heads, (cuuint64_t)tokens};
+  cuuint64_t strides[2] = {(cuuint64_t)kMlaDqk * 2, (cuuint64_t)heads * kMlaDqk * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over the cached latent rows [rows][576] bf16 for four-row gathers:
+// a one-row-high box of 64 dimensions.
+bool make_map_kv(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kMlaDqk, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kMlaDqk * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1372,6 +1402,48 @@ int resmisa_index(const dsa_problem* p, const dsa_route_params* rp, const void* 
   rc = run_pseudo_stages(p, L, q, k, w, out_idx, out_score, nullptr, ws, st);
   if (rc != DSA_OK) return rc;
   return finish(p, workspace, st);
+}
+
+int dsa_sparse_mla(const dsa_mla_problem* p, const void* q, const void* kv, const int32_t* idx,
+                   void* out, float* out_lse, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  if (!p || !q || !kv || !idx || !out) return DSA_ERR_INVALID;
+  if (p->batch < 1 || p->tokens_per_seq < 1 || p->n_k < 1 || p->heads < 1 || p->topk < 1)
+    return DSA_ERR_INVALID;
+  if (p->dim_qk != kMlaDqk || p->dim_v != kMlaDv || p->heads > 128 || p->topk > 65536)
+    return DSA_ERR_UNSUPPORTED;
+  const long long T = (long long)p->batch * p->tokens_per_seq;
+  if (T * 2 > 0x7fffffffll || (long long)p->batch * p->n_k > (1ll << 31)) return DSA_ERR_UNSUPPORTED;
+  if (!(p->scale > 0.f) || !(p->scale < 3.0e38f)) return DSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(idx))
+    return DSA_ERR_INVALID;
+  if (!workspace || workspace_bytes < kWsHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t* status = reinterpret_cast<int32_t*>(workspace);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap qm, km;
+  if (!make_map_q3d(&qm, q, (uint64_t)T, (uint64_t)p->heads)) return DSA_ERR_CUDA;
+  if (!make_map_kv(&km, kv, (uint64_t)p->batch * p->n_k)) return DSA_ERR_CUDA;
+  MlaArgs a{};
+  a.T = (int32_t)T;
+  a.tps = p->tokens_per_seq;
+  a.n_k = p->n_k;
+  a.heads = p->heads;
+  a.topk = p->topk;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.idx = idx;
+  a.out = reinterpret_cast<uint16_t*>(out);
+  a.lse = out_lse;
+  a.status = status;
+  const int smem = (int)mla_smem_bytes();
+  if (cudaFuncSetAttribute(sparse_mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return DSA_ERR_CUDA;
+  sparse_mla_kernel<<<(unsigned)(T * 2), kMlaThreads, smem, st>>>(qm, km, a);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(workspace, stream);
+  return DSA_OK;
 }
 
 }  // extern "C"
