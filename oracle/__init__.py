@@ -73,6 +73,7 @@ def lib():
         _lib.orc_resmisa_pairs.argtypes = [vp, vp, vp, i64, vp, i32, vp]
         _lib.orc_sparse_mla.argtypes = [vp, vp, vp, i64, i32, i32, i32, i32, i32, i32,
                                         C.c_double, vp, vp, vp, vp]
+        _lib.orc_indexer_backward.argtypes = [vp, vp, vp, i32, vp, vp, vp]
         _lib.orc_residual_bounds.restype = C.c_int64
         _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_score_row.restype = C.c_int64
@@ -336,5 +337,19 @@ def sparse_mla(q, kv, idx, scale, dv, tps):
                max=np.empty((T, H), np.float64), den=np.empty((T, H), np.float64))
     rc = lib().orc_sparse_mla(_p(q), _p(kv), _p(idx), T, tps, n_k, H, dqk, dv, topk, float(scale),
                               _p(out["o"]), _p(out["lse"]), _p(out["max"]), _p(out["den"]))
+    assert rc == 0
+    return out
+
+
+def indexer_backward(inp: Inputs, sel, grad):
+    """Gradients of sum_{t, s in S_t} g_{t,s} I_{t,s}: dict(dq [rows, H, d],
+    dk [batch, n_k, d], dw [rows, H]) in fp64."""
+    p = inp.prob
+    sel = np.ascontiguousarray(sel, np.int32).reshape(p.batch * p.n_q, -1)
+    grad = np.ascontiguousarray(grad, np.float32).reshape(sel.shape)
+    out = dict(dq=np.empty((p.batch * p.n_q, p.heads, p.dim)),
+               dk=np.empty((p.batch, p.n_k, p.dim)), dw=np.empty((p.batch * p.n_q, p.heads)))
+    rc = lib().orc_indexer_backward(inp.ref, _p(sel), _p(grad), sel.shape[1], _p(out["dq"]),
+                                    _p(out["dk"]), _p(out["dw"]))
     assert rc == 0
     return out

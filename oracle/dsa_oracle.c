@@ -41,6 +41,14 @@
  *         -q_{t,j} . k over the block (q+ = max(q, 0), q- = max(-q, 0));
  *         S_{t,j} = |w_{t,j}| max_b ReLU(U^-_{t,b,j}); the top-r heads A_t;
  *         I^_{t,s} = l_{t,s} + sum_{j in A_t} w_{t,j} ReLU(-q_{t,j} . k_s).
+ *  [BWD]  "PaperTrace 2.2.2", section 2.3 "why training gradients need
+ *         recomputation": with z_{t,s,j} = q_{t,j} . k_s, m = 1[z > 0] (the ReLU
+ *         derivative is 0 at 0) and an upstream gradient g_{t,s} on I_{t,s},
+ *         the chain rule through I = sum_j w_j ReLU(z_j) gives
+ *           dq_{t,j} = sum_s g_{t,s} w_{t,j} m_{t,s,j} k_s
+ *           dk_s     = sum_t sum_j g_{t,s} w_{t,j} m_{t,s,j} q_{t,j}
+ *           dw_{t,j} = sum_s g_{t,s} ReLU(z_{t,s,j})
+ *         over the selected set S_t (the sparse stage recomputes only there).
  *  [SMLA] "PaperTrace 2.2.2", section 2.3 "end-to-end acceptance", second step:
  *         Sparse MLA on a fixed candidate set S_t, checked by logits, row
  *         maximum, softmax denominator and output against a naive gather
@@ -994,6 +1002,46 @@ int orc_resmisa_pairs(const orc_inputs* in, const int64_t* rows, const int64_t* 
     out[a] = v;
     free(g);
   }
+  return ORC_OK;
+}
+
+/* ---------------------------------------------------- indexer backward -- */
+
+/* [BWD] Gradients of L = sum_t sum_{s in S_t} g_{t,s} I_{t,s} with respect to q,
+ * k and w, recomputing z over each row's selected positions sel [rows, topk]
+ * (entries < 0 ignored) with upstream gradients grad [rows, topk].
+ * dq [rows, heads, dim] and dw [rows, heads] are written; dk [batch, n_k, dim]
+ * is written too (zero where no row selected the key).  Rows are processed in
+ * order, so dk sums in a fixed order (single-threaded for that reason). */
+int orc_indexer_backward(const orc_inputs* in, const int32_t* sel, const float* grad,
+                         int32_t topk, double* dq, double* dk, double* dw) {
+  int64_t rows = (int64_t)in->batch * in->n_q;
+  memset(dq, 0, sizeof(double) * (size_t)rows * in->heads * in->dim);
+  memset(dw, 0, sizeof(double) * (size_t)rows * in->heads);
+  memset(dk, 0, sizeof(double) * (size_t)in->batch * in->n_k * in->dim);
+  double* kd = (double*)malloc(sizeof(double) * in->dim);
+  for (int64_t row = 0; row < rows; ++row) {
+    int32_t b = (int32_t)(row / in->n_q);
+    for (int32_t i = 0; i < topk; ++i) {
+      int32_t s = sel[row * topk + i];
+      if (s < 0) continue;
+      double g = (double)grad[row * topk + i];
+      for (int32_t c = 0; c < in->dim; ++c) kd[c] = k_val(in, b, s, c);
+      for (int32_t j = 0; j < in->heads; ++j) {
+        double z = 0.0;
+        for (int32_t c = 0; c < in->dim; ++c) z += q_val(in, row, j, c) * kd[c];
+        double wj = (double)in->w[row * in->heads + j];
+        dw[row * in->heads + j] += g * (MUT(46) ? z : (z > 0.0 ? z : 0.0));
+        if (!(MUT(44) ? z >= 0.0 : z > 0.0)) continue;
+        double coef = g * (MUT(45) ? 1.0 : wj);
+        for (int32_t c = 0; c < in->dim; ++c) {
+          dq[(row * in->heads + j) * in->dim + c] += coef * kd[c];
+          dk[((int64_t)b * in->n_k + s) * in->dim + c] += coef * q_val(in, row, j, c);
+        }
+      }
+    }
+  }
+  free(kd);
   return ORC_OK;
 }
 

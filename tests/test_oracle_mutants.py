@@ -57,6 +57,9 @@ MUTANTS = {
     40: "sparse attention logits without the softmax scale",
     41: "sparse attention value taken from the wrong end of the latent row",
     43: "sparse attention reads an empty (-1) entry as position 0",
+    44: "backward mask 1[z >= 0] instead of 1[z > 0]",
+    45: "backward drops the head weight from dq and dk",
+    46: "backward dw uses z instead of ReLU(z)",
 }
 
 

@@ -797,3 +797,70 @@ def test_sparse_mla_ignores_order_and_empty_entries(oracle_mod):
         np.testing.assert_allclose(a[key], b[key], rtol=1e-12, atol=1e-13)
     z = oracle_mod.sparse_mla(q, kv, np.full((5, 3), -1, np.int32), 0.125, 48, 5)
     assert np.all(z["o"] == 0.0) and np.all(np.isneginf(z["lse"])) and np.all(z["den"] == 0.0)
+
+
+# ---------------------------------------------------------- indexer backward --
+
+def _loss(oracle_mod, p, q, k, w, sel, g):
+    """L = sum_{t, s in S_t} g_{t,s} I_{t,s}, evaluated with the oracle's forward
+    score (fp32 operands)."""
+    pp = gen.Problem(p.batch, p.n_q, p.n_k, p.heads, p.dim, p.topk, F32, F32, q, k, w,
+                     p.q_pos0, p.k_len)
+    inp = oracle_mod.Inputs(pp)
+    rows = np.repeat(np.arange(p.batch * p.n_q), sel.shape[1])
+    s = sel.ravel()
+    ok = s >= 0
+    return float(np.sum(g.ravel()[ok] * oracle_mod.score_pairs(inp, rows[ok], s[ok])))
+
+
+def test_backward_matches_central_differences(oracle_mod):
+    """The three gradients of [PT] 2.3 against central differences of the
+    forward score (the definition the chain rule starts from), on inputs whose
+    dot products stay far from the ReLU kink."""
+    rng = np.random.default_rng(30)
+    B_, nq, nk, H, d, kk = 1, 3, 12, 3, 4, 5
+    q = rng.standard_normal((B_, nq, H, d))
+    k = rng.standard_normal((B_, nk, d))
+    w = rng.standard_normal((B_, nq, H))
+    z = np.einsum("bthd,bsd->bths", q, k)
+    q[np.abs(z).min(axis=(2, 3)) < 0.05] *= 1.1                 # keep |z| away from 0
+    q, k, w = (x.astype(np.float32).astype(np.float64) for x in (q, k, w))
+    p = gen.Problem(B_, nq, nk, H, d, kk, F32, F32, q.astype(np.float32), k.astype(np.float32),
+                    w.astype(np.float32))
+    sel = np.array([[0, 3, 7, -1, 9], [1, 2, -1, 4, 10], [11, 0, 5, 6, -1]], np.int32)
+    g = rng.standard_normal(sel.shape).astype(np.float32)
+    got = oracle_mod.indexer_backward(oracle_mod.Inputs(p), sel, g)
+    eps = 1e-3
+    for name, arr, grad in (("q", q, got["dq"].reshape(q.shape)), ("k", k, got["dk"].reshape(k.shape)),
+                            ("w", w, got["dw"].reshape(w.shape))):
+        flat = arr.reshape(-1)
+        num = np.empty_like(flat)
+        for i in range(flat.size):
+            old = flat[i]
+            flat[i] = old + eps
+            lp = _loss(oracle_mod, p, q.astype(np.float32), k.astype(np.float32),
+                       w.astype(np.float32), sel, g)
+            flat[i] = old - eps
+            lm = _loss(oracle_mod, p, q.astype(np.float32), k.astype(np.float32),
+                       w.astype(np.float32), sel, g)
+            flat[i] = old
+            num[i] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad.reshape(-1), num, rtol=1e-3, atol=1e-3, err_msg=name)
+
+
+def test_backward_relu_kink_has_zero_derivative(oracle_mod):
+    """z exactly 0 (integer operands): m = 1[z > 0] = 0, so no gradient flows to
+    q or k through that head, and its ReLU(z) = 0 adds nothing to dw."""
+    q = np.zeros((1, 1, 2, 4), np.float32)
+    q[0, 0, 0] = [1, -1, 0, 0]         # z = 0 against k = (1, 1, 0, 0)
+    q[0, 0, 1] = [1, 1, 0, 0]          # z = 2
+    k = np.zeros((1, 1, 4), np.float32)
+    k[0, 0] = [1, 1, 0, 0]
+    w = np.array([[[3.0, 5.0]]], np.float32)
+    p = make(q, k, w, topk=1)
+    out = oracle_mod.indexer_backward(oracle_mod.Inputs(p), np.array([[0]], np.int32),
+                                      np.array([[2.0]], np.float32))
+    assert np.all(out["dq"][0, 0] == 0.0)
+    assert np.array_equal(out["dq"][0, 1], 2.0 * 5.0 * k[0, 0])
+    assert np.array_equal(out["dk"][0, 0], 2.0 * 5.0 * q[0, 0, 1])
+    assert np.array_equal(out["dw"][0], [0.0, 2.0 * 2.0])
