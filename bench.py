@@ -448,6 +448,61 @@ def mla_line(steps, warmup, dev):
             "gpu_launches": steps}
 
 
+BWD_WORKLOAD = dict(
+    desc="Indexer backward with score recompute (sparse stage): L=8192 prefill rows, H_I=64, "
+         "d=128, 2048 selected causal positions per row, bf16 q,k ~N(0,1), upstream gradient "
+         "N(0,1); dq, dk, dw in fp32",
+    n_q=8192, heads=64, topk=2048, seed=7)
+
+
+def backward_line(steps, warmup, dev):
+    """Indexer backward timed with CUDA events; tensor roofline by its algorithmic
+    FLOPs: three products (recomputed z, dq, dk) of 2 * 64 * 128 per selected
+    (row, position)."""
+    import torch
+    from sparse_attention_token_dsa_b200 import binding as B
+    from sparse_attention_token_dsa_b200 import workloads
+    w = BWD_WORKLOAD
+    p, sel, grad = workloads.backward_problem(w["n_q"], w["heads"], w["topk"], seed=w["seed"])
+    q = torch.from_numpy(p.q.view(np.int16)).to(dev).view(torch.bfloat16)
+    k = torch.from_numpy(p.k.view(np.int16)).to(dev).view(torch.bfloat16)
+    wt = torch.from_numpy(p.w).to(dev)
+    sd = torch.from_numpy(sel).to(dev).view(1, w["n_q"], w["topk"])
+    gd = torch.from_numpy(grad).to(dev).view(1, w["n_q"], w["topk"])
+    dk = torch.zeros(k.shape, dtype=torch.float32, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def call():
+        B.indexer_backward(q, k, wt, sd, gd, dk=dk, workspace=ws, stream=stream)
+
+    for _ in range(max(warmup, 3)):
+        call()
+    st = B.dsa_read_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st}: {B.status_string(st)}")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    nsel = int((sel >= 0).sum())
+    flops = 3 * 2.0 * nsel * w["heads"] * 128
+    pk = peaks()
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"workload": w["desc"], "value": ms, "unit": "ms/layer", "ms_per_step": ms,
+            "steps": steps, "warmup": max(warmup, 3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": pk["bf16"],
+                         "unit": "TFLOP/s", "frac": tf / pk["bf16"],
+                         "peak_source": f"{pk['src']} bf16 burst",
+                         "work": f"{flops / 1e12:.3f} TFLOP per call",
+                         "kernel": "indexer_backward_kernel", "kernel_ms": ms, "traffic": None},
+            "gpu_launches": steps}
+
+
 # in an order that reuses generated problems: MISA and MISA-dagger share the
 # headline problem, stacked HISA shares HISA's clustered keys
 SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "lisa_prefill_128k",
@@ -920,6 +975,7 @@ def main():
             cache.clear()
             torch.cuda.empty_cache()
             line["secondary"].append(mla_line(min(args.steps, 5), args.warmup, dev))
+            line["secondary"].append(backward_line(min(args.steps, 5), args.warmup, dev))
             line["gpu_launches"] += sum(s["gpu_launches"] for s in line["secondary"])
             cache.clear()
         if not args.no_cpu_baseline:

@@ -310,6 +310,23 @@ int dsa_sparse_mla(const dsa_mla_problem* p, const void* q, const void* kv, cons
                    void* out, float* out_lse, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/* Indexer backward with score recompute ("PaperTrace 2.2.2", section 2.3 "why
+ * training gradients need recomputation"): for the loss L = sum_t sum_{s in S_t}
+ * g_{t,s} I_{t,s}, with z = q_{t,j} . k_s recomputed over each row's selected
+ * positions and m = 1[z > 0] (ReLU's derivative 0 at 0):
+ *   dq_{t,j} = sum_s g_{t,s} w_{t,j} m k_s        dq [batch, n_q, heads, dim] fp32, written
+ *   dk_s    += sum_t sum_j g_{t,s} w_{t,j} m q_{t,j}  dk [batch, n_k, dim] fp32, ADDED TO
+ *   dw_{t,j} = sum_s g_{t,s} ReLU(z)              dw [batch, n_q, heads] fp32, written
+ * sel / grad [batch, n_q, p->topk]: selected positions (-1 empty) and the
+ * upstream gradient on I at each.  q, k bf16 (dim 128), w fp32; heads == 64.
+ * The products g w m enter the dq / dk tensor-core products in bf16 (fp32
+ * accumulation); dw is exact up to fp32 sums.  dk receives one vector reduction
+ * per (row, selected position), so its summation order is not fixed.
+ * workspace >= 256 bytes (status word). */
+int dsa_indexer_backward(const dsa_problem* p, const void* q, const void* k, const float* w,
+                         const int32_t* sel, const float* grad, float* dq, float* dk, float* dw,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Operand preparation for the FP8 path: per-row scale a = amax/448 (amax == 0
  * gives a = 1), code = round-to-nearest-even, saturating e4m3 of x/a, both
  * divisions in IEEE fp32 ("PaperTrace 2.2.2", section 2.3 "from formula to

@@ -75,12 +75,13 @@ def _load():
     lib.resmisa_index.argtypes = [P, R, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
     lib.dsa_sparse_mla.argtypes = [C.POINTER(DsaMlaProblem), vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_indexer_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     for f in ("dsa_read_status", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
               "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
               "misa_dagger_index", "hisa_index", "lisa_index", "resmisa_index",
-              "dsa_quantize_e4m3", "dsa_sparse_mla"):
+              "dsa_quantize_e4m3", "dsa_sparse_mla", "dsa_indexer_backward"):
         getattr(lib, f).restype = C.c_int
     return lib
 
@@ -324,6 +325,23 @@ def sparse_mla(q, kv, idx, scale, tokens_per_seq=None, flags=0, out=None, out_ls
     _check(lib.dsa_sparse_mla(C.byref(p), _ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(out_lse),
                               _ptr(ws), ws.numel(), _stream(stream)), "dsa_sparse_mla")
     return out, out_lse
+
+
+def indexer_backward(q, k, w, sel, grad, dk=None, flags=0, workspace=None, stream=None):
+    """Gradients of sum g I over the selected positions: returns (dq [B, n_q, H, d],
+    dk [B, n_k, d], dw [B, n_q, H]) in fp32; dk is added to when given."""
+    _args(q=(q, (torch.bfloat16,)), k=(k, (torch.bfloat16,)), w=(w, _F32), sel=(sel, _I32),
+          grad=(grad, _F32), dk=(dk, _F32), workspace=(workspace, _U8))
+    p = problem(q, k, sel.shape[-1], flags=flags)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    dw = torch.empty(w.shape, dtype=torch.float32, device=q.device)
+    if dk is None:
+        dk = torch.zeros(k.shape, dtype=torch.float32, device=q.device)
+    ws = _workspace(256, q.device, workspace)
+    _check(lib.dsa_indexer_backward(C.byref(p), _ptr(q), _ptr(k), _ptr(w), _ptr(sel), _ptr(grad),
+                                    _ptr(dq), _ptr(dk), _ptr(dw), _ptr(ws), ws.numel(),
+                                    _stream(stream)), "dsa_indexer_backward")
+    return dq, dk, dw
 
 
 def dsa_quantize_e4m3(x: torch.Tensor, stream=None):

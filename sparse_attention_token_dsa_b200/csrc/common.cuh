@@ -122,6 +122,11 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
       "r"(r2), "r"(r3)
       : "memory");
 }
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy reads of them (an MMA operand written by threads).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

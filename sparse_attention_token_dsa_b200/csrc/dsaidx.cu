@@ -12,6 +12,7 @@
 
 #include "../../include/dsaidx.h"
 #include "common.cuh"
+#include "bwd.cuh"
 #include "finalize.cuh"
 #include "mla.cuh"
 #include "prep.cuh"
@@ -1441,6 +1442,47 @@ int dsa_sparse_mla(const dsa_mla_problem* p, const void* q, const void* kv, cons
       cudaSuccess)
     return DSA_ERR_CUDA;
   sparse_mla_kernel<<<(unsigned)(T * 2), kMlaThreads, smem, st>>>(qm, km, a);
+  if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
+  if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(workspace, stream);
+  return DSA_OK;
+}
+
+int dsa_indexer_backward(const dsa_problem* p, const void* q, const void* k, const float* w,
+                         const int32_t* sel, const float* grad, float* dq, float* dk, float* dw,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (!p || !q || !k || !w || !sel || !grad || !dq || !dk || !dw) return DSA_ERR_INVALID;
+  if (p->batch < 1 || p->n_q < 1 || p->n_k < 1 || p->topk < 1) return DSA_ERR_INVALID;
+  if (p->dim != 128 || p->heads != kBwdH || p->q_dtype != DSA_BF16 || p->k_dtype != DSA_BF16)
+    return DSA_ERR_UNSUPPORTED;
+  const long long rows = (long long)p->batch * p->n_q;
+  if (rows > 0x7fffffffll || rows * kBwdH > (1ll << 31) ||
+      (long long)p->batch * p->n_k > (1ll << 31) || p->topk > (1 << 20))
+    return DSA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(dq) || !aligned16(dk)) return DSA_ERR_INVALID;
+  if (!workspace || workspace_bytes < kWsHeaderBytes) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(workspace, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+  CUtensorMap qm, km;
+  if (!make_map(&qm, q, 2, (uint64_t)rows * kBwdH, kBwdH)) return DSA_ERR_CUDA;
+  if (!make_map(&km, k, 2, (uint64_t)p->batch * p->n_k, 1)) return DSA_ERR_CUDA;
+  BwdArgs a{};
+  a.rows = (int32_t)rows;
+  a.n_q = p->n_q;
+  a.n_k = p->n_k;
+  a.topk = p->topk;
+  a.sel = sel;
+  a.grad = grad;
+  a.w = w;
+  a.dq = dq;
+  a.dk = dk;
+  a.dw = dw;
+  a.status = reinterpret_cast<int32_t*>(workspace);
+  const int smem = (int)bwd_smem_bytes();
+  if (cudaFuncSetAttribute(indexer_backward_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           smem) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  indexer_backward_kernel<<<(unsigned)rows, kBwdThreads, smem, st>>>(qm, km, a);
   if (cudaGetLastError() != cudaSuccess) return DSA_ERR_CUDA;
   if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(workspace, stream);
   return DSA_OK;

@@ -38,3 +38,21 @@ def mla_problem(n_q: int, n_k: int, heads: int, topk: int, seed: int = 1, batch:
             sel = np.sort(r.choice(pos + 1, size=topk, replace=False))
         idx[t, :len(sel)] = sel
     return dict(q=q, kv=kv, idx=idx, scale=SCALE, tps=n_q)
+
+
+def backward_problem(n_q: int, heads: int, topk: int, seed: int = 1):
+    """Indexer backward workload: one prefill sequence of n_q tokens (q, k bf16
+    N(0,1), w N(0, 1/heads)), each row's topk distinct causal positions in
+    ascending order (all of them when the prefix is shorter), upstream
+    gradient N(0,1).  Returns (problem, sel, grad)."""
+    p = gen.normal_problem(seed, 1, n_q, n_q, heads, 128, topk)
+    r = np.random.Generator(np.random.PCG64(1000 * seed + 5))
+    sel = np.full((n_q, topk), -1, np.int32)
+    for t in range(n_q):
+        if t + 1 <= topk:
+            pick = np.arange(t + 1)
+        else:
+            pick = np.sort(r.choice(t + 1, size=topk, replace=False))
+        sel[t, :len(pick)] = pick
+    grad = r.standard_normal(sel.shape, dtype=np.float32)
+    return p, sel, grad
