@@ -118,6 +118,24 @@ WORKLOADS = {
         desc="ResMiSA prefill, batch 1, L=131072 causal, H_I=64, d=128, shared linear term + "
              "r=7 residual heads routed by block bounds (B=1024), top-k=2048, bf16 q,k ~N(0,1)",
         kind="resmisa", batch=1, L=_L128, H=64, topk=2048, seed=4, block=1024, r=7),
+    "dosa_prefill_128k": dict(
+        desc="DoSA (exact bound pruning) over the DSA prefill scan, batch 1, L=131072 causal, "
+             "H_I=64, d=128, top-k=2048, 1024-token bound blocks, bf16 q,k ~N(0,1), "
+             "w ~N(0,1/64) (the headline problem: independent keys, loose bounds)",
+        kind="prefill", batch=1, L=_L128, H=64, topk=2048, fp8=False, seed=4, needles=0,
+        dosa=True),
+    "dsa_locality_prefill_128k": dict(
+        desc="DSA indexer prefill, batch 1, L=131072 causal, H_I=64, d=128, top-k=2048, bf16, "
+             "keys with locality: 64 Gaussian centres in contiguous runs (mean 8192 tokens) "
+             "+ 0.01 N(0,1) noise",
+        kind="prefill", batch=1, L=_L128, H=64, topk=2048, fp8=False, seed=7, needles=0,
+        keys="locality"),
+    "dosa_locality_prefill_128k": dict(
+        desc="DoSA (exact bound pruning) over the DSA prefill scan, batch 1, L=131072 causal, "
+             "H_I=64, d=128, top-k=2048, 1024-token bound blocks, keys with locality (64 "
+             "centres in runs of mean 8192 tokens + 0.01 noise)",
+        kind="prefill", batch=1, L=_L128, H=64, topk=2048, fp8=False, seed=7, needles=0,
+        keys="locality", dosa=True),
     "hisa_misa_prefill_128k": dict(
         desc="Stacked MISA (B=1024, h=8) + HISA (b=64, r=128) prefill, batch 1, L=131072 "
              "causal, H_I=64, d=128, top-k=2048, bf16, clustered keys",
@@ -173,9 +191,18 @@ def make_problem(w):
     if w["kind"] == "decode":
         p, _ = gen.decode_problem(w["seed"], w["batch"], w["L"], w["H"], 128, w["topk"])
         return p
+    if w.get("keys") == "locality":
+        return gen.normal_problem(w["seed"], w["batch"], w["L"], w["L"], w["H"], 128, w["topk"],
+                                  key_structure="clusters", n_centres=64, mean_run=8192.0,
+                                  noise=0.01)
     return gen.normal_problem(w["seed"], w["batch"], w["L"], w["L"], w["H"], 128, w["topk"],
                               n_needles=w.get("needles", 0),
                               key_structure=w.get("keys", "iid"))
+
+
+def tile_pairs(p):
+    """(query row, 128-key tile) pairs of the legal prefixes: what DoSA may skip."""
+    return int(((legal_counts(p) + 127) // 128).sum())
 
 
 def legal_counts(p):
@@ -503,11 +530,13 @@ def backward_line(steps, warmup, dev):
             "gpu_launches": steps}
 
 
-# in an order that reuses generated problems: MISA and MISA-dagger share the
-# headline problem, stacked HISA shares HISA's clustered keys
-SECONDARY = ["misa_prefill_128k", "misa_dagger_prefill_128k", "lisa_prefill_128k",
-             "lisa_dagger_prefill_128k", "resmisa_prefill_128k", "hisa_prefill_128k",
-             "hisa_misa_prefill_128k", "dsa_decode_128k"]
+# in an order that reuses generated problems: DoSA, MISA and MISA-dagger share
+# the headline problem, stacked HISA shares HISA's clustered keys, DoSA on keys
+# with locality follows the unpruned scan of the same problem
+SECONDARY = ["dosa_prefill_128k", "misa_prefill_128k", "misa_dagger_prefill_128k",
+             "lisa_prefill_128k", "lisa_dagger_prefill_128k", "resmisa_prefill_128k",
+             "hisa_prefill_128k", "hisa_misa_prefill_128k", "dsa_locality_prefill_128k",
+             "dosa_locality_prefill_128k", "dsa_decode_128k"]
 
 
 def max_over_ranks(x: float, device=None) -> float:
@@ -588,7 +617,8 @@ class Case:
         for key in ("q", "w", "q_scale", "idx", "sc"):
             if c[key] is not None and not c[key].is_contiguous():
                 raise ValueError("partitioned rows must be contiguous (batch 1 prefill)")
-        c["prob"] = B.problem(c["q"], c["k"], p.topk, pos0, klen)
+        c["prob"] = B.problem(c["q"], c["k"], p.topk, pos0, klen,
+                              B.DSA_FLAG_DOSA if w.get("dosa") else 0)
         if self.kind in ROUTED:
             algo = {"misa": B.DSA_ALGO_MISA, "dagger": B.DSA_ALGO_MISA_DAGGER,
                     "hisa": B.DSA_ALGO_HISA, "lisa": B.DSA_ALGO_LISA,
@@ -619,6 +649,8 @@ class Case:
         else:
             c["ws_bytes"] = B.dsa_workspace_size(c["prob"])
             c["launches"] = 2 + (1 if (self.fp8 and self.kind == "decode") else 0)
+            if w.get("dosa"):
+                c["launches"] += 2                   # key ranges + bounds
         return c
 
     def _routed(self, c, q, k, w_, out):
@@ -704,7 +736,8 @@ class Case:
                         q2, qs_ = B.dsa_quantize_e4m3(qq.reshape(n, -1))
                         qq, qs_ = q2.reshape(b["dq"].shape), qs_.reshape(qq.shape[0], qq.shape[1])
                 B.dsa_index(qq, kk, b["dw"], p.topk, q_scale=qs_, k_scale=ks_, q_pos0=c["pos0"],
-                            k_len=c["klen"], out=out, workspace=self.ws, stream=self.stream)
+                            k_len=c["klen"], flags=c["prob"].flags, out=out, workspace=self.ws,
+                            stream=self.stream)
             b["hi"].copy_(c["idx"], non_blocking=True)
             b["hs"].copy_(c["sc"], non_blocking=True)
 
@@ -853,11 +886,20 @@ def quality(case, name, ms_per_step, dense=None):
         for b, t, s_ in zip(p.needles["b"], p.needles["t"], p.needles["s"]):
             found += int((gi[b * p.n_q + t] == s_).any().item())
         out["needle_recall"] = found / len(p.needles["s"])
-    if case.kind in ROUTED:
+    if case.kind in ROUTED or case.w.get("dosa"):
         didx, dense_ms = dense if dense is not None else dense_reference(case)
         rows = torch.linspace(p.n_q // 16, p.n_q - 1, 512).long().to(case.dev)
         out.update({"iou_vs_dsa": iou_rows(case.idx, didx, rows), "dsa_ms": dense_ms,
                     "speedup_vs_dsa": dense_ms / ms_per_step})
+    if case.w.get("dosa"):
+        # exactness at full size: every row's set equals the unpruned scan's
+        a_ = case.idx.reshape(-1, p.topk).sort(dim=1).values
+        b_ = didx.reshape(-1, p.topk).sort(dim=1).values
+        out["identical_to_dsa"] = bool(torch.equal(a_, b_))
+        del a_, b_
+        pruned = case.B.dsa_read_pruned(case.ws)
+        out["dosa_pruned_pairs"] = pruned
+        out["dosa_pruned_frac"] = pruned / tile_pairs(p)
     return out
 
 
@@ -876,10 +918,12 @@ def secondary_line(name, steps, warmup, dev, cache):
     unit, scale = unit_of(w)
     roof, dots = roofline(case, name, ms, kms, ms * steps > 1000.0)
     dense = cache.get(("dense",) + key)
-    if case.kind in ROUTED and dense is None:
+    if (case.kind in ROUTED or w.get("dosa")) and dense is None:
         dense = dense_reference(case)
         cache[("dense",) + key] = dense
     q = quality(case, name, ms, dense)
+    if case.kind == "prefill" and not case.fp8 and not w.get("dosa"):
+        cache[("dense",) + key] = (case.idx.clone(), ms)   # exact DSA of this problem
     line = {"workload": w["desc"], "value": ms * scale, "unit": unit, "ms_per_step": ms,
             "steps": steps, "warmup": max(warmup, 3), "roofline": roof,
             "scored_dots_per_s": dots / (ms * 1e-3), "gpu_launches": steps * case.launches}

@@ -112,6 +112,17 @@ enum {
  * ("PaperTrace 2.2.2", section 2.2: re-sorting score-ordered indices by
  * position makes the gather more contiguous).  Not with DSA_FLAG_SORTED. */
 #define DSA_FLAG_BY_POSITION 4u
+/* DoSA bound pruning ("The new bottleneck of sparse attention", route five:
+ * DoSA, exact pruning by upper and lower bounds).  dsa_index / dsa_index_scan
+ * first compute, for every query row and every 1024-token key block, an upper
+ * bound of I over the block's keys from the block's per-dimension key range;
+ * the scan then skips the head sums of a (row, 128-key tile) pair whose bound
+ * lies below the row's running threshold (a lower bound of its final k-th best
+ * key).  The selected set and scores are bit-identical to the call without the
+ * flag; only the work differs.  bf16 q and k, heads >= 32; otherwise
+ * DSA_ERR_UNSUPPORTED.  Needs the larger workspace dsa_workspace_size reports
+ * for the flagged problem.  dsa_read_pruned returns the count of skipped pairs. */
+#define DSA_FLAG_DOSA 8u
 /* For tests of the timeout path only, never in production: dsa_index /
  * dsa_index_scan run with a wait budget of about 1 ms instead of about 4 s, and
  * the scan's first CTA withholds one stage of keys, so its bounded waits run
@@ -338,6 +349,12 @@ int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
 /* Device status word recorded in `workspace` by the last call that used it
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_NONFINITE).  Synchronises `stream`. */
 int dsa_read_status(const void* workspace, void* stream);
+
+/* DoSA pruning count recorded in `workspace` by the last dsa_index /
+ * dsa_index_scan call with DSA_FLAG_DOSA: (query row, 128-key tile) pairs whose
+ * head sums were skipped (0 without the flag).  Synchronises `stream`; the
+ * count is written to *pruned.  DSA_ERR_INVALID for a null argument. */
+int dsa_read_pruned(const void* workspace, void* stream, unsigned long long* pruned);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 const char* dsa_status_string(int32_t status);

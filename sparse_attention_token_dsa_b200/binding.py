@@ -23,6 +23,7 @@ DSA_ALGO_LISA, DSA_ALGO_RESMISA = 4, 5
 DSA_FLAG_CHECK = 1
 DSA_FLAG_SORTED = 2
 DSA_FLAG_BY_POSITION = 4
+DSA_FLAG_DOSA = 8                    # exact bound pruning of the dense scan
 DSA_FLAG_TEST_STALL = 0x80000000   # tests of the timeout path only (see include/dsaidx.h)
 
 
@@ -62,6 +63,7 @@ def _load():
     lib.dsa_status_string.restype = C.c_char_p
     lib.dsa_status_string.argtypes = [i32]
     lib.dsa_read_status.argtypes = [vp, vp]
+    lib.dsa_read_pruned.argtypes = [vp, vp, C.POINTER(C.c_ulonglong)]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_route_chunk_rows.argtypes = [P, i32, R, C.POINTER(i32)]
@@ -76,7 +78,7 @@ def _load():
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
     lib.dsa_sparse_mla.argtypes = [C.POINTER(DsaMlaProblem), vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_indexer_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-    for f in ("dsa_read_status", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
+    for f in ("dsa_read_status", "dsa_read_pruned", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
               "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
@@ -359,3 +361,11 @@ def dsa_quantize_e4m3(x: torch.Tensor, stream=None):
 def dsa_read_status(workspace: torch.Tensor, stream=None) -> int:
     _args(workspace=(workspace, _U8))
     return lib.dsa_read_status(_ptr(workspace), _stream(stream))
+
+
+def dsa_read_pruned(workspace: torch.Tensor, stream=None) -> int:
+    """(query row, key tile) pairs the last DSA_FLAG_DOSA call on `workspace` skipped."""
+    _args(workspace=(workspace, _U8))
+    n = C.c_ulonglong(0)
+    _check(lib.dsa_read_pruned(_ptr(workspace), _stream(stream), C.byref(n)), "dsa_read_pruned")
+    return int(n.value)

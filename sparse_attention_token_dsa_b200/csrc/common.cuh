@@ -17,8 +17,10 @@ namespace dsa {
 struct WsHeader {
   int32_t status;     // DSA_OK or a negative device status (first error wins)
   int32_t where;      // which wait gave up (diagnostic)
-  int32_t pad[62];
+  unsigned long long pruned;  // DoSA: (query row, key tile) pairs skipped
+  int32_t pad[60];
 };
+static_assert(sizeof(WsHeader) == 256, "header size");
 constexpr size_t kWsHeaderBytes = 256;
 
 __device__ __forceinline__ void set_status(int32_t* st, int32_t code, int32_t where) {
@@ -109,6 +111,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
 // Four arbitrary rows (one-row-high box) into consecutive 128-byte smem rows.

@@ -6,13 +6,17 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stddef.h>
 #include <string.h>
+
+#include <algorithm>
 
 #include <mutex>
 
 #include "../../include/dsaidx.h"
 #include "common.cuh"
 #include "bwd.cuh"
+#include "dosa.cuh"
 #include "finalize.cuh"
 #include "mla.cuh"
 #include "prep.cuh"
@@ -233,6 +237,21 @@ bool make_map_q3d(CUtensorMap* m, const void* base, uint64_t tokens, uint64_t he
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over the DoSA block ranges [batch * 2][nblk][256] bf16: box of 64
+// dimensions x 32 blocks x one (sequence, hi / lo) plane, 128-byte swizzle;
+// blocks past nblk read as zeros.
+bool make_map_ranges(CUtensorMap* m, const void* base, uint64_t nblk, uint64_t batch) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {256, (cuuint64_t)nblk, (cuuint64_t)batch * 2};
+  cuuint64_t strides[2] = {256 * 2, (cuuint64_t)nblk * 256 * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)kDosaBT, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D map over the cached latent rows [rows][576] bf16 for four-row gathers:
 // a one-row-high box of 64 dimensions.
 bool make_map_kv(CUtensorMap* m, const void* base, uint64_t rows) {
@@ -247,10 +266,10 @@ bool make_map_kv(CUtensorMap* m, const void* base, uint64_t rows) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <MmaKind K, bool S, int HT, int GATHER = 0>
+template <MmaKind K, bool S, int HT, int GATHER = 0, bool DOSA = false>
 cudaError_t launch_scan_t(const ScanPlan& pl, const CUtensorMap& qm, const CUtensorMap& km,
                           const ScanArgs& a, cudaStream_t st) {
-  auto kern = scan_kernel<K, S, HT, GATHER>;
+  auto kern = scan_kernel<K, S, HT, GATHER, DOSA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)pl.smem);
   if (e != cudaSuccess) return e;
@@ -292,6 +311,13 @@ cudaError_t launch_scan(const ScanPlan& pl, const CUtensorMap& qm, const CUtenso
                         const ScanArgs& a, cudaStream_t st, int gather = 0) {
   if (gather == 1) return launch_scan_gather<1>(pl, qm, km, a, st);
   if (gather == 2) return launch_scan_gather<2>(pl, qm, km, a, st);
+  if (a.dosa_ub != nullptr) {  // bound pruning: bf16 operands, heads >= 32 (validated)
+    switch (a.H) {
+      case 32: return launch_scan_t<MmaKind::BF16, false, 32, 0, true>(pl, qm, km, a, st);
+      case 64: return launch_scan_t<MmaKind::BF16, false, 64, 0, true>(pl, qm, km, a, st);
+      default: return launch_scan_t<MmaKind::BF16, false, 128, 0, true>(pl, qm, km, a, st);
+    }
+  }
   switch (pl.kind) {
     case MmaKind::TF32: return launch_scan_h<MmaKind::TF32, false>(pl, qm, km, a, st);
     case MmaKind::BF16: return launch_scan_h<MmaKind::BF16, false>(pl, qm, km, a, st);
@@ -408,6 +434,8 @@ int validate_problem(const dsa_problem* p) {
   if (!same && !split) return DSA_ERR_UNSUPPORTED;
   if (split && p->heads < 32) return DSA_ERR_UNSUPPORTED;
   if ((p->flags & DSA_FLAG_SORTED) && (p->flags & DSA_FLAG_BY_POSITION)) return DSA_ERR_INVALID;
+  if ((p->flags & DSA_FLAG_DOSA) && !(qd == DSA_BF16 && kd == DSA_BF16 && p->heads >= 32))
+    return DSA_ERR_UNSUPPORTED;
   return DSA_OK;
 }
 
@@ -430,9 +458,15 @@ void kind_of(const dsa_problem* p, MmaKind* kind, bool* split) {
     *kind = MmaKind::TF32;
 }
 
+// DoSA bound blocks: 2^kDosaShift tokens (a whole number of 128-key tiles).
+constexpr int kDosaShift = 10;
+
 struct DsaLayout {
   ScanPlan pl;
-  size_t off_logs, off_cnt, off_thr, off_parts, off_hscale, total;
+  size_t off_logs, off_cnt, off_thr, off_parts, off_hscale;
+  size_t off_ranges, off_mx, off_ub;  // DoSA (DSA_FLAG_DOSA) only
+  int dosa_nblk;
+  size_t total;
 };
 
 DsaLayout dsa_layout(const dsa_problem* p) {
@@ -453,6 +487,16 @@ DsaLayout dsa_layout(const dsa_problem* p) {
   if (split) off += align_up((size_t)L.pl.rows * 2 * p->heads * p->dim);
   L.off_hscale = off;
   if (split) off += align_up((size_t)L.pl.rows * p->heads * sizeof(float));
+  L.off_ranges = L.off_mx = L.off_ub = off;
+  L.dosa_nblk = 0;
+  if (p->flags & DSA_FLAG_DOSA) {
+    L.dosa_nblk = (p->n_k + (1 << kDosaShift) - 1) >> kDosaShift;
+    off += align_up((size_t)p->batch * 2 * L.dosa_nblk * 256 * 2);
+    L.off_mx = off;
+    off += align_up((size_t)p->batch * L.dosa_nblk * sizeof(float));
+    L.off_ub = off;
+    off += align_up((size_t)p->batch * p->n_q * L.dosa_nblk * sizeof(float));
+  }
   L.total = off;
   return L;
 }
@@ -533,6 +577,7 @@ int route_cfg(const dsa_problem* p, int algo, const dsa_route_params* rp, RouteC
     return DSA_ERR_INVALID;
   if (p->q_dtype != DSA_BF16 || p->k_dtype != DSA_BF16) return DSA_ERR_UNSUPPORTED;
   if (p->batch > 65535) return DSA_ERR_UNSUPPORTED;
+  if (p->flags & DSA_FLAG_DOSA) return DSA_ERR_UNSUPPORTED;  // bounds of the dense scan only
   *c = RouteCfg{};
   c->algo = algo;
   if (algo == DSA_ALGO_LISA || algo == DSA_ALGO_RESMISA) {
@@ -978,6 +1023,16 @@ int dsa_read_status(const void* workspace, void* stream) {
   return s;
 }
 
+int dsa_read_pruned(const void* workspace, void* stream, unsigned long long* pruned) {
+  if (!workspace || !pruned) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+  if (cudaMemcpy(pruned, reinterpret_cast<const uint8_t*>(workspace) + offsetof(WsHeader, pruned),
+                 sizeof(*pruned), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  return DSA_OK;
+}
+
 int dsa_workspace_size(const dsa_problem* p, int32_t algo, const dsa_route_params* rp,
                        size_t* bytes) {
   if (!bytes) return DSA_ERR_INVALID;
@@ -1088,6 +1143,40 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   const bool stall = (p->flags & DSA_FLAG_TEST_STALL) != 0;
   a.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
   a.test_stall = stall ? 1 : 0;
+  if (p->flags & DSA_FLAG_DOSA) {
+    // per-block key ranges, then per-(row, block) upper bounds of I
+    uint16_t* E = reinterpret_cast<uint16_t*>(ws + L.off_ranges);
+    float* mx = reinterpret_cast<float*>(ws + L.off_mx);
+    float* ub = reinterpret_cast<float*>(ws + L.off_ub);
+    dosa_ranges_kernel<<<dim3((unsigned)L.dosa_nblk, (unsigned)p->batch), 128, 0, st>>>(
+        reinterpret_cast<const uint16_t*>(k), p->n_k, kDosaShift, L.dosa_nblk, E, mx);
+    CUtensorMap qbm, em;
+    if (!make_map(&qbm, q, 2, (uint64_t)p->batch * p->n_q * p->heads, 128)) return DSA_ERR_CUDA;
+    if (!make_map_ranges(&em, E, (uint64_t)L.dosa_nblk, (uint64_t)p->batch)) return DSA_ERR_CUDA;
+    DosaArgs da{};
+    da.batch = p->batch;
+    da.n_q = p->n_q;
+    da.n_tok = p->n_k;
+    da.H = p->heads;
+    da.shift = kDosaShift;
+    da.nblk = L.dosa_nblk;
+    da.q_pos0 = p->q_pos0;
+    da.k_len = p->k_len;
+    da.w = w;
+    da.mx = mx;
+    da.ub = ub;
+    da.status = status;
+    if (cudaFuncSetAttribute(dosa_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)dosa_smem_bytes()) != cudaSuccess)
+      return DSA_ERR_CUDA;
+    const int rpc = 128 / p->heads;
+    const int64_t nct = (int64_t)p->batch * ((p->n_q + rpc - 1) / rpc);
+    dosa_bound_kernel<<<(unsigned)nct, kDosaThreads, dosa_smem_bytes(), st>>>(qbm, em, da);
+    a.dosa_ub = ub;
+    a.dosa_nblk = L.dosa_nblk;
+    a.dosa_shift = kDosaShift;
+    a.dosa_pruned = reinterpret_cast<unsigned long long*>(ws + offsetof(WsHeader, pruned));
+  }
   if (launch_scan(pl, qm, km, a, st) != cudaSuccess) return DSA_ERR_CUDA;
   return DSA_OK;
 }

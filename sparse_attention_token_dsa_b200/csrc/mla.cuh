@@ -62,14 +62,6 @@ constexpr size_t mla_smem_bytes() {
          sizeof(MlaSmemTail);
 }
 
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                            int32_t x, int32_t y, int32_t z) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
 
 // Shared-memory descriptor of an MN-major operand in 128-byte swizzled rows:
 // each 128-byte row holds 64 consecutive MN elements of one K index, 8 rows form

@@ -84,6 +84,10 @@ struct ScanArgs {
   unsigned long long* log_thr;  // [rows * C] final threshold of the slot
   int32_t* status;       // workspace status word
   long long wait_cycles; // budget of every bounded wait (kWaitCycles; shorter in tests)
+  const float* dosa_ub;  // DoSA: per (row, block) upper bounds of I [rows, dosa_nblk], or null
+  int32_t dosa_nblk;     //   bound blocks per row
+  int32_t dosa_shift;    //   log2 tokens per bound block (>= 7: a key tile lies in one block)
+  unsigned long long* dosa_pruned;  // (row, unit) pairs skipped, or null
   int32_t test_stall;    // DSA_FLAG_TEST_STALL: CTA 0 withholds the second K stage of
                          //   its first item, so the waits on it run out (tests only)
 };
@@ -135,6 +139,7 @@ struct ScanSmemTail {
   int32_t subcnt[kMaxRows][8]; // sub-log fill, written only by the owning warp
   unsigned long long row_thr[kMaxRows];
   int32_t item_min_nleg;       // smallest row_nleg of the item's rows
+  unsigned int dosa_skips;     // (row, unit) pairs this CTA skipped by their DoSA bound
   alignas(16) float wsm[kMaxItemCols];
   SelectScratch sel;
 };
@@ -485,7 +490,7 @@ __device__ __forceinline__ float row_acc(uint32_t taddr, const float* w) {
 
 // 320 threads: ten warps over four sub-partitions of 16K registers each allow
 // at most 168 registers per thread.
-template <MmaKind KIND, bool SPLIT, int HT, int GATHER>
+template <MmaKind KIND, bool SPLIT, int HT, int GATHER, bool DOSA = false>
 __global__ void __launch_bounds__(kScanThreads, 1)
     scan_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                 const ScanArgs a) {
@@ -531,6 +536,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       mbar_init(&T->t_empty[s], modeB ? 4 : 8);
     }
     T->abort = 0;
+    T->dosa_skips = 0u;
     fence_barrier_init();
   }
   if (warp == kMmaWarp) {
@@ -947,10 +953,15 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     uint32_t ucount = 0;
     int step_par = 0;
     bool stop = false;
+    uint32_t dosa_n = 0;                       // DoSA: (row, unit) pairs this warp skipped
     for (int round = 0; !stop; ++round) {
       const int item = sched_item(round, blockIdx.x, grid);
       if (item >= a.n_items) break;
       ItemGeom g = item_geom<GATHER>(a, item);
+      // DoSA: per query group, the bound block of the cached skip decision
+      // (decided once per block, on entering it, with the thresholds of then)
+      int dblk0 = -1, dblk1 = -1;
+      unsigned dmask0 = 0u, dmask1 = 0u;
       const int pos0 = (a.q_pos0 ? a.q_pos0[g.b] : a.n_tok - a.q_stride) + a.q_off;
       const int klen = a.k_len ? a.k_len[g.b] : a.n_tok;
       const int64_t slot0 = ((int64_t)g.b * a.n_q + g.row0) * a.C + g.c;  // slot of row 0
@@ -1028,6 +1039,26 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             ks1 = ks_next1;
             if (KT > 1 && uu + ustep < nunits) ks_next1 = ks_at1(uu + ustep);
           }
+          // DoSA bounds of this warp's rows over the tile's bound block (rows past
+          // the item and rows of an unbounded problem: +inf, never skipped)
+          // DoSA: on entering a bound block, this warp's rows' bounds over it
+          // (loaded before the wait; rows past the item: +inf, never skipped)
+          float ubv[4];
+          bool dfresh = false;
+          int dblk = 0;
+          if constexpr (DOSA) {   // heads >= 32: at most four rows per warp
+            dblk = ((g.t_hi - t * KT) << 7) >> a.dosa_shift;
+            dfresh = dblk != (gg ? dblk1 : dblk0);
+            if (dfresh) {
+              const int rb = gg * a.QG + (modeB ? 0 : half * qhalf);
+              const int64_t gr = (int64_t)g.b * a.q_stride + a.q_off + g.row0 + rb;
+#pragma unroll
+              for (int qi = 0; qi < 4; ++qi)
+                ubv[qi] = qi < qhalf && rb + qi < g.nrows
+                              ? __ldg(a.dosa_ub + (gr + qi) * a.dosa_nblk + dblk)
+                              : __int_as_float(0x7f800000);
+            }
+          }
           const bool got = mbar_wait(&T->t_full[s], (uc / NS) & 1, abort, a.status, 6, a.wait_cycles);
           __syncwarp();
           if (!__all_sync(0xffffffffu, got)) continue;
@@ -1051,7 +1082,37 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           fc.T = T;
           fc.capw = a.capw;
           fc.status = a.status;
-          if constexpr (HT >= 32) {
+          if constexpr (DOSA) {
+            // DoSA: a row whose upper bound over the tile's block lies below its
+            // threshold (a lower bound of its final keep-th best) has no candidate
+            // the filter could keep in the block; its head sums are skipped.  A
+            // threshold raised inside the block only prunes from the next one.
+            if (dfresh) {
+              unsigned m = 0u;
+#pragma unroll
+              for (int qi = 0; qi < 4; ++qi) {
+                if (qi >= qhalf) break;
+                const unsigned long long th = T->row_thr[rbase + qi];
+                if (th != 0ull && ubv[qi] < key_score((uint32_t)(th >> 32))) m |= 1u << qi;
+              }
+              if (gg) { dblk1 = dblk; dmask1 = m; } else { dblk0 = dblk; dmask0 = m; }
+            }
+            const unsigned skipm = gg ? dmask1 : dmask0;
+            if (skipm == 0u) {
+              if (qhalf == 2)
+                unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+              else if (qhalf == 1)
+                unit_heads_n<HT, 1>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
+              else
+                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
+            } else {
+              dosa_n += __popc(skipm);
+              for (int qi = 0; qi < qhalf; ++qi)
+                if (!((skipm >> qi) & 1u))
+                  unit_heads_n<HT, 1>(fc, taddr + (qbeg + qi) * HT, &T->wsm[(rbase + qi) * HT],
+                                      rbase + qi);
+            }
+          } else if constexpr (HT >= 32) {
             if (qhalf == 2)
               unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
             else if (qhalf == 1)
@@ -1218,9 +1279,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       stop = stop || T->epi_stop[step_par] != 0;
       step_par ^= 1;
     }
+    if constexpr (DOSA) {
+      // each (row, unit) is counted by the quadrant-0 warp of its half
+      if (lane == 0 && quad == 0 && dosa_n) atomicAdd(&T->dosa_skips, dosa_n);
+    }
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (DOSA) {
+    if (threadIdx.x == 0 && a.dosa_pruned && T->dosa_skips)
+      atomicAdd(a.dosa_pruned, (unsigned long long)T->dosa_skips);
+  }
   if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();

@@ -89,7 +89,8 @@ def integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, d
 
 
 def segment_integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int,
-                            dim: int, topk: int, seg: int, q_pos0=None, k_len=None) -> Problem:
+                            dim: int, topk: int, seg: int, q_pos0=None, k_len=None,
+                            tail: bool = True) -> Problem:
     """Integer problem whose keys are constant on aligned segments of `seg` tokens.
 
     q uniform integers in [-3, 3], w in [-2, 2]; every key of segment i equals
@@ -99,6 +100,7 @@ def segment_integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads
     either c_i or c_i + e_i / (block size): a dyadic number with a small
     numerator, so pooled keys, their dot products with q and the sums over
     heads and blocks stay exactly representable in fp32 at the test sizes.
+    tail=False leaves out the e_i (keys exactly constant on each segment).
     """
     q = _rng(workload, 1).integers(-3, 4, size=(batch, n_q, heads, dim)).astype(np.float32)
     r = _rng(workload, 2)
@@ -106,8 +108,9 @@ def segment_integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads
     c = r.integers(-2, 3, size=(batch, nseg, dim)).astype(np.float32)
     e = r.integers(-1, 2, size=(batch, nseg, dim)).astype(np.float32)
     k = np.repeat(c, seg, axis=1)[:, :n_k].copy()
-    last = np.arange(seg - 1, n_k, seg)
-    k[:, last] += e[:, : len(last)]
+    if tail:
+        last = np.arange(seg - 1, n_k, seg)
+        k[:, last] += e[:, : len(last)]
     w = _rng(workload, 3).integers(-2, 3, size=(batch, n_q, heads)).astype(np.float32)
     return Problem(batch, n_q, n_k, heads, dim, topk, BF16, BF16, f32_to_bf16_bits(q),
                    f32_to_bf16_bits(k), w,
@@ -118,14 +121,14 @@ def segment_integer_problem(workload: int, batch: int, n_q: int, n_k: int, heads
 def normal_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, dim: int,
                    topk: int, q_pos0=None, k_len=None, n_needles: int = 0,
                    key_structure: str = "iid", n_centres: int = 256,
-                   mean_run: float = 512.0) -> Problem:
+                   mean_run: float = 512.0, noise: float = 0.5) -> Problem:
     """q, k ~ N(0,1) rounded to bf16; w ~ N(0, 1/H) fp32.
 
     key_structure
       "iid"      independent N(0,1) keys;
       "clusters" keys drawn from `n_centres` Gaussian centres assigned to
                  contiguous runs of geometric length (mean `mean_run`), plus
-                 0.5 N(0,1) noise, rescaled to unit variance — important tokens
+                 `noise` N(0,1), rescaled to unit variance — important tokens
                  gathered in contiguous regions, the structure HISA's block
                  filter relies on ("The new bottleneck of sparse attention",
                  route one: HISA, observation).
@@ -140,7 +143,7 @@ def normal_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, di
         r = _rng(workload, 4)
         centres = r.standard_normal(size=(batch, n_centres, dim), dtype=np.float32)
         k32 = np.empty((batch, n_k, dim), np.float32)
-        noise = _normal(_rng(workload, 2), (batch, n_k, dim), 0.5)
+        eps = _normal(_rng(workload, 2), (batch, n_k, dim), noise)
         for b in range(batch):
             pos = 0
             while pos < n_k:
@@ -148,8 +151,8 @@ def normal_problem(workload: int, batch: int, n_q: int, n_k: int, heads: int, di
                 c = int(r.integers(0, n_centres))
                 k32[b, pos:pos + run] = centres[b, c]
                 pos += run
-        k32 += noise
-        k32 /= np.float32(np.sqrt(1.25))
+        k32 += eps
+        k32 /= np.float32(np.sqrt(1.0 + noise * noise))
     else:
         raise ValueError(key_structure)
     w = _normal(_rng(workload, 3), (batch, n_q, heads), 1.0 / np.sqrt(heads))

@@ -196,3 +196,35 @@ def test_binding_checks_tensors_before_any_call(bind):
         bind.dsa_quantize_e4m3(k)
     with pytest.raises(TypeError, match="workspace: dtype"):
         bind.dsa_read_status(torch.zeros(4, dtype=torch.int32))
+
+
+def _flagged(bind, flags, **kw):
+    p = _prob(bind, **kw)
+    p.flags = flags
+    return p
+
+
+def test_dosa_flag_validation_and_workspace(bind):
+    D = bind.DSA_FLAG_DOSA
+    # bf16 q and k with >= 32 heads only
+    for kw in (dict(heads=16), dict(q_dtype=2, k_dtype=2), dict(q_dtype=0, k_dtype=0)):
+        rc, _ = _ws(bind, _flagged(bind, D, **kw), 0, None)
+        assert rc == -2, kw
+    # routed algorithms take no DoSA bounds
+    rc, _ = _ws(bind, _flagged(bind, D, n_q=256, n_k=1024), 1,
+                bind.route_params(misa_block=128, misa_h=8))
+    assert rc == -2
+    # extra workspace: two range rows and a magnitude per block, bounds per (row, block)
+    for nq, nk in ((16, 64), (300, 5000), (4096, 4096)):
+        rc0, plain = _ws(bind, _prob(bind, n_q=nq, n_k=nk), 0, None)
+        rc1, dosa = _ws(bind, _flagged(bind, D, n_q=nq, n_k=nk), 0, None)
+        assert rc0 == 0 and rc1 == 0
+        nblk = (nk + 1023) // 1024
+        need = nblk * 2 * 512 + nblk * 4 + nq * nblk * 4
+        assert need <= dosa - plain <= need + 3 * 256, (nq, nk, dosa - plain)
+
+
+def test_read_pruned_rejects_null(bind):
+    n = C.c_ulonglong(0)
+    assert bind.lib.dsa_read_pruned(None, None, C.byref(n)) == -1
+    assert bind.lib.dsa_read_pruned(C.c_void_p(0x1000), None, None) == -1
