@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(128)
 // ------------------------------------------------------------ bound GEMM --
 constexpr int kDosaThreads = 192;      // warps 0-3 epilogue, 4 TMA producer, 5 MMA issuer
 constexpr int kDosaBT = 32;            // bound blocks per B tile (N = 64: hi and lo rows)
-constexpr int kDosaKS = 2;             // B tile pipeline depth
+constexpr int kDosaKS = 1;             // B tile buffers (one: two CTAs fit an SM)
 
 struct DosaArgs {
   int32_t batch, n_q, n_tok, H;
@@ -98,14 +98,15 @@ struct DosaSmemTail {
 };
 
 // A [4 atoms][128 x 128 B] (q+ dims 0-63, 64-127, q- dims 0-63, 64-127),
-// B [KS][4 atoms][64 x 128 B] (32 hi rows, then 32 lo rows).
+// B [KS][4 atoms][64 x 128 B] (32 hi rows, then 32 lo rows): about 97 KB, so
+// two CTAs share an SM and one's loads overlap the other's epilogue.
 constexpr size_t dosa_smem_bytes() {
   return 1024 + 65536 + (size_t)kDosaKS * 32768 + sizeof(DosaSmemTail);
 }
 
 // CTA: 128 (row, head) pairs = 128 / H query rows of one sequence (TMEM lane =
 // pair); the B tiles cover the blocks up to the CTA's last legal key.
-__global__ void __launch_bounds__(kDosaThreads, 1)
+__global__ void __launch_bounds__(kDosaThreads, 2)
     dosa_bound_kernel(const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap emap, const DosaArgs a) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
