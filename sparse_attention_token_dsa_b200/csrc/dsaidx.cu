@@ -789,6 +789,7 @@ int run_stage(const dsa_problem* p, const ScanPlan& pl, const StageIO& io, int q
   a.bs_shift = io.bs_shift;
   a.klist = io.klist;
   a.klist_len = io.klist_len;
+  a.kraw = reinterpret_cast<const uint16_t*>(io.k);
   a.lb_shift = io.lb_shift;
   a.keep = pl.keep;
   a.QG = pl.QG;

@@ -57,6 +57,7 @@ struct ScanArgs {
                          //      a row sees block b iff (b + 1) << bs_shift <= min(pos + 1, k_len)
   const int32_t* klist;  // gathered keys: per-row lists [rows, klist_len] (-1 = empty slot)
   int32_t klist_len;
+  const uint16_t* kraw;  // token-list gathers: the key rows themselves [batch * n_k, 128] bf16
   int32_t lb_shift;      // block lists: log2 tokens per listed block
   int32_t keep;          // entries each row must keep (top-k or k')
   int32_t QG;            // query rows per accumulator group (<= 256 / (H * parts))
@@ -596,9 +597,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         // list entries outside [-1, n_k) (never written by this library's own
         // selects) are recorded and read as empty slots
         if constexpr (GATHER == 1) {
+          // lane L holds tile rows 2 (L % 16) + L / 16 + 32 j (j = 0..3): the rows
+          // that the copies below need from it, one register per copy round
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int e = t * 128 + lane * 4 + j;
+            const int e = t * 128 + 2 * (lane & 15) + (lane >> 4) + 32 * j;
             int kk = e < a.klist_len ? lst[e] : -1;
             if (kk < -1 || kk >= a.n_k) {
               set_status(a.status, DSA_ERR_INTERNAL, 111);
@@ -627,7 +630,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
         const bool stall = GATHER == 0 && a.test_stall && blockIdx.x == 0 && it == 1 && t == 1;
         if (lane == 0) {
           ok = mbar_wait(&T->k_empty[slot], ph ^ 1, abort, a.status, 2, a.wait_cycles);
-          if (ok && !stall) mbar_arrive_expect_tx(&T->k_full[slot], nvalid * Cfg::KTILE_BYTES);
+          if (ok && !stall && GATHER != 1)
+            mbar_arrive_expect_tx(&T->k_full[slot], nvalid * Cfg::KTILE_BYTES);
         }
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
@@ -645,10 +649,25 @@ __global__ void __launch_bounds__(kScanThreads, 1)
             }
           }
         } else if constexpr (GATHER == 1) {
-          // four arbitrary key rows per copy (one-row-high boxes), 32 copies per atom
-          for (int at = 0; at < Cfg::A; ++at)
-            tma_gather4(Ks + (slot * Cfg::A + at) * 16384 + lane * 4 * 128, &kmap,
-                        &T->k_full[slot], at * Cfg::EPA, rr[0], rr[1], rr[2], rr[3]);
+          // arbitrary key rows: 16-byte asynchronous copies, two whole 256-byte
+          // rows per warp instruction (lane = row parity x 16-byte chunk), into
+          // the 128-byte swizzled layout the MMA reads.  In round i lanes 0-15
+          // copy tile row 2i and lanes 16-31 row 2i + 1, whose entries lanes
+          // i % 16 and 16 + i % 16 hold in register i / 16.  The stage's barrier
+          // completes once every lane's copies have landed and lane 0 arrived.
+          static_assert(Cfg::A == 2, "bf16 key rows");
+          const int ch = lane & 15, at = ch >> 3, cc = ch & 7, odd = lane >> 4;
+          uint8_t* kb = Ks + (slot * Cfg::A + at) * 16384;
+          const uint8_t* kg = reinterpret_cast<const uint8_t*>(a.kraw) + ch * 16;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int v = __shfl_sync(0xffffffffu, rr[i >> 4], (i & 15) + 16 * odd);
+            const int r = 2 * i + odd;
+            cp_async_16(kb + r * 128 + ((cc ^ (r & 7)) << 4), kg + (size_t)v * 256);
+          }
+          cp_async_mbar_arrive(&T->k_full[slot]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&T->k_full[slot]);
         } else {
           // runs of 2^lb_shift consecutive keys (box of min(bs, 128) rows)
           const int bs = 1 << a.lb_shift;
@@ -689,6 +708,9 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           const int slot = kcount % KS;
           if (gg == 0) {
             if (!mbar_wait(&T->k_full[slot], (kcount / KS) & 1, abort, a.status, 4, a.wait_cycles)) { ok = false; break; }
+            // rows written by 16-byte asynchronous copies (generic proxy): order
+            // them before the tensor core's reads
+            if constexpr (GATHER == 1) fence_proxy_async_smem();
           }
           const int s = ucount % NS;
           if (!mbar_wait(&T->t_empty[s], ((ucount / NS) & 1) ^ 1, abort, a.status, 5, a.wait_cycles)) { ok = false; break; }
