@@ -74,6 +74,11 @@ WORKLOADS = {
         desc="DSA indexer decode, 32 sequences x 131072 cached keys, one query each, H_I=64, "
              "d=128, e4m3 K with per-token fp32 scale, bf16 q, fp32 w, top-k=2048",
         kind="decode", batch=32, L=131072, H=64, topk=2048, fp8=True, seed=3, needles=0),
+    "dsa_decode_32k": dict(
+        desc="DSA indexer decode, 32 sequences x 32768 cached keys, one query each, H_I=64, "
+             "d=128, e4m3 K with per-token fp32 scale, bf16 q, fp32 w, top-k=2048 (small case "
+             "of the 128K decode, sized for ncu captures)",
+        kind="decode", batch=32, L=32768, H=64, topk=2048, fp8=True, seed=3, needles=0),
     "misa_prefill_16k": dict(
         desc="MISA prefill, batch 1, L=16384 causal, H_I=64, d=128, B=1024, h=8, top-k=2048, "
              "bf16 (small case of the 128K workload, sized for ncu captures)",

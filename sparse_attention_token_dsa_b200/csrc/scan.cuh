@@ -1066,6 +1066,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           // DoSA: on entering a bound block, this warp's rows' bounds over it
           // (loaded before the wait; rows past the item: +inf, never skipped)
           float ubv[4];
+          unsigned skipm = 0u;
           bool dfresh = false;
           int dblk = 0;
           if constexpr (DOSA) {   // heads >= 32: at most four rows per warp
@@ -1119,21 +1120,17 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               }
               if (gg) { dblk1 = dblk; dmask1 = m; } else { dblk0 = dblk; dmask0 = m; }
             }
-            const unsigned skipm = gg ? dmask1 : dmask0;
-            if (skipm == 0u) {
-              if (qhalf == 2)
-                unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
-              else if (qhalf == 1)
-                unit_heads_n<HT, 1>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
-              else
-                unit_heads<HT>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], qhalf, rbase);
-            } else {
+            skipm = gg ? dmask1 : dmask0;
+            if (skipm != 0u) {
               dosa_n += __popc(skipm);
               for (int qi = 0; qi < qhalf; ++qi)
                 if (!((skipm >> qi) & 1u))
                   unit_heads_n<HT, 1>(fc, taddr + (qbeg + qi) * HT, &T->wsm[(rbase + qi) * HT],
                                       rbase + qi);
             }
+          }
+          if (DOSA && skipm != 0u) {
+            // (pruned rows handled above)
           } else if constexpr (HT >= 32) {
             if (qhalf == 2)
               unit_heads_n<HT, 2>(fc, taddr + qbeg * HT, &T->wsm[rbase * HT], rbase);
