@@ -338,6 +338,28 @@ int dsa_indexer_backward(const dsa_problem* p, const void* q, const void* k, con
                          const int32_t* sel, const float* grad, float* dq, float* dk, float* dw,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* dsa_index with the query rows and results in host memory ("PaperTrace 2.2.2
+ * MISA, LISA and ResMiSA", section 2.3: the indexer runs once per layer on the
+ * whole prefix, its inputs arriving from the host in serving): q_host [batch,
+ * n_q, heads, dim], w_host [batch, n_q, heads] (and q_scale_host [batch, n_q]
+ * for e4m3 q) in page-locked host memory, k / k_scale on the device as for
+ * dsa_index, idx_host / score_host [batch, n_q, topk] in page-locked host
+ * memory.  The rows stream in chunks of chunk_rows through two device slots in
+ * `staging`: host->device copies on one library-owned stream, the scan and
+ * select on `stream`, device->host copies on another, so the copies of one
+ * chunk overlap the scan of the next.  The results equal dsa_index's (same
+ * order rules and flags); work on `stream` after the call starts after every
+ * result has reached the host.  staging: caller-owned device memory of at
+ * least dsa_host_staging_size() bytes, 16-byte aligned; its first 256 bytes
+ * hold the call's device status (the first error of any chunk), read with
+ * dsa_read_status(staging) or returned under DSA_FLAG_CHECK.  Pageable host
+ * memory also works but serialises the copies. */
+int dsa_host_staging_size(const dsa_problem* p, int32_t chunk_rows, size_t* bytes);
+int dsa_index_host(const dsa_problem* p, const void* q_host, const float* q_scale_host,
+                   const void* k, const float* k_scale, const float* w_host,
+                   int32_t* idx_host, float* score_host, int32_t chunk_rows, void* staging,
+                   size_t staging_bytes, void* stream);
+
 /* Operand preparation for the FP8 path: per-row scale a = amax/448 (amax == 0
  * gives a = 1), code = round-to-nearest-even, saturating e4m3 of x/a, both
  * divisions in IEEE fp32 ("PaperTrace 2.2.2", section 2.3 "from formula to

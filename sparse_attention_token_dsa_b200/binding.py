@@ -64,6 +64,8 @@ def _load():
     lib.dsa_status_string.argtypes = [i32]
     lib.dsa_read_status.argtypes = [vp, vp]
     lib.dsa_read_pruned.argtypes = [vp, vp, C.POINTER(C.c_ulonglong)]
+    lib.dsa_host_staging_size.argtypes = [P, i32, C.POINTER(sz)]
+    lib.dsa_index_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_route_chunk_rows.argtypes = [P, i32, R, C.POINTER(i32)]
@@ -78,7 +80,8 @@ def _load():
     lib.dsa_quantize_e4m3.argtypes = [vp, i32, i64, i32, vp, vp, vp]
     lib.dsa_sparse_mla.argtypes = [C.POINTER(DsaMlaProblem), vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_indexer_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
-    for f in ("dsa_read_status", "dsa_read_pruned", "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
+    for f in ("dsa_read_status", "dsa_read_pruned", "dsa_host_staging_size", "dsa_index_host",
+              "dsa_workspace_size", "dsa_route_chunk_rows", "dsa_index",
               "dsa_index_noalloc",
               "dsa_index_scan",
               "dsa_index_select", "misa_index",
@@ -219,6 +222,52 @@ def dsa_index_noalloc(q, k, w, topk, q_scale=None, k_scale=None, q_pos0=None, k_
     _check(lib.dsa_index_noalloc(C.byref(p), _ptr(q), _ptr(q_scale), _ptr(k), _ptr(k_scale),
                                  _ptr(w), _ptr(idx), _ptr(sc), _stream(stream)),
            "dsa_index_noalloc")
+    return idx, sc
+
+
+def _host_args(**named):
+    """Host-side tensors of dsa_index_host: dtype, C-contiguous, on the CPU."""
+    for name, (t, dtypes) in named.items():
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+        if t.dtype not in dtypes:
+            raise TypeError(f"{name}: dtype {t.dtype}, expected one of {dtypes}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if t.device.type != "cpu":
+            raise ValueError(f"{name}: must be in host memory, not {t.device}")
+
+
+def dsa_host_staging_size(p: DsaProblem, chunk_rows: int) -> int:
+    n = C.c_size_t(0)
+    _check(lib.dsa_host_staging_size(C.byref(p), chunk_rows, C.byref(n)), "dsa_host_staging_size")
+    return n.value
+
+
+def dsa_index_host(q_host, k, w_host, topk, q_scale_host=None, k_scale=None, q_pos0=None,
+                   k_len=None, flags=0, chunk_rows=16384, out=None, staging=None, stream=None):
+    """dsa_index with q, w (and q_scale) in (page-locked) host memory and the
+    results written to host tensors; the rows stream in chunks so the copies
+    overlap the scan.  k, k_scale, q_pos0, k_len on the GPU.  Returns host
+    (idx int32 [B, n_q, k], score fp32 [B, n_q, k]); with `out` given, writes there."""
+    _host_args(q_host=(q_host, _OPERAND), w_host=(w_host, _F32), q_scale_host=(q_scale_host, _F32))
+    _args(k=(k, _OPERAND), k_scale=(k_scale, _F32), q_pos0=(q_pos0, _I32), k_len=(k_len, _I32),
+          staging=(staging, _U8))
+    p = problem(q_host, k, topk, q_pos0, k_len, flags)
+    B, nq = q_host.shape[0], q_host.shape[1]
+    if out is None:
+        out = (torch.empty((B, nq, topk), dtype=torch.int32).pin_memory(),
+               torch.empty((B, nq, topk), dtype=torch.float32).pin_memory())
+    idx, sc = out
+    _host_args(out_idx=(idx, _I32), out_score=(sc, _F32))
+    nbytes = dsa_host_staging_size(p, chunk_rows)
+    if staging is None or staging.numel() < nbytes:
+        staging = torch.empty(nbytes, dtype=torch.uint8, device=k.device)
+    _check(lib.dsa_index_host(C.byref(p), _ptr(q_host), _ptr(q_scale_host), _ptr(k), _ptr(k_scale),
+                              _ptr(w_host), _ptr(idx), _ptr(sc), chunk_rows, _ptr(staging),
+                              staging.numel(), _stream(stream)), "dsa_index_host")
     return idx, sc
 
 

@@ -1225,6 +1225,215 @@ int dsa_index_noalloc(const dsa_problem* p, const void* q, const float* q_scale,
                    kNoAllocScratchBytes, stream);
 }
 
+// ------------------------------------------------------- host-buffer path --
+// dsa_index with q, w (and q_scale) in page-locked host memory and the results
+// written back to host memory.  The rows stream in chunks through two device
+// slots: host->device copies on one internal stream, the scan and select on
+// the caller's stream, device->host copies on another, so the copies of one
+// chunk overlap the scan of its neighbours.  Staging layout: a 256-byte header
+// (the call's status, first error over all chunks), then per slot q, w,
+// q_scale, the chunk's causal offsets and its results, then the workspace of
+// one chunk.
+
+}  // extern "C"
+
+namespace {
+
+__global__ void chunk_meta_kernel(const int32_t* q_pos0, const int32_t* k_len, int b, int r0,
+                                  int n_q, int n_k, int32_t* meta) {
+  meta[0] = (q_pos0 ? q_pos0[b] : n_k - n_q) + r0;
+  meta[1] = k_len ? k_len[b] : n_k;
+}
+
+__global__ void sticky_status_kernel(const int32_t* chunk_status, int32_t* call_status) {
+  if (call_status[0] == DSA_OK && chunk_status[0] != DSA_OK) {
+    call_status[0] = chunk_status[0];
+    call_status[1] = chunk_status[1];
+  }
+}
+
+struct HostLayout {
+  int rows;                      // rows per chunk
+  size_t q_row, w_row;           // bytes per query row
+  size_t off_q[2], off_w[2], off_qs[2], off_meta[2], off_idx[2], off_sc[2], off_ws;
+  size_t ws_bytes, total;
+};
+
+int host_layout(const dsa_problem* p, int chunk_rows, HostLayout* L) {
+  if (chunk_rows < 1) return DSA_ERR_INVALID;
+  L->rows = std::min(chunk_rows, p->n_q);
+  const int qesz = p->q_dtype == DSA_F32 ? 4 : (p->q_dtype == DSA_BF16 ? 2 : 1);
+  L->q_row = (size_t)p->heads * p->dim * qesz;
+  L->w_row = (size_t)p->heads * sizeof(float);
+  dsa_problem c = *p;
+  c.batch = 1;
+  c.n_q = L->rows;
+  const size_t R = (size_t)L->rows;
+  size_t off = kWsHeaderBytes;
+  for (int s = 0; s < 2; ++s) {
+    L->off_q[s] = off;
+    off += align_up(R * L->q_row);
+    L->off_w[s] = off;
+    off += align_up(R * L->w_row);
+    L->off_qs[s] = off;
+    if (p->q_dtype == DSA_E4M3) off += align_up(R * sizeof(float));
+    L->off_meta[s] = off;
+    off += align_up(2 * sizeof(int32_t));
+    L->off_idx[s] = off;
+    off += align_up(R * p->topk * sizeof(int32_t));
+    L->off_sc[s] = off;
+    off += align_up(R * p->topk * sizeof(float));
+  }
+  L->off_ws = off;
+  L->ws_bytes = dsa_layout(&c).total;
+  L->total = off + align_up(L->ws_bytes);
+  return DSA_OK;
+}
+
+constexpr int kHostMaxDevices = 64;
+std::mutex g_host_mu;
+cudaStream_t g_host_h2d[kHostMaxDevices], g_host_d2h[kHostMaxDevices];
+
+// The two copy streams of the current device, created once (non-blocking).
+int host_streams(cudaStream_t* h2d, cudaStream_t* d2h) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kHostMaxDevices) {
+    cudaGetLastError();
+    return DSA_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_host_mu);
+  if (!g_host_h2d[dev]) {
+    if (cudaStreamCreateWithFlags(&g_host_h2d[dev], cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&g_host_d2h[dev], cudaStreamNonBlocking) != cudaSuccess) {
+      cudaGetLastError();
+      return DSA_ERR_CUDA;
+    }
+  }
+  *h2d = g_host_h2d[dev];
+  *d2h = g_host_d2h[dev];
+  return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int dsa_host_staging_size(const dsa_problem* p, int32_t chunk_rows, size_t* bytes) {
+  if (!bytes) return DSA_ERR_INVALID;
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  HostLayout L;
+  v = host_layout(p, chunk_rows, &L);
+  if (v != DSA_OK) return v;
+  *bytes = L.total;
+  return DSA_OK;
+}
+
+int dsa_index_host(const dsa_problem* p, const void* q_host, const float* q_scale_host,
+                   const void* k, const float* k_scale, const float* w_host,
+                   int32_t* idx_host, float* score_host, int32_t chunk_rows, void* staging,
+                   size_t staging_bytes, void* stream) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  if (!q_host || !k || !w_host || !idx_host || !score_host) return DSA_ERR_INVALID;
+  if (p->q_dtype == DSA_E4M3 && !q_scale_host) return DSA_ERR_INVALID;
+  if (p->k_dtype == DSA_E4M3 && !k_scale) return DSA_ERR_INVALID;
+  if (!aligned16(k)) return DSA_ERR_INVALID;
+  HostLayout L;
+  v = host_layout(p, chunk_rows, &L);
+  if (v != DSA_OK) return v;
+  if (!staging || staging_bytes < L.total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(staging)) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream), h2d, d2h;
+  v = host_streams(&h2d, &d2h);
+  if (v != DSA_OK) return v;
+  uint8_t* sg = reinterpret_cast<uint8_t*>(staging);
+  int32_t* call_status = reinterpret_cast<int32_t*>(sg);
+  void* ws = sg + L.off_ws;
+  const int kesz = p->k_dtype == DSA_F32 ? 4 : (p->k_dtype == DSA_BF16 ? 2 : 1);
+  const size_t k_seq = (size_t)p->n_k * p->dim * kesz;
+  cudaEvent_t start, h2d_done[2], comp_done[2], d2h_done[2];
+  cudaEvent_t* evs[7] = {&start, &h2d_done[0], &h2d_done[1], &comp_done[0], &comp_done[1],
+                         &d2h_done[0], &d2h_done[1]};
+  int made = 0;
+  for (; made < 7; ++made)
+    if (cudaEventCreateWithFlags(evs[made], cudaEventDisableTiming) != cudaSuccess) break;
+  int rc = made == 7 ? DSA_OK : DSA_ERR_CUDA;
+  int c = 0;
+  if (rc == DSA_OK) {
+    // the copy streams start after the caller's earlier work on its stream
+    if (cudaMemsetAsync(sg, 0, kWsHeaderBytes, st) != cudaSuccess ||
+        cudaEventRecord(start, st) != cudaSuccess || cudaStreamWaitEvent(h2d, start, 0) != cudaSuccess ||
+        cudaStreamWaitEvent(d2h, start, 0) != cudaSuccess)
+      rc = DSA_ERR_CUDA;
+  }
+  for (int b = 0; b < p->batch && rc == DSA_OK; ++b) {
+    for (int r0 = 0; r0 < p->n_q && rc == DSA_OK; r0 += L.rows, ++c) {
+      const int n = std::min(L.rows, p->n_q - r0);
+      const int s = c & 1;
+      const size_t row0 = (size_t)b * p->n_q + r0;
+      bool ok = true;
+      // slot s: its inputs free once chunk c - 2 was scanned, its results once copied out
+      if (c >= 2) ok = ok && cudaStreamWaitEvent(h2d, comp_done[s], 0) == cudaSuccess;
+      ok = ok && cudaMemcpyAsync(sg + L.off_q[s], reinterpret_cast<const uint8_t*>(q_host) + row0 * L.q_row,
+                                 (size_t)n * L.q_row, cudaMemcpyHostToDevice, h2d) == cudaSuccess;
+      ok = ok && cudaMemcpyAsync(sg + L.off_w[s], w_host + row0 * p->heads, (size_t)n * L.w_row,
+                                 cudaMemcpyHostToDevice, h2d) == cudaSuccess;
+      if (p->q_dtype == DSA_E4M3)
+        ok = ok && cudaMemcpyAsync(sg + L.off_qs[s], q_scale_host + row0, (size_t)n * sizeof(float),
+                                   cudaMemcpyHostToDevice, h2d) == cudaSuccess;
+      ok = ok && cudaEventRecord(h2d_done[s], h2d) == cudaSuccess;
+      ok = ok && cudaStreamWaitEvent(st, h2d_done[s], 0) == cudaSuccess;
+      if (c >= 2) ok = ok && cudaStreamWaitEvent(st, d2h_done[s], 0) == cudaSuccess;
+      if (!ok) {
+        rc = DSA_ERR_CUDA;
+        break;
+      }
+      int32_t* meta = reinterpret_cast<int32_t*>(sg + L.off_meta[s]);
+      chunk_meta_kernel<<<1, 1, 0, st>>>(p->q_pos0, p->k_len, b, r0, p->n_q, p->n_k, meta);
+      dsa_problem cp = *p;
+      cp.batch = 1;
+      cp.n_q = n;
+      cp.q_pos0 = meta;
+      cp.k_len = meta + 1;
+      cp.flags = p->flags & ~DSA_FLAG_CHECK;
+      int32_t* idx_d = reinterpret_cast<int32_t*>(sg + L.off_idx[s]);
+      float* sc_d = reinterpret_cast<float*>(sg + L.off_sc[s]);
+      rc = dsa_index(&cp, sg + L.off_q[s],
+                     p->q_dtype == DSA_E4M3 ? reinterpret_cast<const float*>(sg + L.off_qs[s]) : nullptr,
+                     reinterpret_cast<const uint8_t*>(k) + (size_t)b * k_seq,
+                     k_scale ? k_scale + (size_t)b * p->n_k : nullptr,
+                     reinterpret_cast<const float*>(sg + L.off_w[s]), idx_d, sc_d, ws, L.ws_bytes, st);
+      if (rc != DSA_OK) break;
+      sticky_status_kernel<<<1, 1, 0, st>>>(reinterpret_cast<const int32_t*>(ws), call_status);
+      ok = cudaEventRecord(comp_done[s], st) == cudaSuccess &&
+           cudaStreamWaitEvent(d2h, comp_done[s], 0) == cudaSuccess &&
+           cudaMemcpyAsync(idx_host + row0 * p->topk, idx_d, (size_t)n * p->topk * sizeof(int32_t),
+                           cudaMemcpyDeviceToHost, d2h) == cudaSuccess &&
+           cudaMemcpyAsync(score_host + row0 * p->topk, sc_d, (size_t)n * p->topk * sizeof(float),
+                           cudaMemcpyDeviceToHost, d2h) == cudaSuccess &&
+           cudaEventRecord(d2h_done[s], d2h) == cudaSuccess;
+      if (!ok) rc = DSA_ERR_CUDA;
+    }
+  }
+  // the caller's stream continues once every result has reached the host
+  if (rc == DSA_OK) {
+    for (int s = 0; s < 2 && s < c; ++s)
+      if (cudaStreamWaitEvent(st, d2h_done[s], 0) != cudaSuccess) rc = DSA_ERR_CUDA;
+  }
+  for (int i = 0; i < made; ++i) cudaEventDestroy(*evs[i]);
+  if (rc != DSA_OK) {
+    cudaGetLastError();
+    return rc;
+  }
+  if (cudaPeekAtLastError() != cudaSuccess) {
+    cudaGetLastError();
+    return DSA_ERR_CUDA;
+  }
+  if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(staging, stream);
+  return DSA_OK;
+}
+
 int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols, uint8_t* out,
                       float* out_scale, void* stream) {
   if (!x || !out || !out_scale || rows < 0 || cols < 1) return DSA_ERR_INVALID;

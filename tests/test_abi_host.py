@@ -228,3 +228,37 @@ def test_read_pruned_rejects_null(bind):
     n = C.c_ulonglong(0)
     assert bind.lib.dsa_read_pruned(None, None, C.byref(n)) == -1
     assert bind.lib.dsa_read_pruned(C.c_void_p(0x1000), None, None) == -1
+
+
+def test_host_path_validation(bind):
+    f = bind.lib.dsa_index_host
+    fake = C.c_void_p(0x1000)
+    p = _prob(bind)
+    n = C.c_size_t(0)
+    assert bind.lib.dsa_host_staging_size(C.byref(p), 0, C.byref(n)) == -1     # chunk rows < 1
+    assert bind.lib.dsa_host_staging_size(C.byref(_prob(bind, dim=64)), 16, C.byref(n)) == -2
+    sizes = []
+    for rows in (1, 8, 16, 1000):
+        assert bind.lib.dsa_host_staging_size(C.byref(p), rows, C.byref(n)) == 0
+        sizes.append(n.value)
+    assert sizes[0] < sizes[1] < sizes[2] == sizes[3]      # chunks never exceed n_q = 16 rows
+    big = 1 << 34
+    assert f(None, fake, None, fake, None, fake, fake, fake, 8, fake, big, None) == -1
+    assert f(C.byref(p), None, None, fake, None, fake, fake, fake, 8, fake, big, None) == -1
+    assert f(C.byref(p), fake, None, fake, None, fake, None, fake, 8, fake, big, None) == -1
+    assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, 0, fake, big, None) == -1
+    assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, 8, fake, 16, None) == -3
+    assert f(C.byref(p), fake, None, fake, None, fake, fake, fake, 8, C.c_void_p(0x1008), big,
+             None) == -1                                              # misaligned staging
+    e4 = _prob(bind, q_dtype=2, k_dtype=2)
+    assert f(C.byref(e4), fake, None, fake, fake, fake, fake, fake, 8, fake, big, None) == -1
+
+
+def test_host_path_binding_checks_devices(bind):
+    import torch
+    q = torch.zeros((1, 4, 64, 128), dtype=torch.bfloat16)
+    w = torch.zeros((1, 4, 64), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        bind.dsa_index_host(q, q[0, :, 0], w, 2)       # keys must be on the GPU
+    with pytest.raises(TypeError):
+        bind.dsa_index_host(q.float().int(), q[0, :, 0], w, 2)
