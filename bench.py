@@ -896,13 +896,47 @@ def dense_reference(case):
     return didx, d0.elapsed_time(d1)
 
 
+def cutoff_margin(case):
+    """Top-k cut-off margin m = I_(k) - I_(k+1) per row ("PaperTrace 2.2.2",
+    section 2.3: a score error E leaves the selected set unchanged while
+    2E < m), from one sorted top-(k+1) call of the same layer outside the timed
+    region.  Quantiles of m and of m / |I_(k)| over the rows with more than k
+    legal keys, and the rows whose k-th and (k+1)-th scores tie exactly."""
+    import torch
+    B, p = case.B, case.p
+    c = case.calls[0]
+    kk = p.topk + 1
+    prob = B.problem(c["q"], c["k"], kk, c["pos0"], c["klen"], B.DSA_FLAG_SORTED)
+    ws = torch.empty(B.dsa_workspace_size(prob), dtype=torch.uint8, device=case.dev)
+    _, sc = B.dsa_index(c["q"], c["k"], c["w"], kk, q_scale=c["q_scale"], k_scale=c["k_scale"],
+                        q_pos0=c["pos0"], k_len=c["klen"], flags=B.DSA_FLAG_SORTED, workspace=ws)
+    torch.cuda.synchronize()
+    del ws
+    sc = sc.reshape(-1, kk)
+    full = torch.isfinite(sc[:, kk - 1])
+    sk, sk1 = sc[full, kk - 2].double(), sc[full, kk - 1].double()
+    m = sk - sk1
+    rel = m / sk.abs().clamp_min(1e-30)
+    qs = torch.tensor([0.01, 0.1, 0.5, 0.9], dtype=torch.float64, device=m.device)
+    out = {"rows": int(full.sum().item()), "exact_ties": int((m == 0).sum().item()),
+           "quantiles": [0.01, 0.1, 0.5, 0.9],
+           "m": [float(x) for x in torch.quantile(m, qs).tolist()],
+           "m_over_kth": [float(x) for x in torch.quantile(rel, qs).tolist()]} if m.numel() else {}
+    del sc
+    torch.cuda.empty_cache()
+    return out
+
+
 def quality(case, name, ms_per_step, dense=None):
     """Selection quality outside every timed region: needle recall at the probe
     rows; for routed methods the IoU with the exact DSA top-k of the same rows
-    (both on the GPU) and the speed-up over that dense layer."""
+    (both on the GPU) and the speed-up over that dense layer; for the dense
+    layers the top-k cut-off margin."""
     import torch
     p = case.p
     out = {}
+    if case.kind in ("prefill", "decode") and not case.w.get("dosa") and len(case.calls) == 1:
+        out["cutoff_margin"] = cutoff_margin(case)
     gi = case.idx.reshape(p.batch * p.n_q, p.topk)
     if p.needles:
         found = 0

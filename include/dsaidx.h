@@ -372,6 +372,19 @@ int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_NONFINITE).  Synchronises `stream`. */
 int dsa_read_status(const void* workspace, void* stream);
 
+/* The DoSA block upper bounds themselves ("The new bottleneck of sparse
+ * attention", route five), as dsa_index computes them under DSA_FLAG_DOSA:
+ * ub [batch * n_q, ceil(n_k / 1024)] fp32 (caller-owned device memory), for
+ * row t and block a (keys [1024 a, min(1024 (a + 1), n_k)) of its sequence)
+ *   UB = sum_j (w_j > 0 ? w_j ReLU(hi_j) : w_j ReLU(lo_j))
+ *        + 2^-12 sum_j |w_j| ||q_j||_1 max_c max(|kmin_c|, |kmax_c|),
+ * hi_j / lo_j the largest / smallest q_{t,j} . k over the block's
+ * per-dimension key range [kmin, kmax]; -inf for blocks past the row's legal
+ * keys.  p->flags must include DSA_FLAG_DOSA (else DSA_ERR_INVALID); workspace
+ * as dsa_workspace_size reports for that problem. */
+int dsa_dosa_bounds(const dsa_problem* p, const void* q, const void* k, const float* w,
+                    float* ub, void* workspace, size_t workspace_bytes, void* stream);
+
 /* DoSA pruning count recorded in `workspace` by the last dsa_index /
  * dsa_index_scan call with DSA_FLAG_DOSA: (query row, 128-key tile) pairs whose
  * head sums were skipped (0 without the flag).  Synchronises `stream`; the

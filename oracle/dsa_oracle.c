@@ -49,6 +49,14 @@
  *           dk_s     = sum_t sum_j g_{t,s} w_{t,j} m_{t,s,j} q_{t,j}
  *           dw_{t,j} = sum_s g_{t,s} ReLU(z_{t,s,j})
  *         over the selected set S_t (the sparse stage recomputes only there).
+ *  [DOSA] "The new bottleneck of sparse attention", route five (DoSA): a
+ *         candidate whose upper bound lies below a lower bound of the k-th best
+ *         score cannot enter the top-k, so skipping it leaves the top-k exact.
+ *         The bound here is the library's reading: per block of 2^shift keys
+ *         its per-dimension key range, hi / lo the largest / smallest q_j . k
+ *         over that box, UB = sum_j (w_j > 0 ? w_j ReLU(hi_j) : w_j ReLU(lo_j))
+ *         (ReLU is monotone), plus a rounding allowance 2^-12 sum_j |w_j|
+ *         ||q_j||_1 max_c |k|_c.  DoSA's output is DSA's, which [DSA] defines.
  *  [SMLA] "PaperTrace 2.2.2", section 2.3 "end-to-end acceptance", second step:
  *         Sparse MLA on a fixed candidate set S_t, checked by logits, row
  *         maximum, softmax denominator and output against a naive gather
@@ -887,6 +895,61 @@ static int64_t residual_bounds(const orc_inputs* in, int64_t row, int32_t blk, d
   free(kmin);
   free(kmax);
   return m;
+}
+
+/* [DOSA] block upper bounds of one row over the n_k keys of its sequence in
+ * blocks of 2^shift (the last may be partial; every key of a block counts,
+ * legal or not): out[a] = UB_a, out_slack[a] = the rounding allowance (may be
+ * NULL); blocks holding none of the row's legal keys: -inf and 0.  Returns the
+ * number of blocks, ceil(n_k / 2^shift). */
+int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double* out,
+                        double* out_slack) {
+  int32_t b = (int32_t)(row / in->n_q);
+  int64_t bs = (int64_t)1 << shift;
+  int64_t nblk = (in->n_k + bs - 1) / bs;
+  int64_t nleg = row_legal(in, row);
+  int64_t nb_leg = (nleg + bs - 1) / bs;
+  double* kmin = (double*)malloc(sizeof(double) * in->dim);
+  double* kmax = (double*)malloc(sizeof(double) * in->dim);
+  for (int64_t a = 0; a < nblk; ++a) {
+    if (a >= nb_leg) {
+      out[a] = -INFINITY;
+      if (out_slack) out_slack[a] = 0.0;
+      continue;
+    }
+    int64_t lo = a * bs, hi = lo + bs < in->n_k ? lo + bs : in->n_k;
+    double kabs = 0.0;
+    for (int32_t c = 0; c < in->dim; ++c) {
+      kmin[c] = INFINITY;
+      kmax[c] = -INFINITY;
+      for (int64_t s = lo; s < hi; ++s) {
+        double v = k_val(in, b, s, c);
+        if (v < kmin[c]) kmin[c] = v;
+        if (v > kmax[c]) kmax[c] = v;
+      }
+      if (fabs(kmin[c]) > kabs) kabs = fabs(kmin[c]);
+      if (fabs(kmax[c]) > kabs) kabs = fabs(kmax[c]);
+    }
+    double ub = 0.0, sl = 0.0;
+    for (int32_t j = 0; j < in->heads; ++j) {
+      double zhi = 0.0, zlo = 0.0, l1 = 0.0;
+      for (int32_t c = 0; c < in->dim; ++c) {
+        double qc = q_val(in, row, j, c);
+        double a0 = qc * kmin[c], a1 = qc * kmax[c];
+        zhi += MUT(47) ? a0 : (a0 > a1 ? a0 : a1);
+        zlo += a0 < a1 ? a0 : a1;
+        l1 += fabs(qc);
+      }
+      double wj = (double)in->w[row * in->heads + j];
+      ub += wj > 0.0 ? wj * (zhi > 0.0 ? zhi : 0.0) : wj * (zlo > 0.0 ? zlo : 0.0);
+      sl += fabs(wj) * l1;
+    }
+    out[a] = ub;
+    if (out_slack) out_slack[a] = ldexp(sl * kabs, -12);
+  }
+  free(kmin);
+  free(kmax);
+  return nblk;
 }
 
 /* Exported for tests: U^- [M_t, H] of one row; returns M_t. */

@@ -1062,6 +1062,58 @@ int dsa_route_chunk_rows(const dsa_problem* p, int32_t algo, const dsa_route_par
   return DSA_OK;
 }
 
+// DoSA: per-block key ranges into the workspace, then the per-(row, block)
+// upper bounds of I into ub [batch * n_q, L.dosa_nblk].
+static int run_dosa_bounds(const dsa_problem* p, const DsaLayout& L, const void* q, const void* k,
+                    const float* w, uint8_t* ws, float* ub, cudaStream_t st) {
+  uint16_t* E = reinterpret_cast<uint16_t*>(ws + L.off_ranges);
+  float* mx = reinterpret_cast<float*>(ws + L.off_mx);
+  dosa_ranges_kernel<<<dim3((unsigned)L.dosa_nblk, (unsigned)p->batch), 128, 0, st>>>(
+      reinterpret_cast<const uint16_t*>(k), p->n_k, kDosaShift, L.dosa_nblk, E, mx);
+  CUtensorMap qbm, em;
+  if (!make_map(&qbm, q, 2, (uint64_t)p->batch * p->n_q * p->heads, 128)) return DSA_ERR_CUDA;
+  if (!make_map_ranges(&em, E, (uint64_t)L.dosa_nblk, (uint64_t)p->batch)) return DSA_ERR_CUDA;
+  DosaArgs da{};
+  da.batch = p->batch;
+  da.n_q = p->n_q;
+  da.n_tok = p->n_k;
+  da.H = p->heads;
+  da.shift = kDosaShift;
+  da.nblk = L.dosa_nblk;
+  da.q_pos0 = p->q_pos0;
+  da.k_len = p->k_len;
+  da.w = w;
+  da.mx = mx;
+  da.ub = ub;
+  da.status = reinterpret_cast<int32_t*>(ws);
+  if (cudaFuncSetAttribute(dosa_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)dosa_smem_bytes()) != cudaSuccess)
+    return DSA_ERR_CUDA;
+  const int rpc = 128 / p->heads;
+  const int64_t nct = (int64_t)p->batch * ((p->n_q + rpc - 1) / rpc);
+  dosa_bound_kernel<<<(unsigned)nct, kDosaThreads, dosa_smem_bytes(), st>>>(qbm, em, da);
+  return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+int dsa_dosa_bounds(const dsa_problem* p, const void* q, const void* k, const float* w,
+                    float* ub, void* workspace, size_t workspace_bytes, void* stream) {
+  int v = validate_problem(p);
+  if (v != DSA_OK) return v;
+  if (!(p->flags & DSA_FLAG_DOSA)) return DSA_ERR_INVALID;
+  if (!q || !k || !w || !ub) return DSA_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k)) return DSA_ERR_INVALID;
+  const DsaLayout L = dsa_layout(p);
+  if (!workspace || workspace_bytes < L.total) return DSA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return DSA_ERR_INVALID;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+  v = run_dosa_bounds(p, L, q, k, w, ws, ub, st);
+  if (v != DSA_OK) return v;
+  if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(workspace, stream);
+  return DSA_OK;
+}
+
 int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, const void* k,
                    const float* k_scale, const float* w, void* workspace, size_t workspace_bytes,
                    void* stream) {
@@ -1145,34 +1197,9 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.wait_cycles = stall ? kTestWaitCycles : kWaitCycles;
   a.test_stall = stall ? 1 : 0;
   if (p->flags & DSA_FLAG_DOSA) {
-    // per-block key ranges, then per-(row, block) upper bounds of I
-    uint16_t* E = reinterpret_cast<uint16_t*>(ws + L.off_ranges);
-    float* mx = reinterpret_cast<float*>(ws + L.off_mx);
     float* ub = reinterpret_cast<float*>(ws + L.off_ub);
-    dosa_ranges_kernel<<<dim3((unsigned)L.dosa_nblk, (unsigned)p->batch), 128, 0, st>>>(
-        reinterpret_cast<const uint16_t*>(k), p->n_k, kDosaShift, L.dosa_nblk, E, mx);
-    CUtensorMap qbm, em;
-    if (!make_map(&qbm, q, 2, (uint64_t)p->batch * p->n_q * p->heads, 128)) return DSA_ERR_CUDA;
-    if (!make_map_ranges(&em, E, (uint64_t)L.dosa_nblk, (uint64_t)p->batch)) return DSA_ERR_CUDA;
-    DosaArgs da{};
-    da.batch = p->batch;
-    da.n_q = p->n_q;
-    da.n_tok = p->n_k;
-    da.H = p->heads;
-    da.shift = kDosaShift;
-    da.nblk = L.dosa_nblk;
-    da.q_pos0 = p->q_pos0;
-    da.k_len = p->k_len;
-    da.w = w;
-    da.mx = mx;
-    da.ub = ub;
-    da.status = status;
-    if (cudaFuncSetAttribute(dosa_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)dosa_smem_bytes()) != cudaSuccess)
-      return DSA_ERR_CUDA;
-    const int rpc = 128 / p->heads;
-    const int64_t nct = (int64_t)p->batch * ((p->n_q + rpc - 1) / rpc);
-    dosa_bound_kernel<<<(unsigned)nct, kDosaThreads, dosa_smem_bytes(), st>>>(qbm, em, da);
+    v = run_dosa_bounds(p, L, q, k, w, ws, ub, st);
+    if (v != DSA_OK) return v;
     a.dosa_ub = ub;
     a.dosa_nblk = L.dosa_nblk;
     a.dosa_shift = kDosaShift;

@@ -60,6 +60,7 @@ MUTANTS = {
     44: "backward mask 1[z >= 0] instead of 1[z > 0]",
     45: "backward drops the head weight from dq and dk",
     46: "backward dw uses z instead of ReLU(z)",
+    47: "DoSA block bound takes q . kmin for the largest dot product",
 }
 
 
