@@ -115,10 +115,12 @@ enum {
 /* DoSA bound pruning ("The new bottleneck of sparse attention", route five:
  * DoSA, exact pruning by upper and lower bounds).  dsa_index / dsa_index_scan
  * first compute, for every query row and every 1024-token key block, an upper
- * bound of I over the block's keys from the block's per-dimension key range;
- * the scan then skips the head sums of a (row, 128-key tile) pair whose bound
- * lies below the row's running threshold (a lower bound of its final k-th best
- * key).  The selected set and scores are bit-identical to the call without the
+ * and a lower bound of I over the block's keys from the block's per-dimension
+ * key range.  The blocks of largest lower bound holding k legal keys (the seed
+ * set) give each row a starting threshold that none of its k best keys can be
+ * below; the scan raises it as it goes, filters candidates by it, and skips the
+ * head sums of a (row, 128-key tile) pair whose block's upper bound lies below
+ * it.  The selected set and scores are bit-identical to the call without the
  * flag; only the work differs.  bf16 q and k, heads >= 32; otherwise
  * DSA_ERR_UNSUPPORTED.  Needs the larger workspace dsa_workspace_size reports
  * for the flagged problem.  dsa_read_pruned returns the count of skipped pairs. */
@@ -372,18 +374,20 @@ int dsa_quantize_e4m3(const void* x, int32_t x_dtype, int64_t rows, int32_t cols
  * (DSA_OK, DSA_ERR_TIMEOUT or DSA_ERR_NONFINITE).  Synchronises `stream`. */
 int dsa_read_status(const void* workspace, void* stream);
 
-/* The DoSA block upper bounds themselves ("The new bottleneck of sparse
- * attention", route five), as dsa_index computes them under DSA_FLAG_DOSA:
- * ub [batch * n_q, ceil(n_k / 1024)] fp32 (caller-owned device memory), for
- * row t and block a (keys [1024 a, min(1024 (a + 1), n_k)) of its sequence)
- *   UB = sum_j (w_j > 0 ? w_j ReLU(hi_j) : w_j ReLU(lo_j))
- *        + 2^-12 sum_j |w_j| ||q_j||_1 max_c max(|kmin_c|, |kmax_c|),
+/* The DoSA block bounds themselves ("The new bottleneck of sparse attention",
+ * route five), as dsa_index computes them under DSA_FLAG_DOSA:
+ * ub and lb [batch * n_q, ceil(n_k / 1024)] fp32 (caller-owned device memory;
+ * lb may be NULL), for row t and block a (keys [1024 a, min(1024 (a + 1), n_k))
+ * of its sequence), with slack = 2^-12 sum_j |w_j| ||q_j||_1 max_c max(|kmin_c|, |kmax_c|):
+ *   UB = sum_j (w_j > 0 ? w_j ReLU(hi_j) : w_j ReLU(lo_j)) + slack,
+ *   LB = sum_j (w_j > 0 ? w_j ReLU(lo_j) : w_j ReLU(hi_j)) - slack,
  * hi_j / lo_j the largest / smallest q_{t,j} . k over the block's
- * per-dimension key range [kmin, kmax]; -inf for blocks past the row's legal
- * keys.  p->flags must include DSA_FLAG_DOSA (else DSA_ERR_INVALID); workspace
- * as dsa_workspace_size reports for that problem. */
+ * per-dimension key range [kmin, kmax]; -inf (both) for blocks past the row's
+ * legal keys.  UB bounds every key's score in the block from above and LB from
+ * below.  p->flags must include DSA_FLAG_DOSA (else DSA_ERR_INVALID);
+ * workspace as dsa_workspace_size reports for that problem. */
 int dsa_dosa_bounds(const dsa_problem* p, const void* q, const void* k, const float* w,
-                    float* ub, void* workspace, size_t workspace_bytes, void* stream);
+                    float* ub, float* lb, void* workspace, size_t workspace_bytes, void* stream);
 
 /* DoSA pruning count recorded in `workspace` by the last dsa_index /
  * dsa_index_scan call with DSA_FLAG_DOSA: (query row, 128-key tile) pairs whose

@@ -77,7 +77,7 @@ def lib():
         _lib.orc_residual_bounds.restype = C.c_int64
         _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_dosa_bounds.restype = C.c_int64
-        _lib.orc_dosa_bounds.argtypes = [vp, i64, i32, vp, vp]
+        _lib.orc_dosa_bounds.argtypes = [vp, i64, i32, vp, vp, vp]
         _lib.orc_score_row.restype = C.c_int64
         _lib.orc_score_row.argtypes = [vp, i64, vp, i32, vp]
     return _lib
@@ -236,15 +236,17 @@ def residual_bounds(inp: Inputs, row: int, block: int):
 
 
 def dosa_bounds(inp: Inputs, row: int, shift: int):
-    """DoSA block upper bounds of one row ([nblk] UB, [nblk] rounding allowance),
-    blocks of 2^shift keys over the whole sequence; -inf past the legal prefix."""
+    """DoSA block bounds of one row: ([nblk] UB, [nblk] LB, [nblk] rounding
+    allowance), blocks of 2^shift keys over the whole sequence; -inf past the
+    legal prefix."""
     p = inp.prob
     nblk = (p.n_k + (1 << shift) - 1) >> shift
     ub = np.empty(nblk, np.float64)
+    lb = np.empty(nblk, np.float64)
     sl = np.empty(nblk, np.float64)
-    got = lib().orc_dosa_bounds(inp.ref, int(row), shift, _p(ub), _p(sl))
+    got = lib().orc_dosa_bounds(inp.ref, int(row), shift, _p(ub), _p(lb), _p(sl))
     assert got == nblk
-    return ub, sl
+    return ub, lb, sl
 
 
 def score_pairs(inp: Inputs, rows, s, heads=None):

@@ -897,13 +897,14 @@ static int64_t residual_bounds(const orc_inputs* in, int64_t row, int32_t blk, d
   return m;
 }
 
-/* [DOSA] block upper bounds of one row over the n_k keys of its sequence in
- * blocks of 2^shift (the last may be partial; every key of a block counts,
- * legal or not): out[a] = UB_a, out_slack[a] = the rounding allowance (may be
- * NULL); blocks holding none of the row's legal keys: -inf and 0.  Returns the
- * number of blocks, ceil(n_k / 2^shift). */
+/* [DOSA] block bounds of one row over the n_k keys of its sequence in blocks
+ * of 2^shift (the last may be partial; every key of a block counts, legal or
+ * not): out[a] = UB_a, out_lb[a] = LB_a = sum_j (w_j > 0 ? w_j ReLU(lo_j) :
+ * w_j ReLU(hi_j)) (the box's smallest score; may be NULL), out_slack[a] = the
+ * rounding allowance (may be NULL); blocks holding none of the row's legal
+ * keys: -inf, -inf and 0.  Returns the number of blocks, ceil(n_k / 2^shift). */
 int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double* out,
-                        double* out_slack) {
+                        double* out_lb, double* out_slack) {
   int32_t b = (int32_t)(row / in->n_q);
   int64_t bs = (int64_t)1 << shift;
   int64_t nblk = (in->n_k + bs - 1) / bs;
@@ -914,6 +915,7 @@ int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double
   for (int64_t a = 0; a < nblk; ++a) {
     if (a >= nb_leg) {
       out[a] = -INFINITY;
+      if (out_lb) out_lb[a] = -INFINITY;
       if (out_slack) out_slack[a] = 0.0;
       continue;
     }
@@ -930,7 +932,7 @@ int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double
       if (fabs(kmin[c]) > kabs) kabs = fabs(kmin[c]);
       if (fabs(kmax[c]) > kabs) kabs = fabs(kmax[c]);
     }
-    double ub = 0.0, sl = 0.0;
+    double ub = 0.0, lb = 0.0, sl = 0.0;
     for (int32_t j = 0; j < in->heads; ++j) {
       double zhi = 0.0, zlo = 0.0, l1 = 0.0;
       for (int32_t c = 0; c < in->dim; ++c) {
@@ -942,9 +944,14 @@ int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double
       }
       double wj = (double)in->w[row * in->heads + j];
       ub += wj > 0.0 ? wj * (zhi > 0.0 ? zhi : 0.0) : wj * (zlo > 0.0 ? zlo : 0.0);
+      if (MUT(48) ? wj > 0.0 : wj <= 0.0)
+        lb += wj * (zhi > 0.0 ? zhi : 0.0);
+      else
+        lb += wj * (zlo > 0.0 ? zlo : 0.0);
       sl += fabs(wj) * l1;
     }
     out[a] = ub;
+    if (out_lb) out_lb[a] = lb;
     if (out_slack) out_slack[a] = ldexp(sl * kabs, -12);
   }
   free(kmin);

@@ -65,7 +65,7 @@ def _load():
     lib.dsa_read_status.argtypes = [vp, vp]
     lib.dsa_read_pruned.argtypes = [vp, vp, C.POINTER(C.c_ulonglong)]
     lib.dsa_host_staging_size.argtypes = [P, i32, C.POINTER(sz)]
-    lib.dsa_dosa_bounds.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+    lib.dsa_dosa_bounds.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.dsa_index_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, i32, vp, sz, vp]
     lib.dsa_workspace_size.argtypes = [P, i32, R, C.POINTER(sz)]
     lib.dsa_index.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -423,12 +423,14 @@ def dsa_read_pruned(workspace: torch.Tensor, stream=None) -> int:
 
 
 def dsa_dosa_bounds(q, k, w, q_pos0=None, k_len=None, flags=0, workspace=None, stream=None):
-    """DoSA block upper bounds [B * n_q, ceil(n_k / 1024)] fp32 (see include/dsaidx.h)."""
+    """DoSA block upper and lower bounds, each [B * n_q, ceil(n_k / 1024)] fp32
+    (see include/dsaidx.h)."""
     _common_args(q, k, w, q_pos0=q_pos0, k_len=k_len, workspace=workspace)
     p = problem(q, k, 1, q_pos0, k_len, flags | DSA_FLAG_DOSA)
     ws = _workspace(dsa_workspace_size(p), q.device, workspace)
     nblk = (k.shape[1] + 1023) // 1024
     ub = torch.empty((q.shape[0] * q.shape[1], nblk), dtype=torch.float32, device=q.device)
-    _check(lib.dsa_dosa_bounds(C.byref(p), _ptr(q), _ptr(k), _ptr(w), _ptr(ub), _ptr(ws),
-                               ws.numel(), _stream(stream)), "dsa_dosa_bounds")
-    return ub
+    lb = torch.empty_like(ub)
+    _check(lib.dsa_dosa_bounds(C.byref(p), _ptr(q), _ptr(k), _ptr(w), _ptr(ub), _ptr(lb),
+                               _ptr(ws), ws.numel(), _stream(stream)), "dsa_dosa_bounds")
+    return ub, lb

@@ -19,9 +19,15 @@
 // largest |k_c| of the block; UB adds 2^-12 sum_j |w_j| ||q_j||_1 mx_b, so
 // it bounds the score exactly as the scan computes it.
 //
-// The lower bound is the scan's running per-row threshold (its final keep-th
-// best key can only be larger); the scan skips the head sums of a (row, key
-// tile) whose block bound lies below it, so the selected set is unchanged.
+// The same box gives a lower bound of every key's score in the block,
+//     LB_{t,b} = sum_j (w_j > 0 ? w_j ReLU(lo_j) : w_j ReLU(hi_j)) - slack,
+// and so the seed set of the pages' DoSA: the blocks of largest LB, taken until
+// they hold keep legal keys, guarantee keep keys scoring at least the last
+// one's LB — a lower bound of the row's keep-th best score before any key is
+// scanned.  The scan starts each row's threshold there, then raises it as it
+// goes; it skips the head sums of a (row, key tile) whose block UB lies below
+// the threshold.  Every candidate either skipped or filtered out by the seed
+// lies below the keep-th best, so the selected set is unchanged.
 #pragma once
 #include "common.cuh"
 
@@ -83,6 +89,7 @@ struct DosaArgs {
   const float* w;            // [batch * n_q, H]
   const float* mx;           // [batch, nblk]
   float* ub;                 // [batch * n_q, nblk]; blocks past the row's legal keys: -inf
+  float* lb;                 // [batch * n_q, nblk] lower bounds (same blocks), or null
   int32_t* status;
 };
 
@@ -93,6 +100,7 @@ struct DosaSmemTail {
   uint32_t tmem_base;
   int32_t abort;
   float part[2][4][kDosaBT];  // per-warp head sums of a tile (double-buffered)
+  float partl[2][4][kDosaBT]; // the same for the lower bounds
   int32_t okw[2][4];          // the warp's round completed (its partials are valid)
   float slack[4];             // per-warp sum of |w_j| ||q_j||_1
 };
@@ -288,25 +296,35 @@ __global__ void __launch_bounds__(kDosaThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&T->d_empty[buf]);
+      // sum over the warp's 32 heads, all 32 blocks at once: each round keeps
+      // one half of the values and adds the partner lane's copy of it; lane l
+      // ends with block l
+      auto head_sum = [&](float (&v)[32]) {
+#pragma unroll
+        for (int bit = 16; bit >= 1; bit >>= 1) {
+          const bool up = (lane & bit) != 0;
+#pragma unroll
+          for (int x = 0; x < bit; ++x) {
+            const float keep = up ? v[x + bit] : v[x];
+            const float send = up ? v[x] : v[x + bit];
+            v[x] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+          }
+        }
+        return v[0];
+      };
       float v[32];
 #pragma unroll
       for (int x = 0; x < 32; ++x)
         v[x] = wj > 0.f ? wj * fmaxf(__uint_as_float(hv[x]), 0.f)
                         : wj * fmaxf(__uint_as_float(lv[x]), 0.f);
-      // sum over the warp's 32 heads, all 32 blocks at once: each round keeps
-      // one half of the values and adds the partner lane's copy of it; lane l
-      // ends with block l
+      T->part[buf][warp][lane] = head_sum(v);
+      if (a.lb) {
 #pragma unroll
-      for (int bit = 16; bit >= 1; bit >>= 1) {
-        const bool up = (lane & bit) != 0;
-#pragma unroll
-        for (int x = 0; x < bit; ++x) {
-          const float keep = up ? v[x + bit] : v[x];
-          const float send = up ? v[x] : v[x + bit];
-          v[x] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
-        }
+        for (int x = 0; x < 32; ++x)
+          v[x] = wj > 0.f ? wj * fmaxf(__uint_as_float(lv[x]), 0.f)
+                          : wj * fmaxf(__uint_as_float(hv[x]), 0.f);
+        T->partl[buf][warp][lane] = head_sum(v);
       }
-      T->part[buf][warp][lane] = v[0];
       named_bar_sync(1, 128);
       if (leader && active) {
         const int blk = i * kDosaBT + lane;
@@ -316,13 +334,21 @@ __global__ void __launch_bounds__(kDosaThreads, 2)
           float s = 0.f;
           for (int x = 0; x < wpr; ++x) s += T->part[buf][warp + x][lane];
           ubr[blk] = blk < nb_t ? s + srow * mxb[blk] : -__int_as_float(0x7f800000);
+          if (a.lb) {
+            float sl = 0.f;
+            for (int x = 0; x < wpr; ++x) sl += T->partl[buf][warp + x][lane];
+            a.lb[grow * a.nblk + blk] =
+                blk < nb_t ? sl - srow * mxb[blk] : -__int_as_float(0x7f800000);
+          }
         }
       }
     }
     // blocks past the CTA's last legal key
     if (ok && leader && active)
-      for (int blk = nt * kDosaBT + lane; blk < a.nblk; blk += 32)
+      for (int blk = nt * kDosaBT + lane; blk < a.nblk; blk += 32) {
         ubr[blk] = -__int_as_float(0x7f800000);
+        if (a.lb) a.lb[grow * a.nblk + blk] = -__int_as_float(0x7f800000);
+      }
   }
   tc_fence_before();
   __syncthreads();
@@ -331,6 +357,63 @@ __global__ void __launch_bounds__(kDosaThreads, 2)
     tc_fence_after();
     tmem_dealloc(tmem, 128);
   }
+}
+
+// ------------------------------------------------------------- seed set --
+// One warp per query row: the blocks of largest lower bound (ties to the lower
+// block), taken until they hold `keep` of the row's legal keys; the seed is the
+// last one's lower bound (-inf when the row has fewer than keep legal keys or
+// the blocks run out first).  The row's keep best scores are all at least the
+// seed.
+__global__ void __launch_bounds__(256)
+    dosa_seed_kernel(int32_t batch, int32_t n_q, int32_t n_tok, int32_t nblk, int32_t shift,
+                     int32_t keep, const int32_t* __restrict__ q_pos0,
+                     const int32_t* __restrict__ k_len, const float* __restrict__ lb,
+                     float* __restrict__ seed) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (int64_t)batch * n_q) return;
+  const int b = (int)(row / n_q), t = (int)(row % n_q);
+  const int pos0 = q_pos0 ? q_pos0[b] : n_tok - n_q;
+  const int klen = k_len ? k_len[b] : n_tok;
+  const int nleg = max(0, min(pos0 + t + 1, klen));
+  const int nb = min((nleg + (1 << shift) - 1) >> shift, nblk);
+  const float* l = lb + row * nblk;
+  const float ninf = -__int_as_float(0x7f800000);
+  float out = ninf;
+  if (nleg >= keep) {
+    // descending (value, lower block first): the next pick is the largest
+    // entry strictly after the previous one in that order
+    float pv = __int_as_float(0x7f800000);
+    int pa = -1, got = 0;
+    for (int it = 0; it < nb && got < keep; ++it) {
+      float bv = ninf;
+      int ba = nb;
+      for (int x = lane; x < nb; x += 32) {
+        const float v = l[x];
+        const bool after = v < pv || (v == pv && x > pa);
+        if (after && (v > bv || (v == bv && x < ba))) {
+          bv = v;
+          ba = x;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, ba, o);
+        if (ov > bv || (ov == bv && oa < ba)) {
+          bv = ov;
+          ba = oa;
+        }
+      }
+      if (ba >= nb || bv == ninf) break;
+      got += min(1 << shift, nleg - (ba << shift));
+      pv = bv;
+      pa = ba;
+    }
+    if (got >= keep) out = pv;
+  }
+  if (lane == 0) seed[row] = out;
 }
 
 }  // namespace dsa

@@ -464,7 +464,7 @@ constexpr int kDosaShift = 10;
 struct DsaLayout {
   ScanPlan pl;
   size_t off_logs, off_cnt, off_thr, off_parts, off_hscale;
-  size_t off_ranges, off_mx, off_ub;  // DoSA (DSA_FLAG_DOSA) only
+  size_t off_ranges, off_mx, off_ub, off_lb, off_seed;  // DoSA (DSA_FLAG_DOSA) only
   int dosa_nblk;
   size_t total;
 };
@@ -487,7 +487,7 @@ DsaLayout dsa_layout(const dsa_problem* p) {
   if (split) off += align_up((size_t)L.pl.rows * 2 * p->heads * p->dim);
   L.off_hscale = off;
   if (split) off += align_up((size_t)L.pl.rows * p->heads * sizeof(float));
-  L.off_ranges = L.off_mx = L.off_ub = off;
+  L.off_ranges = L.off_mx = L.off_ub = L.off_lb = L.off_seed = off;
   L.dosa_nblk = 0;
   if (p->flags & DSA_FLAG_DOSA) {
     L.dosa_nblk = (p->n_k + (1 << kDosaShift) - 1) >> kDosaShift;
@@ -496,6 +496,10 @@ DsaLayout dsa_layout(const dsa_problem* p) {
     off += align_up((size_t)p->batch * L.dosa_nblk * sizeof(float));
     L.off_ub = off;
     off += align_up((size_t)p->batch * p->n_q * L.dosa_nblk * sizeof(float));
+    L.off_lb = off;
+    off += align_up((size_t)p->batch * p->n_q * L.dosa_nblk * sizeof(float));
+    L.off_seed = off;
+    off += align_up((size_t)p->batch * p->n_q * sizeof(float));
   }
   L.total = off;
   return L;
@@ -1065,7 +1069,7 @@ int dsa_route_chunk_rows(const dsa_problem* p, int32_t algo, const dsa_route_par
 // DoSA: per-block key ranges into the workspace, then the per-(row, block)
 // upper bounds of I into ub [batch * n_q, L.dosa_nblk].
 static int run_dosa_bounds(const dsa_problem* p, const DsaLayout& L, const void* q, const void* k,
-                    const float* w, uint8_t* ws, float* ub, cudaStream_t st) {
+                    const float* w, uint8_t* ws, float* ub, float* lb, cudaStream_t st) {
   uint16_t* E = reinterpret_cast<uint16_t*>(ws + L.off_ranges);
   float* mx = reinterpret_cast<float*>(ws + L.off_mx);
   dosa_ranges_kernel<<<dim3((unsigned)L.dosa_nblk, (unsigned)p->batch), 128, 0, st>>>(
@@ -1085,6 +1089,7 @@ static int run_dosa_bounds(const dsa_problem* p, const DsaLayout& L, const void*
   da.w = w;
   da.mx = mx;
   da.ub = ub;
+  da.lb = lb ? lb : reinterpret_cast<float*>(ws + L.off_lb);
   da.status = reinterpret_cast<int32_t*>(ws);
   if (cudaFuncSetAttribute(dosa_bound_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dosa_smem_bytes()) != cudaSuccess)
@@ -1092,11 +1097,16 @@ static int run_dosa_bounds(const dsa_problem* p, const DsaLayout& L, const void*
   const int rpc = 128 / p->heads;
   const int64_t nct = (int64_t)p->batch * ((p->n_q + rpc - 1) / rpc);
   dosa_bound_kernel<<<(unsigned)nct, kDosaThreads, dosa_smem_bytes(), st>>>(qbm, em, da);
+  // the seed set: a lower bound of each row's keep-th best score
+  const int64_t rows = (int64_t)p->batch * p->n_q;
+  dosa_seed_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
+      p->batch, p->n_q, p->n_k, L.dosa_nblk, kDosaShift, p->topk, p->q_pos0, p->k_len, da.lb,
+      reinterpret_cast<float*>(ws + L.off_seed));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 int dsa_dosa_bounds(const dsa_problem* p, const void* q, const void* k, const float* w,
-                    float* ub, void* workspace, size_t workspace_bytes, void* stream) {
+                    float* ub, float* lb, void* workspace, size_t workspace_bytes, void* stream) {
   int v = validate_problem(p);
   if (v != DSA_OK) return v;
   if (!(p->flags & DSA_FLAG_DOSA)) return DSA_ERR_INVALID;
@@ -1108,7 +1118,7 @@ int dsa_dosa_bounds(const dsa_problem* p, const void* q, const void* k, const fl
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   if (cudaMemsetAsync(ws, 0, kWsHeaderBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
-  v = run_dosa_bounds(p, L, q, k, w, ws, ub, st);
+  v = run_dosa_bounds(p, L, q, k, w, ws, ub, lb, st);
   if (v != DSA_OK) return v;
   if (p->flags & DSA_FLAG_CHECK) return dsa_read_status(workspace, stream);
   return DSA_OK;
@@ -1198,9 +1208,10 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
   a.test_stall = stall ? 1 : 0;
   if (p->flags & DSA_FLAG_DOSA) {
     float* ub = reinterpret_cast<float*>(ws + L.off_ub);
-    v = run_dosa_bounds(p, L, q, k, w, ws, ub, st);
+    v = run_dosa_bounds(p, L, q, k, w, ws, ub, nullptr, st);
     if (v != DSA_OK) return v;
     a.dosa_ub = ub;
+    a.dosa_seed = reinterpret_cast<const float*>(ws + L.off_seed);
     a.dosa_nblk = L.dosa_nblk;
     a.dosa_shift = kDosaShift;
     a.dosa_pruned = reinterpret_cast<unsigned long long*>(ws + offsetof(WsHeader, pruned));

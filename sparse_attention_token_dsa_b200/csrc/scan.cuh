@@ -89,6 +89,8 @@ struct ScanArgs {
   int32_t dosa_nblk;     //   bound blocks per row
   int32_t dosa_shift;    //   log2 tokens per bound block (>= 7: a key tile lies in one block)
   unsigned long long* dosa_pruned;  // (row, unit) pairs skipped, or null
+  const float* dosa_seed;  // DoSA: per row a lower bound of its keep-th best score [rows]
+                           //   (-inf: none), the row threshold's starting value
   int32_t test_stall;    // DSA_FLAG_TEST_STALL: CTA 0 withholds the second K stage of
                          //   its first item, so the waits on it run out (tests only)
 };
@@ -989,7 +991,16 @@ __global__ void __launch_bounds__(kScanThreads, 1)
       const int64_t slot0 = ((int64_t)g.b * a.n_q + g.row0) * a.C + g.c;  // slot of row 0
       // ---- item init: row states, histograms, head weights
       for (int r = etid; r < QT; r += kEpiThreads) {
-        T->row_thr[r] = 0ull;
+        unsigned long long thr0 = 0ull;
+        if constexpr (DOSA) {
+          // the seed set's guarantee: keep legal keys score at least the seed, so
+          // a threshold at its key (index part 0) drops none of the keep best
+          if (r < g.nrows) {
+            const float sd = a.dosa_seed[(int64_t)g.b * a.q_stride + a.q_off + g.row0 + r];
+            if (sd != -__int_as_float(0x7f800000)) thr0 = (unsigned long long)score_key(sd) << 32;
+          }
+        }
+        T->row_thr[r] = thr0;
         T->row_b1[r] = -1;
         T->row_raise[r] = 0;
         int nleg = 0;

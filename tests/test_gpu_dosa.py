@@ -184,34 +184,38 @@ def test_full_size_32k_bit_identical(B):
 @pytest.mark.parametrize("kind", ["integer", "normal"])
 def test_block_bounds_match_oracle_and_dominate_every_legal_score(B, kind):
     """The bound kernel (tcgen05 GEMM of [q+ | q-] against the block ranges)
-    against the oracle's block bound plus its rounding allowance: exact on
+    against the oracle's block bounds with their rounding allowance: exact on
     integer inputs up to the fp32 allowance, within half the allowance on real
-    inputs; and never below the oracle's score of any legal key of the block
-    (partial last blocks, ragged prefixes, blocks past the prefix at -inf)."""
+    inputs; the upper bound never below and the lower bound never above the
+    oracle's score of any legal key of the block (partial last blocks, ragged
+    prefixes, blocks past the prefix at -inf)."""
     if kind == "integer":
         p = gen.segment_integer_problem(47, 2, 150, 3000, 64, 128, 32, seg=512,
                                         q_pos0=[2850, 100], k_len=[3000, 2400])
     else:
         p = gen.normal_problem(48, 2, 150, 3000, 64, 128, 32, q_pos0=[2850, 100],
                                k_len=[3000, 2400])
-    ub = B.dsa_dosa_bounds(dev(p.q), dev(p.k), dev(p.w), q_pos0=dev(p.q_pos0),
-                           k_len=dev(p.k_len)).cpu().numpy().astype(np.float64)
+    ubt, lbt = B.dsa_dosa_bounds(dev(p.q), dev(p.k), dev(p.w), q_pos0=dev(p.q_pos0),
+                                 k_len=dev(p.k_len))
+    ub = ubt.cpu().numpy().astype(np.float64)
+    lb = lbt.cpu().numpy().astype(np.float64)
     inp = oracle.Inputs(p)
     nblk = ub.shape[1]
     assert nblk == 3
     worst = 0.0
     for row in range(p.batch * p.n_q):
-        ref, sl = oracle.dosa_bounds(inp, row, 10)
+        ref, lref, sl = oracle.dosa_bounds(inp, row, 10)
         n = p.legal_count(row)
         for a in range(nblk):
             if a * 1024 >= n:
-                assert ub[row, a] == -np.inf
+                assert ub[row, a] == -np.inf and lb[row, a] == -np.inf
                 continue
-            want = ref[a] + sl[a]
-            tol = (1e-6 * (abs(ref[a]) + sl[a]) + 1e-6) if kind == "integer" else 0.5 * sl[a]
-            assert abs(ub[row, a] - want) <= tol, (row, a, ub[row, a], want)
-            worst = max(worst, abs(ub[row, a] - want) / max(sl[a], 1e-30))
             s = np.arange(a * 1024, min((a + 1) * 1024, n))
             I = oracle.score_pairs(inp, np.full(len(s), row), s)
+            for got, want in ((ub[row, a], ref[a] + sl[a]), (lb[row, a], lref[a] - sl[a])):
+                tol = (1e-6 * (abs(want) + sl[a]) + 1e-6) if kind == "integer" else 0.5 * sl[a]
+                assert abs(got - want) <= tol, (row, a, got, want)
+                worst = max(worst, abs(got - want) / max(sl[a], 1e-30))
             assert ub[row, a] >= I.max()
+            assert lb[row, a] <= I.min()
     print(f"dosa bounds {kind}: largest |gpu - oracle| / allowance {worst:.3e}")

@@ -61,6 +61,7 @@ MUTANTS = {
     45: "backward drops the head weight from dq and dk",
     46: "backward dw uses z instead of ReLU(z)",
     47: "DoSA block bound takes q . kmin for the largest dot product",
+    48: "DoSA lower bound weighs the wrong box extreme by the head sign",
 }
 
 

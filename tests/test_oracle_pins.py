@@ -614,11 +614,11 @@ def test_residual_bound_covers_every_legal_key_and_no_future_key(oracle_mod):
 
 
 def test_dosa_bound_covers_every_legal_key(oracle_mod):
-    """DoSA's block upper bound is >= I_{t,s} for every legal key s of the block
-    (brute force over the row), including the row's partial last block, and
-    -inf for blocks past its legal prefix ("The new bottleneck of sparse
-    attention", route five: only a bound that truly dominates the block keeps
-    the top-k exact)."""
+    """DoSA's block upper bound is >= I_{t,s} and its lower bound <= I_{t,s} for
+    every legal key s of the block (brute force over the row), including the
+    row's partial last block, and both -inf for blocks past its legal prefix
+    ("The new bottleneck of sparse attention", route five: only bounds that
+    truly enclose the block keep the top-k exact)."""
     rng = np.random.default_rng(13)
     nq, nk, H, d, shift = 5, 700, 6, 8, 7
     q = rng.standard_normal((1, nq, H, d)).astype(np.float32)
@@ -627,16 +627,18 @@ def test_dosa_bound_covers_every_legal_key(oracle_mod):
     inp = oracle_mod.Inputs(make(q, k, w, topk=4, q_pos0=[300]))
     bs = 1 << shift
     for row in range(nq):
-        ub, sl = oracle_mod.dosa_bounds(inp, row, shift)
+        ub, lb, sl = oracle_mod.dosa_bounds(inp, row, shift)
         n = 300 + row + 1
         assert ub.shape == ((nk + bs - 1) // bs,)
         s = np.arange(n)
         I = oracle_mod.score_pairs(inp, np.full(n, row), s)
         for a in range(len(ub)):
             if a * bs >= n:
-                assert ub[a] == -np.inf and sl[a] == 0.0
+                assert ub[a] == -np.inf and lb[a] == -np.inf and sl[a] == 0.0
                 continue
-            assert ub[a] >= I[a * bs:min((a + 1) * bs, n)].max() - 1e-12
+            blk = I[a * bs:min((a + 1) * bs, n)]
+            assert ub[a] >= blk.max() - 1e-12
+            assert lb[a] <= blk.min() + 1e-12
             assert sl[a] > 0.0
 
 
@@ -651,10 +653,11 @@ def test_dosa_bound_is_exact_on_constant_blocks(oracle_mod):
     w = rng.standard_normal((1, nq, H)).astype(np.float32)
     inp = oracle_mod.Inputs(make(q, k, w, topk=4))
     for row in range(nq):
-        ub, _ = oracle_mod.dosa_bounds(inp, row, shift)
+        ub, lb, _ = oracle_mod.dosa_bounds(inp, row, shift)
         for a in range(len(ub)):
             I = oracle_mod.score_pairs(inp, [row], [a << shift])[0]
             assert abs(ub[a] - I) <= 1e-12 * max(1.0, abs(I))
+            assert abs(lb[a] - I) <= 1e-12 * max(1.0, abs(I))
 
 
 def test_resmisa_routes_by_weight_magnitude(oracle_mod):
