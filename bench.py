@@ -150,7 +150,7 @@ WORKLOADS = {
 ROUTED = ("misa", "dagger", "hisa", "lisa", "resmisa")
 
 KERNEL_SOURCES = ["common.cuh", "scan.cuh", "select.cuh"]
-TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic_scan_kernel.md")
+TRAFFIC_TABLE = os.path.join(ROOT, "profiles", "traffic_scan_kernel.txt")
 
 
 def kernel_hash() -> str:
