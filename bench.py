@@ -655,7 +655,7 @@ class Case:
             c["ws_bytes"] = B.dsa_workspace_size(c["prob"])
             c["launches"] = 2 + (1 if (self.fp8 and self.kind == "decode") else 0)
             if w.get("dosa"):
-                c["launches"] += 2                   # key ranges + bounds
+                c["launches"] += 3                   # key ranges, bounds, seeds
         return c
 
     def _routed(self, c, q, k, w_, out):

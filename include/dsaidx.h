@@ -355,7 +355,9 @@ int dsa_indexer_backward(const dsa_problem* p, const void* q, const void* k, con
  * least dsa_host_staging_size() bytes, 16-byte aligned; its first 256 bytes
  * hold the call's device status (the first error of any chunk), read with
  * dsa_read_status(staging) or returned under DSA_FLAG_CHECK.  Pageable host
- * memory also works but serialises the copies. */
+ * memory also works but serialises the copies.  The two copy streams are
+ * created on the first call on a device and kept for the process: do not call
+ * it on a device again after a cudaDeviceReset there. */
 int dsa_host_staging_size(const dsa_problem* p, int32_t chunk_rows, size_t* bytes);
 int dsa_index_host(const dsa_problem* p, const void* q_host, const float* q_scale_host,
                    const void* k, const float* k_scale, const float* w_host,
