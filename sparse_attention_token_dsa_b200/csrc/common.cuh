@@ -18,7 +18,9 @@ struct WsHeader {
   int32_t status;     // DSA_OK or a negative device status (first error wins)
   int32_t where;      // which wait gave up (diagnostic)
   unsigned long long pruned;  // DoSA: (query row, key tile) pairs skipped
-  int32_t pad[60];
+  unsigned long long dosa_blocks;      // DoSA: (row, block) pairs holding legal keys
+  unsigned long long dosa_ruled_out;   //   of which the seed alone rules out (UB < seed)
+  int32_t pad[56];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 constexpr size_t kWsHeaderBytes = 256;

@@ -365,11 +365,15 @@ __global__ void __launch_bounds__(kDosaThreads, 2)
 // last one's lower bound (-inf when the row has fewer than keep legal keys or
 // the blocks run out first).  The row's keep best scores are all at least the
 // seed.
+// It also counts the row's blocks and those whose upper bound already lies
+// below the seed (atomically, into counts[0] and counts[1]): the share the
+// bounds are sure to prune, which decides whether the scan checks them.
 __global__ void __launch_bounds__(256)
     dosa_seed_kernel(int32_t batch, int32_t n_q, int32_t n_tok, int32_t nblk, int32_t shift,
                      int32_t keep, const int32_t* __restrict__ q_pos0,
                      const int32_t* __restrict__ k_len, const float* __restrict__ lb,
-                     float* __restrict__ seed) {
+                     const float* __restrict__ ub, float* __restrict__ seed,
+                     unsigned long long* __restrict__ counts) {
   const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (int64_t)batch * n_q) return;
@@ -414,6 +418,15 @@ __global__ void __launch_bounds__(256)
     if (got >= keep) out = pv;
   }
   if (lane == 0) seed[row] = out;
+  unsigned ruled = 0;
+  const float* u = ub + row * nblk;
+  for (int x = lane; x < nb; x += 32) ruled += u[x] < out ? 1u : 0u;
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) ruled += __shfl_xor_sync(0xffffffffu, ruled, o);
+  if (lane == 0 && nb > 0) {
+    atomicAdd(&counts[0], (unsigned long long)nb);
+    if (ruled) atomicAdd(&counts[1], (unsigned long long)ruled);
+  }
 }
 
 }  // namespace dsa

@@ -1101,7 +1101,8 @@ static int run_dosa_bounds(const dsa_problem* p, const DsaLayout& L, const void*
   const int64_t rows = (int64_t)p->batch * p->n_q;
   dosa_seed_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(
       p->batch, p->n_q, p->n_k, L.dosa_nblk, kDosaShift, p->topk, p->q_pos0, p->k_len, da.lb,
-      reinterpret_cast<float*>(ws + L.off_seed));
+      ub, reinterpret_cast<float*>(ws + L.off_seed),
+      reinterpret_cast<unsigned long long*>(ws + offsetof(WsHeader, dosa_blocks)));
   return cudaGetLastError() == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -1212,6 +1213,7 @@ int dsa_index_scan(const dsa_problem* p, const void* q, const float* q_scale, co
     if (v != DSA_OK) return v;
     a.dosa_ub = ub;
     a.dosa_seed = reinterpret_cast<const float*>(ws + L.off_seed);
+    a.dosa_counts = reinterpret_cast<const unsigned long long*>(ws + offsetof(WsHeader, dosa_blocks));
     a.dosa_nblk = L.dosa_nblk;
     a.dosa_shift = kDosaShift;
     a.dosa_pruned = reinterpret_cast<unsigned long long*>(ws + offsetof(WsHeader, pruned));

@@ -91,6 +91,9 @@ struct ScanArgs {
   unsigned long long* dosa_pruned;  // (row, unit) pairs skipped, or null
   const float* dosa_seed;  // DoSA: per row a lower bound of its keep-th best score [rows]
                            //   (-inf: none), the row threshold's starting value
+  const unsigned long long* dosa_counts;  // DoSA: (row, block) pairs with legal keys, and
+                           //   those the seeds alone rule out; the block checks run only
+                           //   when at least 1/32 of them are
   int32_t test_stall;    // DSA_FLAG_TEST_STALL: CTA 0 withholds the second K stage of
                          //   its first item, so the waits on it run out (tests only)
 };
@@ -978,6 +981,11 @@ __global__ void __launch_bounds__(kScanThreads, 1)
     int step_par = 0;
     bool stop = false;
     uint32_t dosa_n = 0;                       // DoSA: (row, unit) pairs this warp skipped
+    // DoSA: check the block bounds only where they are seen to bite (the seeds
+    // alone rule out at least 1/32 of the blocks); otherwise the per-unit checks
+    // would cost more than they save (the seeded thresholds still apply)
+    bool dosa_on = false;
+    if constexpr (DOSA) dosa_on = a.dosa_counts[1] * 32ull >= a.dosa_counts[0] && a.dosa_counts[1] > 0;
     for (int round = 0; !stop; ++round) {
       const int item = sched_item(round, blockIdx.x, grid);
       if (item >= a.n_items) break;
@@ -1080,7 +1088,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           unsigned skipm = 0u;
           bool dfresh = false;
           int dblk = 0;
-          if constexpr (DOSA) {   // heads >= 32: at most four rows per warp
+          if constexpr (DOSA) if (dosa_on) {   // heads >= 32: at most four rows per warp
             dblk = ((g.t_hi - t * KT) << 7) >> a.dosa_shift;
             dfresh = dblk != (gg ? dblk1 : dblk0);
             if (dfresh) {
@@ -1116,7 +1124,7 @@ __global__ void __launch_bounds__(kScanThreads, 1)
           fc.T = T;
           fc.capw = a.capw;
           fc.status = a.status;
-          if constexpr (DOSA) {
+          if constexpr (DOSA) if (dosa_on) {
             // DoSA: a row whose upper bound over the tile's block lies below its
             // threshold (a lower bound of its final keep-th best) has no candidate
             // the filter could keep in the block; its head sums are skipped.  A

@@ -1,9 +1,11 @@
 """DoSA bound pruning (DSA_FLAG_DOSA): the selected set and every score are
 bit-identical to the same call without the flag, on integer inputs (exact, and
 also equal to the oracle), on real-valued inputs (and within the tolerance rule
-of the oracle), on ragged batches, decode and every supported head count; the
-pruning count is positive where the block bound is tight (keys with locality)
-and zero without the flag.
+of the oracle), on ragged batches, decode and every supported head count; most
+(row, tile) pairs are pruned where the block bounds are tight (keys constant
+over blocks), none without the flag.  Where the seeds rule out fewer than 1/32
+of the blocks the scan does not check the bounds at all (the counts and
+thresholds stay exact either way).
 
 DoSA ("The new bottleneck of sparse attention", route five) keeps the exact
 top-k: a (row, key tile) pair is skipped only when an upper bound of every
@@ -87,7 +89,7 @@ def test_integer_segments_bit_exact_and_pruned(B):
     parity.exact(i1, s1, ri, rs)
     total = tile_pairs(p)
     print(f"dosa integer segments: pruned {pruned} of {total} pairs")
-    assert 0 < pruned <= total
+    assert total // 2 < pruned <= total          # the seeds rule out most blocks
 
 
 @pytest.mark.parametrize("heads", [32, 64, 128])
@@ -100,7 +102,6 @@ def test_low_noise_clusters_bit_identical(B, heads):
     i0, s0, i1, s1, pruned = both(B, p)
     identical(i0, s0, i1, s1)
     print(f"dosa clusters H={heads}: pruned {pruned} of {tile_pairs(p)} pairs")
-    assert pruned > 0
     inp = oracle.Inputs(p)
     rows = np.arange(p.n_q)[::37]
     ri, _, rs64, _ = oracle.dsa(inp, p.topk, rows)
@@ -141,6 +142,7 @@ def test_decode_bit_identical(B):
     ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
     parity.exact(i1, s1, ri, rs)
     print(f"dosa decode: pruned {pruned} of {tile_pairs(p)} pairs")
+    assert pruned > tile_pairs(p) // 2          # the seeds rule out most blocks
 
 
 def test_position_order_with_dosa(B):
@@ -178,7 +180,6 @@ def test_full_size_32k_bit_identical(B):
     assert torch.equal(res[0][0], res[1][0])
     assert torch.equal(res[0][1].view(torch.int32), res[1][1].view(torch.int32))
     print(f"dosa 32k: pruned {res[1][2]} of about {L * (L // 128) // 2} pairs")
-    assert res[1][2] > 0
 
 
 @pytest.mark.parametrize("kind", ["integer", "normal"])

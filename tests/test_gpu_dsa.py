@@ -319,3 +319,17 @@ def test_position_order_bit_exact(B, topk):
         assert np.array_equal(gi[r][:nv], ri[r][:nv][order])
         assert np.array_equal(gs[r][:nv], rs[r][:nv][order])
         assert np.all(gi[r][nv:] == -1) and np.all(np.isneginf(gs[r][nv:]))
+
+
+@pytest.mark.parametrize("dosa", [False, True])
+def test_integer_empty_cache_and_positions_past_the_cache(B, dosa):
+    """A sequence with an empty cache (k_len = 0: every row pads), rows whose
+    positions lie past their sequence's cache (all k_len keys legal), and an
+    ordinary sequence, in one call; with and without DoSA."""
+    p = gen.integer_problem(30, 3, 200, 900, 64, 128, 64, q_pos0=[0, 700, 100],
+                            k_len=[0, 300, 900], dtype=gen.BF16)
+    flags = B.DSA_FLAG_CHECK | B.DSA_FLAG_SORTED | (B.DSA_FLAG_DOSA if dosa else 0)
+    gi, gs = run_dsa(B, p, flags=flags)
+    ri, rs, _, _ = oracle.dsa(oracle.Inputs(p), p.topk)
+    parity.exact(gi, gs, ri, rs)
+    assert np.all(gi[:p.n_q] == -1) and np.all(np.isneginf(gs[:p.n_q]))
