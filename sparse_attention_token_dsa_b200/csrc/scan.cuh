@@ -625,7 +625,8 @@ __global__ void __launch_bounds__(kScanThreads, 1)
               set_status(a.status, DSA_ERR_INTERNAL, 112);
               blk = -1;
             }
-            ybox = krow0 + (blk >= 0 ? blk * bs + (e & (bs - 1)) : 0);
+            // an empty slot loads a box wholly before row 0: zero fill, no traffic
+            ybox = blk >= 0 ? krow0 + blk * bs + (e & (bs - 1)) : -box;
           }
         }
         // tiles of this stage inside the item (a ragged last stage loads one)
