@@ -204,27 +204,36 @@ __device__ __forceinline__ int sched_item(int round, int cta, int grid) {
 }
 
 // In-place warp compaction of one sub-log: keep entries >= thr; returns the
-// count.  Eight independent loads per lane are in flight per round.
+// count.  Rounds of 256 entries (eight loads per lane); the next round's loads
+// are issued before this round's writes, which land below the next round's
+// range (the write position never passes the read position), so they overlap.
 __device__ __forceinline__ int compact_sublog(uint64_t* lg, int n, unsigned long long thr,
                                               int lane) {
   int wpos = 0;
+  uint64_t cur[8], nxt[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = j * 32 + lane;
+    cur[j] = i < n ? lg[i] : 0ull;
+  }
   for (int i0 = 0; i0 < n; i0 += 256) {
-    uint64_t vv[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      const int i = i0 + j * 32 + lane;
-      vv[j] = i < n ? lg[i] : 0ull;
+      const int i = i0 + 256 + j * 32 + lane;
+      nxt[j] = i < n ? lg[i] : 0ull;
     }
     __syncwarp();
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const int i = i0 + j * 32 + lane;
-      const bool kp = i < n && vv[j] >= thr;
+      const bool kp = i < n && cur[j] >= thr;
       const unsigned bal = __ballot_sync(0xffffffffu, kp);
-      if (kp) lg[wpos + __popc(bal & ((1u << lane) - 1))] = vv[j];
+      if (kp) lg[wpos + __popc(bal & ((1u << lane) - 1))] = cur[j];
       wpos += __popc(bal);
     }
     __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) cur[j] = nxt[j];
   }
   return wpos;
 }
