@@ -78,6 +78,8 @@ def lib():
         _lib.orc_residual_bounds.argtypes = [vp, i64, i32, vp]
         _lib.orc_dosa_bounds.restype = C.c_int64
         _lib.orc_dosa_bounds.argtypes = [vp, i64, i32, vp, vp, vp]
+        _lib.orc_dosa_seed.restype = C.c_double
+        _lib.orc_dosa_seed.argtypes = [vp, i64, i32, i32]
         _lib.orc_score_row.restype = C.c_int64
         _lib.orc_score_row.argtypes = [vp, i64, vp, i32, vp]
     return _lib
@@ -247,6 +249,12 @@ def dosa_bounds(inp: Inputs, row: int, shift: int):
     got = lib().orc_dosa_bounds(inp.ref, int(row), shift, _p(ub), _p(lb), _p(sl))
     assert got == nblk
     return ub, lb, sl
+
+
+def dosa_seed(inp: Inputs, row: int, shift: int, keep: int) -> float:
+    """DoSA seed-set lower bound of one row's keep-th best score (-inf when the
+    row has fewer than keep legal keys)."""
+    return float(lib().orc_dosa_seed(inp.ref, int(row), shift, keep))
 
 
 def score_pairs(inp: Inputs, rows, s, heads=None):

@@ -959,6 +959,40 @@ int64_t orc_dosa_bounds(const orc_inputs* in, int64_t row, int32_t shift, double
   return nblk;
 }
 
+/* [DOSA] seed-set lower bound of one row's keep-th best score: the blocks of
+ * largest LB (ties to the lower block), taken in that order until they hold
+ * keep of the row's legal keys; the seed is the last block's LB (-INFINITY when
+ * the row has fewer than keep legal keys).  Every key of a chosen block scores
+ * at least its LB, so keep legal keys score at least the seed. */
+double orc_dosa_seed(const orc_inputs* in, int64_t row, int32_t shift, int32_t keep) {
+  int64_t bs = (int64_t)1 << shift;
+  int64_t nblk = (in->n_k + bs - 1) / bs;
+  int64_t nleg = row_legal(in, row);
+  if (nleg < keep) return -INFINITY;
+  double* ub = (double*)malloc(sizeof(double) * nblk);
+  double* lb = (double*)malloc(sizeof(double) * nblk);
+  orc_dosa_bounds(in, row, shift, ub, lb, NULL);
+  int64_t nb = (nleg + bs - 1) / bs;
+  char* used = (char*)calloc((size_t)nb, 1);
+  int64_t got = 0;
+  double seed = -INFINITY;
+  while (got < keep) {
+    int64_t best = -1;
+    for (int64_t a = 0; a < nb; ++a)
+      if (!used[a] && (best < 0 || lb[a] > lb[best])) best = a;
+    if (best < 0) break;
+    used[best] = 1;
+    int64_t cnt = nleg - best * bs;
+    if (cnt > bs) cnt = bs;
+    got += MUT(49) ? bs : cnt;
+    seed = lb[best];
+  }
+  free(ub);
+  free(lb);
+  free(used);
+  return got >= keep ? seed : -INFINITY;
+}
+
 /* Exported for tests: U^- [M_t, H] of one row; returns M_t. */
 int64_t orc_residual_bounds(const orc_inputs* in, int64_t row, int32_t blk, double* out) {
   return residual_bounds(in, row, blk, out);

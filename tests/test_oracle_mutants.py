@@ -62,6 +62,7 @@ MUTANTS = {
     46: "backward dw uses z instead of ReLU(z)",
     47: "DoSA block bound takes q . kmin for the largest dot product",
     48: "DoSA lower bound weighs the wrong box extreme by the head sign",
+    49: "DoSA seed set counts a partial block as full",
 }
 
 

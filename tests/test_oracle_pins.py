@@ -660,6 +660,47 @@ def test_dosa_bound_is_exact_on_constant_blocks(oracle_mod):
             assert abs(lb[a] - I) <= 1e-12 * max(1.0, abs(I))
 
 
+def test_dosa_seed_is_a_lower_bound_of_the_kth_best(oracle_mod):
+    """The seed set guarantees keep legal keys at or above the seed, so the
+    row's keep-th best score is >= the seed (brute force over the row); rows
+    with fewer than keep legal keys get no seed.  On keys constant per block
+    the seed is exactly the score of the block that completes the count."""
+    rng = np.random.default_rng(15)
+    nq, nk, H, d, shift, keep = 6, 900, 6, 8, 7, 200
+    q = rng.standard_normal((1, nq, H, d)).astype(np.float32)
+    k = rng.standard_normal((1, nk, d)).astype(np.float32)
+    w = rng.standard_normal((1, nq, H)).astype(np.float32)
+    inp = oracle_mod.Inputs(make(q, k, w, topk=keep, q_pos0=[300]))
+    for row in range(nq):
+        n = 300 + row + 1
+        seed = oracle_mod.dosa_seed(inp, row, shift, keep)
+        if n < keep:
+            assert seed == -np.inf
+            continue
+        I = np.sort(oracle_mod.score_pairs(inp, np.full(n, row), np.arange(n)))[::-1]
+        assert seed > -np.inf and I[keep - 1] >= seed
+    short = oracle_mod.Inputs(make(q, k, w, topk=keep, q_pos0=[100]))   # rows of 101..106 keys
+    assert all(oracle_mod.dosa_seed(short, r, shift, keep) == -np.inf for r in range(nq))
+    c = rng.standard_normal((nk >> shift, d)).astype(np.float32)
+    kc = np.repeat(c, 1 << shift, axis=0)[None, :nk]
+    kc = np.concatenate([kc, np.zeros((1, nk - kc.shape[1], d), np.float32)], axis=1)
+    inp = oracle_mod.Inputs(make(q, kc, w, topk=keep))
+    for row in range(nq):
+        n = nk - nq + row + 1
+        blk = oracle_mod.score_pairs(inp, np.full(n, row), np.arange(n))
+        per = [blk[a << shift] for a in range((n + (1 << shift) - 1) >> shift)]
+        cnt = [min(1 << shift, n - (a << shift)) for a in range(len(per))]
+        order = sorted(range(len(per)), key=lambda a: (-per[a], a))
+        got, want = 0, None
+        for a in order:
+            got += cnt[a]
+            want = per[a]
+            if got >= keep:
+                break
+        seed = oracle_mod.dosa_seed(inp, row, shift, keep)
+        assert abs(seed - want) <= 1e-12 * max(1.0, abs(want))
+
+
 def test_resmisa_routes_by_weight_magnitude(oracle_mod):
     """S_j = |w_j| max_b ReLU(U-_{b,j}): a head whose weight is negative but large in
     magnitude outranks a positive head with the same bound."""
