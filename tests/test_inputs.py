@@ -66,3 +66,26 @@ def test_clustered_keys_form_runs():
     clu = gen.normal_problem(5, 1, 8, 4096, 8, 128, 16, key_structure="clusters")
     assert abs(neighbour_cos(iid)) < 0.05
     assert neighbour_cos(clu) > 0.5
+
+
+def test_cluster_noise_and_constant_segments():
+    """The locality knobs: clustered keys with small noise stay within a narrow
+    box along each run, the default noise level reproduces the 0.5 recipe, and
+    segment keys without the tail token are exactly constant on each segment."""
+    a = gen.normal_problem(11, 1, 32, 4096, 8, 128, 16, key_structure="clusters",
+                           n_centres=4, mean_run=4096.0, noise=0.01)
+    k = gen.bf16_bits_to_f32(a.k)[0]
+    # adjacent keys inside one run differ by the noise only (a centre change is rare)
+    d = np.abs(np.diff(k, axis=0)).max(axis=1)
+    assert np.median(d) < 0.1
+    b = gen.normal_problem(12, 1, 32, 512, 8, 128, 16, key_structure="clusters")
+    c = gen.normal_problem(12, 1, 32, 512, 8, 128, 16, key_structure="clusters", noise=0.5)
+    assert np.array_equal(b.k, c.k)
+    s = gen.segment_integer_problem(13, 1, 16, 3000, 8, 128, 16, seg=1024, tail=False)
+    ks = gen.bf16_bits_to_f32(s.k)[0]
+    for lo in range(0, 3000, 1024):
+        seg = ks[lo:min(lo + 1024, 3000)]
+        assert np.all(seg == seg[0])
+    t = gen.segment_integer_problem(13, 1, 16, 3000, 8, 128, 16, seg=1024)
+    kt = gen.bf16_bits_to_f32(t.k)[0]
+    assert not np.all(kt[:1024] == kt[0])           # the tail token differs
